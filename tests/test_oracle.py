@@ -1,0 +1,349 @@
+"""Pins of the CPU oracle against facts fixed by the mathematics, not by the oracle itself.
+
+Each test checks the oracle against something independent of its own code:
+a textbook matrix, scipy's Hadamard routine, hand-derived closed forms
+(tests/golden/closed_forms.json), exact rational arithmetic, brute-force
+integer loops, or an invariant of the method (orthogonality, the rotation
+invariance X R (W R)^T = X W^T, equivariance, symmetry). A plausible slip in
+the oracle (a dropped 1/sqrt(g), a transposed Hadamard, a wrong block index, a
+wrong tie rule, a per-tensor instead of per-token scale, a missing bias or
+scale factor) fails at least one of them.
+"""
+
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle
+import synth
+
+
+def _hex(s: str) -> float:
+    return float.fromhex(s)
+
+
+# ---------------------------------------------------------------- rotation
+
+
+def test_hadamard_g2_is_textbook():
+    assert np.array_equal(oracle.hadamard(2), np.array([[1.0, 1.0], [1.0, -1.0]]))
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8, 16, 32, 64, 128, 256])
+def test_hadamard_matches_recursive_sylvester(g):
+    h = np.array([[1.0]])
+    while h.shape[0] < g:
+        h = np.block([[h, h], [h, -h]])
+    assert np.array_equal(oracle.hadamard(g), h)
+
+
+@pytest.mark.parametrize("g", [2, 4, 16, 128, 256])
+def test_hadamard_matches_scipy(g):
+    assert np.array_equal(oracle.hadamard(g), scipy.linalg.hadamard(g).astype(np.float64))
+
+
+@pytest.mark.parametrize("g", [128, 256])
+def test_rotation_is_orthonormal(g):
+    R = oracle.rotation_matrix(3 * g, g)
+    err = np.max(np.abs(R @ R.T - np.eye(3 * g)))
+    assert err < 1e-12  # required: 1e-6
+
+
+@pytest.mark.parametrize("K,g", [(256, 256), (512, 128), (768, 256), (16, 4)])
+def test_rotate_equals_block_diagonal_product(K, g):
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, K))
+    R = np.kron(np.eye(K // g), scipy.linalg.hadamard(g) / math.sqrt(g))
+    assert np.allclose(oracle.rotate(x, g), x @ R, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("g", [128, 256])
+def test_rotation_invariance(g):
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((9, 4 * g))
+    w = rng.standard_normal((13, 4 * g))
+    lhs = oracle.rotate(x, g) @ oracle.rotate(w, g).T
+    rhs = x @ w.T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-12 * np.max(np.abs(rhs))
+
+
+# ---------------------------------------------------------- quantisation
+
+
+def test_golden_quant_cases(golden):
+    for case in golden["quant_cases"]:
+        g = case["g"]
+        x = np.array([case["x"]], dtype=np.float64)
+        rot = oracle.rotate(x, g)
+        assert np.array_equal(rot[0], np.array(case["rotated"])), case["name"]
+        q, s = oracle.quant_act(x, g)
+        assert q.dtype == np.int8
+        assert q[0].tolist() == case["codes"], case["name"]
+        assert float(s[0]) == _hex(case["scale_hex"]), case["name"]
+
+
+def test_tie_rule_on_rotated_rows():
+    # already-rotated row with absmax 127 -> scale exactly 1
+    row = np.array([[127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 126.5]])
+    q, s = oracle.quantize_per_token(row)
+    assert float(s[0]) == 1.0
+    assert q[0].tolist() == [127, 2, 4, -2, -4, 0, 2, 0, 126]
+
+
+@pytest.mark.parametrize("g", [128, 256])
+@pytest.mark.parametrize("j,c", [(0, 1.0), (37, -3.0), (255, 0.125), (130, 1e-3)])
+def test_spike_row_closed_form(g, j, c):
+    K = 2 * g
+    x = np.zeros((1, K))
+    x[0, j] = c
+    q, s = oracle.quant_act(x, g)
+    blk = j // g
+    expect = np.zeros(K, dtype=np.int64)
+    expect[blk * g:(blk + 1) * g] = 127 * int(np.sign(c)) * scipy.linalg.hadamard(g)[j % g]
+    assert np.array_equal(q[0].astype(np.int64), expect)
+    s_closed = abs(c) / (math.sqrt(g) * 127.0)
+    assert abs(float(s[0]) - s_closed) <= 1.2e-7 * s_closed
+
+
+@pytest.mark.parametrize("g", [128, 256])
+@pytest.mark.parametrize("c", [1.0, -0.75, 40.0])
+def test_constant_group_closed_form(g, c):
+    K = 3 * g
+    x = np.zeros((1, K))
+    x[0, g:2 * g] = c
+    q, s = oracle.quant_act(x, g)
+    expect = np.zeros(K, dtype=np.int64)
+    expect[g] = 127 * int(np.sign(c))
+    assert np.array_equal(q[0].astype(np.int64), expect)
+    s_closed = abs(c) * math.sqrt(g) / 127.0
+    assert abs(float(s[0]) - s_closed) <= 1.2e-7 * s_closed
+
+
+def _tiny():
+    d = synth.make_workload("tiny")
+    return d, oracle.bf16_to_f64(d["x"]), oracle.bf16_to_f64(d["w"])
+
+
+def test_codes_in_range_and_every_row_hits_127():
+    d, x, _ = _tiny()
+    q, s = oracle.quant_act(x, d["workload"].g)
+    assert q.min() >= -127 and q.max() <= 127
+    assert np.all(np.max(np.abs(q.astype(np.int32)), axis=1) == 127)
+    assert np.all(s > 0)
+
+
+def test_scale_is_per_token():
+    # two tokens with very different ranges keep their own scales
+    _, x, _ = _tiny()
+    x2 = np.stack([x[0], 1000.0 * x[0], x[1]])
+    q, s = oracle.quant_act(x2, 256)
+    assert s[1] == pytest.approx(1000.0 * s[0], rel=1e-6)
+    assert np.array_equal(q[0], q[1])
+    # each token's codes do not depend on the other tokens in the batch
+    q1, s1 = oracle.quant_act(x2[2:], 256)
+    assert np.array_equal(q[2], q1[0]) and s[2] == s1[0]
+
+
+@pytest.mark.parametrize("k", [-6, -1, 3, 9])
+def test_scale_equivariance_power_of_two(k):
+    _, x, _ = _tiny()
+    q0, s0 = oracle.quant_act(x, 256)
+    q1, s1 = oracle.quant_act(x * 2.0**k, 256)
+    assert np.array_equal(q0, q1)
+    assert np.array_equal(s1, (s0.astype(np.float64) * 2.0**k).astype(np.float32))
+
+
+def test_odd_symmetry():
+    _, x, _ = _tiny()
+    q0, s0 = oracle.quant_act(x, 256)
+    q1, s1 = oracle.quant_act(-x, 256)
+    assert np.array_equal(q1, -q0)
+    assert np.array_equal(s0, s1)
+
+
+def test_tensorwise_weight_quant():
+    d, _, w = _tiny()
+    wq, s_w = oracle.prepare_weight(w, 256)
+    wr = scipy.linalg.hadamard(256) / 16.0
+    w_rot = w @ wr  # one group: K = g = 256
+    assert float(s_w) == float(np.float32(np.max(np.abs(w_rot)) / 127.0))
+    assert np.max(np.abs(wq.astype(np.int32))) == 127
+    # every code is within half a step of the scaled value (rounding to nearest)
+    assert np.max(np.abs(wq - w_rot / np.float64(s_w))) <= 0.5 + 1e-9
+
+
+# --------------------------------------------------------------- GEMM
+
+
+def test_gemm_bruteforce_loops_tiny():
+    rng = np.random.default_rng(5)
+    a = rng.integers(-127, 128, size=(7, 256), dtype=np.int64)
+    b = rng.integers(-127, 128, size=(9, 256), dtype=np.int64)
+    acc = oracle.gemm_s32(a.astype(np.int8), b.astype(np.int8))
+    for m in range(7):
+        for n in range(9):
+            tot = 0
+            for k in range(256):
+                tot += int(a[m, k]) * int(b[n, k])
+            assert acc[m, n] == tot
+
+
+def test_gemm_extreme_codes_exact():
+    # all +-127 over K = 12288: |acc| = 12288 * 127^2 = 198193152, exact in int32
+    K = 12288
+    a = np.full((2, K), 127, np.int8)
+    a[1] = -127
+    b = np.full((3, K), 127, np.int8)
+    b[2, ::2] = -127
+    acc = oracle.gemm_s32(a, b)
+    assert acc[0, 0] == K * 127 * 127
+    assert acc[1, 1] == -K * 127 * 127
+    assert acc[0, 2] == 0
+
+
+def test_gemm_matches_integer_matmul_on_tiny_workload():
+    d, x, w = _tiny()
+    xq, _ = oracle.quant_act(x, 256)
+    wq, _ = oracle.prepare_weight(w, 256)
+    ref = xq.astype(np.int64) @ wq.astype(np.int64).T
+    assert np.array_equal(oracle.gemm_s32(xq, wq).astype(np.int64), ref)
+
+
+# --------------------------------------------------- end to end / dequant
+
+
+def test_golden_linear_case(golden):
+    c = golden["linear_case"]
+    g = c["g"]
+    x = np.array(c["x"])
+    w = np.array(c["w"])
+    bias = np.array(c["bias"])
+    xq, s_x = oracle.quant_act(x, g)
+    wq, s_w = oracle.prepare_weight(w, g)
+    assert xq.tolist() == c["x_codes"]
+    assert [float(v) for v in s_x] == [_hex(h) for h in c["x_scale_hex"]]
+    assert wq.tolist() == c["w_codes"]
+    assert float(s_w) == _hex(c["w_scale_hex"])
+    acc = oracle.gemm_s32(xq, wq)
+    assert acc.tolist() == c["acc"]
+    y = oracle.linear(x, wq, s_w, g, bias)
+    sw = _hex(c["w_scale_hex"])
+    for m in range(2):
+        for n in range(2):
+            expect = c["acc"][m][n] * (_hex(c["x_scale_hex"][m]) * sw) + c["bias"][n]
+            assert y[m, n] == expect
+
+
+def _round_half_even(fr: Fraction) -> int:
+    return round(fr)  # Python rounds Fractions half to even
+
+
+def _exact_linear(x, w, bias, g):
+    """Exact rational ConvRot linear for g in {4, 16} (1/sqrt(g) rational)."""
+    h2 = [[1, 1], [1, -1]]
+    h = [[1]]
+    while len(h) < g:  # Kronecker square of the textbook 2x2
+        h = [[a * b for a in ra for b in rb] for ra in h for rb in h2]
+    inv_sqrt_g = Fraction(1, int(math.isqrt(g)))
+
+    def rot(row):
+        out = []
+        for b0 in range(0, len(row), g):
+            blk = row[b0:b0 + g]
+            for k in range(g):
+                out.append(sum(Fraction(blk[i]) * h[i][k] for i in range(g)) * inv_sqrt_g)
+        return out
+
+    def f32(fr: Fraction) -> Fraction:
+        return Fraction(float(np.float32(float(fr))))
+
+    def quant(rows, per_token):
+        rot_rows = [rot(r) for r in rows]
+        if per_token:
+            scales = [f32(max(abs(v) for v in r) / 127) for r in rot_rows]
+        else:
+            s = f32(max(abs(v) for r in rot_rows for v in r) / 127)
+            scales = [s] * len(rot_rows)
+        codes = [[0 if s == 0 else max(-127, min(127, _round_half_even(v / s))) for v in r]
+                 for r, s in zip(rot_rows, scales)]
+        return codes, scales
+
+    xc, sx = quant(x, True)
+    wc, sw = quant(w, False)
+    y = []
+    for m in range(len(x)):
+        row = []
+        for n in range(len(w)):
+            acc = sum(a * b for a, b in zip(xc[m], wc[n]))
+            row.append(acc * sx[m] * sw[0] + Fraction(bias[n]))
+        y.append(row)
+    return y
+
+
+@pytest.mark.parametrize("g", [4, 16])
+def test_linear_matches_exact_rational_pipeline(g):
+    rng = np.random.default_rng(21 + g)
+    K = 2 * g
+    x = rng.standard_normal((3, K)).astype(np.float32).astype(np.float64)
+    x[1, 3] *= 40.0  # an outlier channel
+    w = (rng.standard_normal((4, K)) * 0.02).astype(np.float32).astype(np.float64)
+    bias = (rng.standard_normal(4) * 0.01).astype(np.float32).astype(np.float64)
+    exact = _exact_linear(x.tolist(), w.tolist(), bias.tolist(), g)
+    wq, s_w = oracle.prepare_weight(w, g)
+    y = oracle.linear(x, wq, s_w, g, bias)
+    for m in range(3):
+        for n in range(4):
+            e = float(exact[m][n])
+            assert abs(y[m, n] - e) <= 1e-14 * max(1.0, abs(e))
+
+
+def test_zero_input_gives_zero_then_bias():
+    d, _, w = _tiny()
+    wq, s_w = oracle.prepare_weight(w, 256)
+    x = np.zeros((4, 256))
+    y = oracle.linear(x, wq, s_w, 256)
+    assert np.all(y == 0.0)
+    bias = oracle.bf16_to_f64(synth.f32_to_bf16_bits(np.linspace(-1, 1, 256).astype(np.float32)))
+    yb = oracle.linear(x, wq, s_w, 256, bias)
+    assert np.array_equal(yb, np.broadcast_to(bias, yb.shape))
+
+
+def test_oracle_is_deterministic():
+    d, x, w = _tiny()
+    wq, s_w = oracle.prepare_weight(w, 256)
+    y1 = oracle.linear(x, wq, s_w, 256)
+    y2 = oracle.linear(x, wq, s_w, 256)
+    assert np.array_equal(y1, y2)
+
+
+def test_rotation_lowers_error_on_outlier_tokens():
+    # the pages' reason for the rotation: without it one outlier channel sets
+    # the scale of the whole token (InvokeAI "int8 Compute", "What stays on the
+    # default path"). Same pipeline with g = 1 (R = I) as the control.
+    d, x, w = _tiny()
+    exact = x @ w.T
+    wq, s_w = oracle.prepare_weight(w, 256)
+    err_rot = oracle.nrmse(oracle.linear(x, wq, s_w, 256), exact)
+    wq1, s_w1 = oracle.prepare_weight(w, 1)
+    err_plain = oracle.nrmse(oracle.linear(x, wq1, s_w1, 1), exact)
+    assert err_rot < 0.5 * err_plain
+    assert err_rot < 2e-2
+
+
+def test_to_bf16_rne_ties():
+    # 1 + 2^-8 is halfway between bf16 neighbours 1 and 1 + 2^-7: ties to even (1.0)
+    vals = np.array([1.0, 1.0 + 2.0**-8, 1.0 + 3 * 2.0**-8, -2.5])
+    bits = oracle.to_bf16_rne(vals)
+    back = synth.bf16_bits_to_f32(bits).astype(np.float64).tolist()
+    assert back == [1.0, 1.0, 1.0 + 2 * 2.0**-7, -2.5]
+
+
+def test_nrmse_definition():
+    ref = np.array([3.0, 4.0])
+    assert oracle.nrmse(ref, ref) == 0.0
+    assert oracle.nrmse(np.array([3.0, 4.0 + 0.5]), ref) == pytest.approx(0.1)

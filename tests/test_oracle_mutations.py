@@ -1,0 +1,47 @@
+"""Plant plausible mistakes in a copy of the oracle and check that its pins catch each one.
+
+The copy lives in a temporary directory; the real oracle is never modified.
+"""
+
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "dropped_inv_sqrt_g": ("(blocks @ (hadamard(g) / np.sqrt(g)))", "(blocks @ hadamard(g))"),
+    "round_half_up": ("q = np.rint(xr / safe[..., None])", "q = np.floor(xr / safe[..., None] + 0.5)"),
+    "per_tensor_activation_scale": ("amax = np.max(np.abs(xr), axis=-1)",
+                                    "amax = np.max(np.abs(xr)) + 0 * np.max(np.abs(xr), axis=-1)"),
+    "bias_dropped": ("y = y + np.asarray(bias, np.float64)[None, :]", "y = y"),
+    "qmax_128": ("QMAX = 127", "QMAX = 128"),
+    "weight_scale_dropped": ("(np.asarray(s_x, np.float64)[:, None] * np.float64(s_w))",
+                             "(np.asarray(s_x, np.float64)[:, None])"),
+    "strided_instead_of_contiguous_groups": (
+        "blocks = x.reshape(x.shape[:-1] + (K // g, g))",
+        "blocks = x.reshape(x.shape[:-1] + (g, K // g)).swapaxes(-1, -2)"),
+    "weight_columns_reversed": ("np.asarray(wq, np.float64).T", "np.asarray(wq, np.float64)[:, ::-1].T"),
+    "token_scale_not_float32": ("s = (amax / QMAX).astype(np.float32)", "s = (amax / QMAX)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTATIONS[name]
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__"))
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), tmp_path / "pytest.ini")
+    path = tmp_path / "oracle" / "convrot_oracle.py"
+    src = path.read_text()
+    assert old in src, "mutation target not found: the oracle changed, update this table"
+    path.write_text(src.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle.py", "-q", "-x"],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
