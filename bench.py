@@ -1,0 +1,401 @@
+"""Benchmark of the INT8 ConvRot linear layer on B200: one JSON line on stdout.
+
+A step is one full ConvRot linear call (rotate + per-token quantise, int8 GEMM
+on tcgen05, dequantise + bias) through the C ABI on one batch of synthetic
+input already resident in HBM. The default workload is the DiT fused-QKV
+projection at 1024^2: M=4608 tokens (4096 image + 512 text), K=3072, N=9216,
+g=256, with bias.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Under torchrun (N > 1) every rank runs an independent replica of the same
+workload on its own GPU (the layer has no cross-GPU step); the value is the
+work of all ranks over the slowest rank's device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ConvRot linear TOPS (rotate+quant+i8 GEMM+dequant) and % of B200 INT8 peak"
+UNIT = "TOPS"
+N_SETS = 4  # rotating input/output sets per rank so that no step finds its data in L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="dit_qkv_1024")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w) -> dict:
+    return {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "g": w.g, "bias": w.bias,
+            "x": f"{w.x_dist}, {w.outlier_frac:g} outlier channels x{w.outlier_mult:g}",
+            "w_std": w.w_std,
+            "l2": f"{N_SETS} rotating input/output sets per GPU, each step on a set last used "
+                  f"{N_SETS - 1} steps earlier (>126 MB L2 in between)"}
+
+
+# --------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running (read only)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+
+def cpu_oracle_leg(d, target_s: float, gpu_rows=None):
+    """Time the oracle (as it stands) on a bounded row sample of the workload."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    w = d["workload"]
+    x = oracle.bf16_to_f64(d["x"])
+    wf = oracle.bf16_to_f64(d["w"])
+    b = None if d["bias"] is None else oracle.bf16_to_f64(d["bias"])
+    wq, sw = oracle.prepare_weight(wf, w.g)  # once per layer, untimed like the GPU side
+    rows = min(16, w.M)
+    t0 = time.perf_counter()
+    oracle.linear(x[:rows], wq, sw, w.g, b)
+    t1 = time.perf_counter() - t0
+    rows = int(max(1, min(w.M, rows * target_s / max(t1, 1e-3))))
+    if gpu_rows is not None:
+        rows = min(rows, gpu_rows.shape[0])
+    t0 = time.perf_counter()
+    y = oracle.linear(x[:rows], wq, sw, w.g, b)
+    dt = time.perf_counter() - t0
+    threads = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+    cores = int(max(threads)) if threads else os.cpu_count()
+    tops = 2.0 * rows * w.N * w.K / dt / 1e12
+    parity = None
+    if gpu_rows is not None:
+        parity = oracle.nrmse(gpu_rows[:rows], y)
+    return {"value": tops, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {rows} of {w.M} tokens of {w.name} through the float64 oracle "
+                      f"(rotate, quantise, GEMM, dequantise), weight prepared beforehand; {dt:.2f} s"}, parity
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, rank 0 only, bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+
+    d = synth.make_workload(args.config)
+    w = d["workload"]
+    import oracle
+
+    x = oracle.bf16_to_f64(d["x"])
+    b = None if d["bias"] is None else oracle.bf16_to_f64(d["bias"])
+    wq, sw = oracle.prepare_weight(oracle.bf16_to_f64(d["w"]), w.g)
+    total_budget = 150.0  # seconds for warm-up + timed steps
+    rows = min(8, w.M)
+    t0 = time.perf_counter()
+    oracle.linear(x[:rows], wq, sw, w.g, b)
+    t_one = max(time.perf_counter() - t0, 1e-3)
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(w.M, rows * per_step / t_one)))
+    for i in range(args.warmup):
+        oracle.linear(x[:rows], wq, sw, w.g, b)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.linear(x[:rows], wq, sw, w.g, b)
+    dt = time.perf_counter() - t0
+    from threadpoolctl import threadpool_info
+
+    threads = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+    cores = int(max(threads)) if threads else os.cpu_count()
+    value = 2.0 * rows * w.N * w.K * args.steps / dt / 1e12
+    sample = f"first {rows} of {w.M} tokens of {w.name} per step through the float64 CPU oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import w8a8_rotated_int8_token_b200 as cr
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the ConvRot path has no CPU implementation)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    d = synth.make_workload(args.config)
+    w = d["workload"]
+    M, K, N, g = w.M, w.K, w.N, w.g
+    L = cr.lib()
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    W = to_dev(d["w"])
+    Wq0, sw = cr.convrot_prepare_weight(W, g)
+    del W
+    bias = None if d["bias"] is None else to_dev(d["bias"])
+    X0 = to_dev(d["x"])
+    ws_bytes = cr.convrot_linear_workspace_bytes(M, N, K, g)
+    sets = []
+    for i in range(N_SETS):
+        sets.append({
+            "X": X0.clone(), "Wq": Wq0.clone(),
+            "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+            "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=dev),
+        })
+    del X0
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    b_ptr = None if bias is None else bias.data_ptr()
+    sw_ptr = sw.data_ptr()
+
+    def step(i):
+        s = sets[i % N_SETS]
+        st = L.convrot_linear(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw_ptr, N, b_ptr, s["Y"].data_ptr(),
+                              s["ws"].data_ptr(), ws_bytes, sp)
+        if st != 0:
+            raise cr.ConvRotError(st, "convrot_linear")
+
+    # ---- device-resident timed region
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    for s in sets:
+        st = cr.convrot_read_device_status(s["ws"])
+        if st != 0:
+            raise cr.ConvRotError(st, "device status after the timed region")
+    ops = 2.0 * M * N * K
+    value = ops * args.steps * world / (t_ms * 1e-3) / 1e12
+
+    # ---- per-kernel breakdown: the same two kernels through the split entry points
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    gws = torch.empty((L.convrot_gemm_workspace_bytes(),), dtype=torch.uint8, device=dev)
+    xsc = [torch.empty((M,), dtype=torch.float32, device=dev) for _ in range(N_SETS)]
+    xq = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(N_SETS)]
+    for i in range(args.warmup):
+        s = sets[i % N_SETS]
+        L.convrot_quant_act(s["X"].data_ptr(), M, K, g, xq[i % N_SETS].data_ptr(), xsc[i % N_SETS].data_ptr(), sp)
+        L.convrot_gemm_dequant(xq[i % N_SETS].data_ptr(), xsc[i % N_SETS].data_ptr(), s["Wq"].data_ptr(), sw_ptr,
+                               M, N, K, b_ptr, s["Y"].data_ptr(), gws.data_ptr(), gws.numel(), sp)
+    torch.cuda.synchronize(dev)
+    barrier()
+    for i in range(args.steps):
+        s = sets[i % N_SETS]
+        e = ev[i]
+        e[0].record(stream)
+        L.convrot_quant_act(s["X"].data_ptr(), M, K, g, xq[i % N_SETS].data_ptr(), xsc[i % N_SETS].data_ptr(), sp)
+        e[1].record(stream)
+        L.convrot_gemm_dequant(xq[i % N_SETS].data_ptr(), xsc[i % N_SETS].data_ptr(), s["Wq"].data_ptr(), sw_ptr,
+                               M, N, K, b_ptr, s["Y"].data_ptr(), gws.data_ptr(), gws.numel(), sp)
+        e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_q = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    t_g = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    del xq, xsc
+
+    peaks, peak_src = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    gemm_tops = ops / (t_g * 1e-3) / 1e12
+    q_bytes = 3.0 * M * K + 4.0 * M
+    q_gbs = q_bytes / (t_q * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        xh = [torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+              for _ in range(2)]
+        yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        e2e_steps = max(1, min(args.steps, 200))
+
+        def e2e_step(i):
+            s = sets[i % N_SETS]
+            s["X"].copy_(xh[i % 2], non_blocking=True)
+            cr.convrot_linear(s["X"], s["Wq"], sw, g, bias, Y=s["Y"], ws=s["ws"])
+            yh[i % 2].copy_(s["Y"], non_blocking=True)
+
+        for i in range(min(args.warmup, 5)):
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ev0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        t_e2e = max_over_ranks(ev0.elapsed_time(ev1))
+        e2e = {"value": ops * e2e_steps * world / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(yh[0].numel() * 2),
+               "steps": e2e_steps, "ms_per_step": t_e2e / e2e_steps}
+
+    cpu = None
+    parity = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        y_rows = sets[(args.steps - 1) % N_SETS]["Y"][:4096].float().cpu().numpy().astype(np.float64)
+        cpu, parity = cpu_oracle_leg(d, args.cpu_seconds, y_rows)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    gemm_frac = gemm_tops / int8_peak
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(w),
+        "pct_int8_peak": 100.0 * value / world / int8_peak,
+        "roofline": {"bound": "tensor", "kernel": "gemm_i8_kernel (tcgen05 kind::i8 + dequant epilogue)",
+                     "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS", "frac": gemm_frac,
+                     "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
+                                    "(nominal int8:bf16 dense ratio)"},
+        "kernels": {
+            "rotate_quant_kernel": {"us": t_q * 1e3, "bound": "hbm", "achieved": q_gbs, "unit": "GB/s",
+                                    "peak": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
+                                    "algorithmic_bytes": q_bytes},
+            "gemm_i8_kernel": {"us": t_g * 1e3, "bound": "tensor", "achieved": gemm_tops, "unit": "TOPS",
+                               "peak": int8_peak, "frac": gemm_frac, "ops": ops},
+        },
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if parity is not None:
+        out["parity_nrmse_vs_oracle_sample"] = parity
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

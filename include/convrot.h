@@ -1,0 +1,178 @@
+/*
+ * convrot.h -- C ABI of libconvrot, the INT8 ConvRot linear layer for NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (restated from the pages that describe the method):
+ *   - The weight is stored as int8 with one scale for the whole tensor
+ *     ("int8_tensorwise"; InvokeAI "int8 Compute" page, opening section).
+ *   - Each call rotates its input, quantises it to int8 with one scale per
+ *     token, and multiplies int8 by int8 on the tensor cores (same page,
+ *     second paragraph).
+ *   - The rotation works on groups of input channels, 256 wide in every
+ *     published build (same page, "What stays on the default path"); it is a
+ *     group-wise rotation slid block by block along the channel axis, so that
+ *     an outlier channel is spread over its group ("Explanation of INT8
+ *     ConvRot", section "What is INT8 ConvRot?").
+ *
+ * Readings this library fixes where the pages are silent:
+ *   R = blockdiag(H_g/sqrt(g), ...), H_g the Sylvester Walsh-Hadamard matrix
+ *   (H[i][j] = (-1)^popcount(i & j)), g in {128, 256}, applied to both X and W
+ *   so that X R (W R)^T = X W^T. Symmetric quantisation, codes in [-127, 127],
+ *   round to nearest with ties to even. Token scale s_x[m] = absmax_k |(X R)[m,k]| / 127
+ *   in float32 (0 for an all-zero token, whose codes are then 0). Output
+ *   Y[m,n] = bf16_rne(float(acc[m,n]) * (s_x[m] * s_w) + bias[n]).
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major with K contiguous: X [M,K], W/Wq [N,K], Y [M,N].
+ *     X, W, bias and Y are bf16 (IEEE bfloat16 bit patterns, 2 bytes each).
+ *   - Every data pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned (workspaces: 256-byte aligned). The library never allocates,
+ *     never frees and never synchronises, except where an entry point says so.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) on the calling thread's current device.
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns an error code and enqueues nothing.
+ *   - A launch failure returns CONVROT_ERR_CUDA.
+ *   - Waits inside the GEMM kernel are bounded (about 2 s). If one runs out,
+ *     the kernel records CONVROT_ERR_DEVICE_TIMEOUT in the workspace status
+ *     word and returns without faulting; convrot_read_device_status reports it.
+ *   - Entry points hold no state between calls and are safe to call from
+ *     several host threads on different streams with separate workspaces.
+ */
+#ifndef CONVROT_H
+#define CONVROT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CONVROT_API __attribute__((visibility("default")))
+#else
+#define CONVROT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* convrot_stream_t;
+
+typedef enum {
+  CONVROT_OK = 0,
+  CONVROT_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer     */
+  CONVROT_ERR_UNSUPPORTED = 2,   /* g not in {128,256}, K above the kernel limit    */
+  CONVROT_ERR_WORKSPACE = 3,     /* workspace null, misaligned or too small         */
+  CONVROT_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed             */
+  CONVROT_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait ran out (see above)  */
+} convrot_status;
+
+/* Largest K the rotation/quantisation kernels take (one CTA holds a token). */
+#define CONVROT_MAX_K 32768
+
+/* Version of this ABI; bumped when a signature or a layout changes. */
+CONVROT_API int convrot_abi_version(void);
+
+/* Static English description of a status code. Never NULL. */
+CONVROT_API const char* convrot_status_string(int status);
+
+/*
+ * convrot_prepare_weight -- rotate and quantise a bf16 weight once per layer.
+ *   Wq = clamp(rne((W R) / s_w), -127, 127),  s_w = max |W R| / 127 (float32).
+ * The stored weight of a ConvRot layer is int8 with one tensorwise scale,
+ * pre-rotated (InvokeAI "int8 Compute", opening section).
+ *   W        [N,K] bf16, device.           N >= 1; K % g == 0; K <= CONVROT_MAX_K.
+ *   g        group size, 128 or 256.
+ *   Wq       [N,K] int8 out, device.
+ *   w_scale  1 float out, device.
+ *   ws       device workspace of ws_bytes >= convrot_prepare_weight_workspace_bytes();
+ *            overwritten; only needed until the enqueued work has run.
+ * Enqueues three operations (a 4-byte memset and two kernels) on `stream`.
+ */
+CONVROT_API size_t convrot_prepare_weight_workspace_bytes(void);
+CONVROT_API convrot_status convrot_prepare_weight(const void* W, int64_t N, int64_t K, int g,
+                                      int8_t* Wq, float* w_scale,
+                                      void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * convrot_quant_act -- the fused activation pass: per token, rotate each
+ * length-g group (fast Walsh-Hadamard transform in float32, never stored),
+ * take the token's absmax, and write int8 codes and the float32 scale
+ * (InvokeAI "int8 Compute", second paragraph: rotate, then quantise per token).
+ *   X        [M,K] bf16, device.            M >= 1; K % g == 0; K <= CONVROT_MAX_K.
+ *   Xq       [M,K] int8 out, device.
+ *   x_scale  [M] float out, device.
+ * One kernel launch.
+ */
+CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g,
+                                 int8_t* Xq, float* x_scale, convrot_stream_t stream);
+
+/*
+ * convrot_linear -- one ConvRot linear call:
+ *   Y = bf16_rne( (Xq Wq^T) * (s_x[m] * s_w) + bias[n] ),  (Xq, s_x) = quant_act(X).
+ * The int8 x int8 product accumulates exactly in int32 on the tcgen05 tensor
+ * cores (InvokeAI "int8 Compute", second paragraph); dequantisation and the
+ * bias are fused into the GEMM epilogue.
+ *   X        [M,K] bf16, device.   M >= 1, N >= 1, K % g == 0, K <= CONVROT_MAX_K,
+ *                                   N % 8 == 0.
+ *   Wq       [N,K] int8, device (from convrot_prepare_weight with the same g).
+ *   w_scale  1 float, device.
+ *   bias     [N] bf16, device, or NULL for none.
+ *   Y        [M,N] bf16 out, device. Must not overlap any input.
+ *   ws       device workspace, 256-byte aligned, ws_bytes >=
+ *            convrot_linear_workspace_bytes(M, N, K, g). It holds the status
+ *            word, the token scales and the int8 activation codes of this call;
+ *            calls that may run at the same time need separate workspaces.
+ * Enqueues two kernels (rotate+quantise, then GEMM+epilogue).
+ */
+CONVROT_API size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+CONVROT_API convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g,
+                              const int8_t* Wq, const float* w_scale, int64_t N,
+                              const void* bias, void* Y,
+                              void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * convrot_gemm_dequant -- the GEMM + epilogue half of convrot_linear, on codes
+ * that are already quantised:  Y = bf16_rne(float(Xq Wq^T) * (x_scale[m] * s_w) + bias[n]).
+ *   Xq [M,K] int8, x_scale [M] float, Wq [N,K] int8, w_scale 1 float, bias [N]
+ *   bf16 or NULL, Y [M,N] bf16 out -- all device. K % 16 == 0, N % 8 == 0.
+ *   ws: at least convrot_gemm_workspace_bytes() bytes (the status word).
+ */
+CONVROT_API size_t convrot_gemm_workspace_bytes(void);
+CONVROT_API convrot_status convrot_gemm_dequant(const int8_t* Xq, const float* x_scale,
+                                    const int8_t* Wq, const float* w_scale,
+                                    int64_t M, int64_t N, int64_t K,
+                                    const void* bias, void* Y,
+                                    void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * convrot_gemm_s32 -- the raw int32 accumulators acc = Xq Wq^T of the same
+ * tcgen05 GEMM (for exactness tests): acc [M,N] int32 out, device.
+ *   K % 16 == 0, N % 4 == 0. ws as for convrot_gemm_dequant.
+ */
+CONVROT_API convrot_status convrot_gemm_s32(const int8_t* Xq, const int8_t* Wq,
+                                int64_t M, int64_t N, int64_t K, int32_t* acc,
+                                void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * convrot_read_device_status -- copy the status word of a workspace used by
+ * convrot_linear / convrot_gemm_* back to the host and return it
+ * (CONVROT_OK, or CONVROT_ERR_DEVICE_TIMEOUT if a bounded wait ran out).
+ * SYNCHRONISES `stream`. The word is reset at the start of every call that
+ * uses the workspace.
+ */
+CONVROT_API convrot_status convrot_read_device_status(const void* ws, convrot_stream_t stream);
+
+/*
+ * convrot_test_wait_timeout -- exercises the bounded device wait: launches one
+ * CTA that waits on a barrier nothing will complete, for at most timeout_ns
+ * nanoseconds (1e3 .. 1e9), then records CONVROT_ERR_DEVICE_TIMEOUT in the
+ * status word of `ws` (>= convrot_gemm_workspace_bytes()) and returns. For tests.
+ */
+CONVROT_API convrot_status convrot_test_wait_timeout(void* ws, size_t ws_bytes, int64_t timeout_ns,
+                                         convrot_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H */

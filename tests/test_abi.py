@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects bad arguments before touching the GPU."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w8a8_rotated_int8_token_b200 import build, _lib
+
+    build.build()
+    return _lib.load()
+
+
+def _declared_entry_points():
+    with open(os.path.join(ROOT, "include", "convrot.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"CONVROT_API\s+[\w\s\*]+?\b(convrot_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_entry_points()
+    for required in ("convrot_prepare_weight", "convrot_quant_act", "convrot_linear",
+                     "convrot_linear_workspace_bytes", "convrot_gemm_s32", "convrot_read_device_status",
+                     "convrot_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from w8a8_rotated_int8_token_b200 import _lib
+
+    for name in _declared_entry_points():
+        assert hasattr(L, name), name
+        assert name in _lib.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_library_exports_nothing_else():
+    import subprocess
+
+    from w8a8_rotated_int8_token_b200 import _lib
+
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert exported == set(_declared_entry_points())
+
+
+def test_status_strings_and_version(L):
+    assert L.convrot_abi_version() == 1
+    for code in range(6):
+        s = L.convrot_status_string(code)
+        assert s and s != b"unknown status"
+    assert L.convrot_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(L):
+    # [status 256 B | scales 4M, 1 KB aligned | codes M*K], 256-aligned
+    M, N, K = 4608, 9216, 3072
+    need = L.convrot_linear_workspace_bytes(M, N, K, 256)
+    scale_end = 256 + 4 * M
+    codes_off = (scale_end + 1023) // 1024 * 1024
+    assert need == (codes_off + M * K + 255) // 256 * 256
+    assert L.convrot_linear_workspace_bytes(M, N, K, 64) == 0       # unsupported g
+    assert L.convrot_linear_workspace_bytes(M, N, 3000, 256) == 0   # K % g != 0
+    assert L.convrot_linear_workspace_bytes(M, 9212, K, 256) == 0   # N % 8 != 0
+    assert L.convrot_linear_workspace_bytes(0, N, K, 256) == 0
+    assert L.convrot_gemm_workspace_bytes() == 256
+    assert L.convrot_prepare_weight_workspace_bytes() >= 4
+
+
+FAKE = 0x10000  # 16-byte aligned non-null value; never dereferenced: every call below fails validation
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes)
+    ((FAKE, 64, 256, 64, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 2),      # g unsupported
+    ((FAKE, 64, 300, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),     # K % g
+    ((FAKE, 64, 65536, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 40), 2),   # K above limit
+    ((FAKE, 0, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),      # M = 0
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 0, None, FAKE, FAKE, 1 << 30), 1),       # N = 0
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 260, None, FAKE, FAKE, 1 << 30), 1),     # N % 8
+    ((None, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),     # null X
+    ((FAKE, 64, 256, 256, None, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),     # null Wq
+    ((FAKE, 64, 256, 256, FAKE, None, 256, None, FAKE, FAKE, 1 << 30), 1),     # null w_scale
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 256, None, None, FAKE, 1 << 30), 1),     # null Y
+    ((FAKE + 2, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),  # misaligned X
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 256, FAKE + 8, FAKE, FAKE, 1 << 30), 1),  # misaligned bias
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, None, 1 << 30), 3),     # null workspace
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE + 16, 1 << 30), 3),  # misaligned workspace
+    ((FAKE, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 100), 3),         # workspace too small
+])
+def test_linear_rejects_bad_arguments_on_host(L, args, expect):
+    assert L.convrot_linear(*args, None) == expect
+
+
+def test_other_entry_points_reject_bad_arguments_on_host(L):
+    assert L.convrot_quant_act(FAKE, 8, 256, 512, FAKE, FAKE, None) == 2
+    assert L.convrot_quant_act(None, 8, 256, 256, FAKE, FAKE, None) == 1
+    assert L.convrot_quant_act(FAKE, 8, 256, 256, FAKE, FAKE + 2, None) == 1
+    assert L.convrot_prepare_weight(FAKE, 8, 384, 256, FAKE, FAKE, FAKE, 256, None) == 1
+    assert L.convrot_prepare_weight(FAKE, 8, 256, 256, FAKE, FAKE, FAKE, 2, None) == 3
+    assert L.convrot_gemm_s32(FAKE, FAKE, 8, 6, 256, FAKE, FAKE, 256, None) == 1    # N % 4
+    assert L.convrot_gemm_s32(FAKE, FAKE, 8, 8, 24, FAKE, FAKE, 256, None) == 1     # K % 16
+    assert L.convrot_gemm_s32(FAKE, FAKE, 8, 8, 256, FAKE, FAKE, 16, None) == 3     # workspace
+    assert L.convrot_gemm_dequant(FAKE, None, FAKE, FAKE, 8, 8, 256, None, FAKE, FAKE, 256, None) == 1
+    assert L.convrot_read_device_status(None, None) == 3
+    assert L.convrot_test_wait_timeout(FAKE, 256, 10, None) == 1
+    assert L.convrot_test_wait_timeout(FAKE, 256, 10**10, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from w8a8_rotated_int8_token_b200 import _lib
+
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib.load()
+
+
+def test_ctypes_signatures_match_header_arity():
+    from w8a8_rotated_int8_token_b200 import _lib
+
+    with open(os.path.join(ROOT, "include", "convrot.h")) as f:
+        src = f.read()
+    for name, (_, args) in _lib.SIGNATURES.items():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", src)
+        assert m, name
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert len(params) == len(args), name
+    assert ctypes.sizeof(ctypes.c_size_t) == 8

@@ -1,0 +1,315 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200.
+
+Small cases are compared element by element; the full-size workloads run in
+the same launch configuration the benchmark times and are compared on sampled
+token rows (rows are independent in every step of the method, so the oracle
+run on a subset of rows gives exactly those rows' results).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import (NRMSE_TOL, bf16_tensor_to_f64, check_codes, nrmse, to_torch_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cr():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import w8a8_rotated_int8_token_b200 as cr
+
+    cr.lib()  # loads libconvrot.so or raises
+    return cr
+
+
+def _rows_sample(M: int, n: int = 512, seed: int = 0) -> np.ndarray:
+    if M <= n:
+        return np.arange(M)
+    rng = np.random.default_rng(seed)
+    head = np.arange(128)
+    tail = np.arange(M - 128, M)
+    mid = rng.choice(np.arange(128, M - 128), n - 256, replace=False)
+    return np.unique(np.concatenate([head, mid, tail]))
+
+
+# ------------------------------------------------------------ rotate + quant
+
+
+def _quant_case(cr, xbits: np.ndarray, g: int):
+    import torch
+
+    X = to_torch_bf16(xbits)
+    Xq, s = cr.convrot_quant_act(X, g)
+    torch.cuda.synchronize()
+    x = oracle.bf16_to_f64(xbits)
+    xr = oracle.rotate(x, g)
+    q_ref, s_ref = oracle.quantize_per_token(xr)
+    return check_codes(Xq.cpu().numpy(), s.cpu().numpy(), xr, q_ref, s_ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "dit_qkv_1024", "textenc_m512"])
+def test_quant_act_matches_oracle_on_workloads(cr, name):
+    d = synth.make_workload(name)
+    _quant_case(cr, d["x"], d["workload"].g)
+
+
+@pytest.mark.parametrize("M,K,g", [(1, 256, 256), (3, 128, 128), (131, 384, 128), (130, 768, 256),
+                                   (300, 12288, 256), (7, 32768, 256), (5, 32768, 128)])
+def test_quant_act_ragged_and_extreme_shapes(cr, M, K, g):
+    rng = np.random.default_rng(M * 7919 + K + g)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, rng.choice(K, max(1, K // 100), replace=False)] *= 50.0
+    _quant_case(cr, synth.f32_to_bf16_bits(x), g)
+
+
+@pytest.mark.parametrize("g", [128, 256])
+def test_quant_act_special_rows(cr, g):
+    K = 4 * g
+    rng = np.random.default_rng(3)
+    rows = [np.zeros(K, np.float32)]                        # zero token: scale 0, codes 0
+    spike = np.zeros(K, np.float32); spike[g + 37] = -3.0   # one channel: a full +-127 group
+    rows.append(spike)
+    const = np.zeros(K, np.float32); const[2 * g:3 * g] = 0.75  # constant group: (127, 0, ...)
+    rows.append(const)
+    rows.append((rng.standard_normal(K) * 1e-34).astype(np.float32))  # tiny token (scale near 2^-120)
+    rows.append((rng.standard_normal(K) * 1e-30).astype(np.float32))  # tiny token
+    rows.append((rng.standard_normal(K) * 1e33).astype(np.float32))   # huge token
+    rows.append(np.full(K, -2.0, np.float32))
+    xbits = synth.f32_to_bf16_bits(np.stack(rows))
+    _quant_case(cr, xbits, g)
+    import torch
+
+    Xq, s = cr.convrot_quant_act(to_torch_bf16(xbits), g)
+    Xq = Xq.cpu().numpy()
+    assert float(s[0]) == 0.0 and not Xq[0].any()
+    h = oracle.hadamard(g)
+    assert np.array_equal(Xq[1, g:2 * g].astype(np.int32), -127 * h[37].astype(np.int32))
+    assert not Xq[1, :g].any() and not Xq[1, 2 * g:].any()
+    expect = np.zeros(K, np.int8); expect[2 * g] = 127
+    assert np.array_equal(Xq[2], expect)
+    torch.cuda.synchronize()
+
+
+def test_quant_act_scale_equivariance_and_symmetry(cr):
+    import torch
+
+    d = synth.make_workload("tiny")
+    x = synth.bf16_bits_to_f32(d["x"])
+    q0, s0 = cr.convrot_quant_act(to_torch_bf16(d["x"]), 256)
+    q1, s1 = cr.convrot_quant_act(to_torch_bf16(synth.f32_to_bf16_bits(x * 8.0)), 256)
+    q2, s2 = cr.convrot_quant_act(to_torch_bf16(synth.f32_to_bf16_bits(-x)), 256)
+    torch.cuda.synchronize()
+    assert torch.equal(q0, q1) and torch.equal(s1, s0 * 8.0)
+    assert torch.equal(q2, -q0) and torch.equal(s2, s0)
+
+
+# -------------------------------------------------------------- weights
+
+
+@pytest.mark.parametrize("name", ["tiny", "dit_qkv_1024", "textenc_m16"])
+def test_prepare_weight_matches_oracle(cr, name):
+    import torch
+
+    d = synth.make_workload(name)
+    g = d["workload"].g
+    W = to_torch_bf16(d["w"])
+    Wq, sw = cr.convrot_prepare_weight(W, g)
+    torch.cuda.synchronize()
+    w = oracle.bf16_to_f64(d["w"])
+    wr = oracle.rotate(w, g)
+    q_ref, s_ref = oracle.quantize_tensorwise(wr)
+    check_codes(Wq.cpu().numpy(), sw.cpu().numpy(), wr, q_ref, np.array([s_ref]), per_token=False)
+    assert int(np.abs(Wq.cpu().numpy().astype(np.int32)).max()) == 127
+
+
+# ---------------------------------------------------------- int32 GEMM
+
+
+def _gemm_exact(cr, xq: np.ndarray, wq: np.ndarray, rows=None):
+    import torch
+
+    acc = cr.convrot_gemm_s32(torch.from_numpy(xq).cuda(), torch.from_numpy(wq).cuda())
+    torch.cuda.synchronize()
+    acc = acc.cpu().numpy()
+    if rows is None:
+        ref = oracle.gemm_s32(xq, wq)
+        assert np.array_equal(acc, ref)
+    else:
+        ref = oracle.gemm_s32(xq[rows], wq)
+        assert np.array_equal(acc[rows], ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 256, 256), (1, 8, 16), (1, 256, 128), (130, 264, 272), (257, 520, 4096),
+                                   (128, 1024, 12288), (513, 12288, 128)])
+def test_gemm_s32_bit_exact(cr, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    xq = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    wq = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    _gemm_exact(cr, xq, wq)
+
+
+def test_gemm_s32_extreme_accumulators(cr):
+    K = 12288  # |acc| up to K * 127^2 = 198,193,152
+    xq = np.full((130, K), 127, np.int8)
+    xq[1::2] = -127
+    wq = np.full((264, K), 127, np.int8)
+    wq[::3] = -127
+    wq[5, ::2] = -127
+    _gemm_exact(cr, xq, wq)
+
+
+def test_gemm_s32_full_size_sampled(cr):
+    d = synth.make_workload("dit_qkv_1024")
+    g = d["workload"].g
+    xq, _ = oracle.quant_act(oracle.bf16_to_f64(d["x"]), g)
+    wq, _ = oracle.prepare_weight(oracle.bf16_to_f64(d["w"]), g)
+    _gemm_exact(cr, xq, wq, rows=_rows_sample(xq.shape[0]))
+
+
+def test_gemm_dequant_on_identical_codes(cr):
+    import torch
+
+    d = synth.make_workload("dit_qkv_1024")
+    g = d["workload"].g
+    x = oracle.bf16_to_f64(d["x"])
+    xq, sx = oracle.quant_act(x, g)
+    wq, sw = oracle.prepare_weight(oracle.bf16_to_f64(d["w"]), g)
+    bias = d["bias"]
+    Y = cr.convrot_gemm_dequant(torch.from_numpy(xq).cuda(), torch.from_numpy(sx).cuda(),
+                                torch.from_numpy(wq).cuda(), torch.tensor([sw], dtype=torch.float32).cuda(),
+                                to_torch_bf16(bias))
+    torch.cuda.synchronize()
+    rows = _rows_sample(xq.shape[0])
+    y = bf16_tensor_to_f64(Y)[rows]
+    ref = oracle.dequant(oracle.gemm_s32(xq[rows], wq), sx[rows], sw, oracle.bf16_to_f64(bias))
+    # same codes, so only float32 dequant rounding and the bf16 rounding remain
+    err = np.abs(y - ref)
+    assert np.all(err <= 2.0**-8 * np.abs(ref) + 1e-6 * np.abs(ref).max())
+    assert nrmse(y, ref) < 2e-3
+
+
+# ------------------------------------------------------------ end to end
+
+
+def _linear_case(cr, d, rows=None):
+    import torch
+
+    w = d["workload"]
+    g = w.g
+    W = to_torch_bf16(d["w"])
+    Wq, sw = cr.convrot_prepare_weight(W, g)
+    bias = None if d["bias"] is None else to_torch_bf16(d["bias"])
+    X = to_torch_bf16(d["x"])
+    M, K = d["x"].shape
+    N = d["w"].shape[0]
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, N, K, g), dtype=torch.uint8, device="cuda")
+    Y = cr.convrot_linear(X, Wq, sw, g, bias, ws=ws)
+    status = cr.convrot_read_device_status(ws)
+    assert status == 0
+    if rows is None:
+        rows = np.arange(M)
+    xs = oracle.bf16_to_f64(d["x"][rows])
+    wq_ref, sw_ref = oracle.prepare_weight(oracle.bf16_to_f64(d["w"]), g)
+    b = None if d["bias"] is None else oracle.bf16_to_f64(d["bias"])
+    ref = oracle.linear(xs, wq_ref, sw_ref, g, b)
+    y = bf16_tensor_to_f64(Y)[rows]
+    err = nrmse(y, ref)
+    assert err <= NRMSE_TOL, f"{w.name}: NRMSE {err}"
+    # the codes and token scales this call left in its workspace
+    wsn = ws.cpu().numpy()
+    codes_off = (256 + 4 * M + 1023) // 1024 * 1024
+    sx_gpu = wsn[256:256 + 4 * M].view(np.float32)[rows]
+    xq_gpu = wsn[codes_off:codes_off + M * K].view(np.int8).reshape(M, K)[rows]
+    xr = oracle.rotate(xs, g)
+    q_ref, s_ref = oracle.quantize_per_token(xr)
+    check_codes(xq_gpu, sx_gpu, xr, q_ref, s_ref)
+    return Y, err
+
+
+@pytest.mark.parametrize("name", ["tiny", "dit_qkv_1024", "dit_mlp_up_1024", "textenc_m1", "textenc_m16",
+                                  "textenc_m128", "textenc_m512"])
+def test_linear_matches_oracle(cr, name):
+    d = synth.make_workload(name)
+    _linear_case(cr, d, rows=_rows_sample(d["x"].shape[0]))
+
+
+def test_linear_matches_oracle_mlp_2048(cr):
+    d = synth.make_workload("dit_mlp_2048")
+    _linear_case(cr, d, rows=_rows_sample(d["x"].shape[0], 384))
+
+
+def test_linear_matches_oracle_mlp_down_1024(cr):
+    up = synth.make_workload("dit_mlp_up_1024")
+    g = up["workload"].g
+    wq, sw = oracle.prepare_weight(oracle.bf16_to_f64(up["w"]), g)
+    y_up = oracle.linear(oracle.bf16_to_f64(up["x"]), wq, sw, g)  # the oracle's up output feeds both sides
+    dn = synth.make_workload("dit_mlp_down_1024", x_up_output=y_up)
+    _linear_case(cr, dn, rows=_rows_sample(dn["x"].shape[0], 256))
+
+
+def test_linear_is_deterministic(cr):
+    import torch
+
+    d = synth.make_workload("dit_qkv_1024")
+    Y1, _ = _linear_case(cr, d, rows=np.arange(64))
+    Y2, _ = _linear_case(cr, d, rows=np.arange(64))
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_zero_input_gives_zero_output_and_bias(cr):
+    import torch
+
+    d = synth.make_workload("dit_qkv_1024")
+    W = to_torch_bf16(d["w"])
+    Wq, sw = cr.convrot_prepare_weight(W, 256)
+    X = torch.zeros((130, 3072), dtype=torch.bfloat16, device="cuda")
+    Y = cr.convrot_linear(X, Wq, sw, 256)
+    assert not Y.view(torch.int16).any()
+    b = to_torch_bf16(d["bias"])
+    Yb = cr.convrot_linear(X, Wq, sw, 256, b)
+    torch.cuda.synchronize()
+    assert torch.equal(Yb.view(torch.int16), b.view(torch.int16).expand(130, -1))
+
+
+@pytest.mark.parametrize("M,N,K", [(130, 264, 256), (1, 8, 128), (257, 1032, 384)])
+def test_linear_writes_only_its_output(cr, M, N, K):
+    import torch
+
+    g = 128 if K % 256 else 256
+    rng = np.random.default_rng(M + N)
+    x = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    w = synth.f32_to_bf16_bits((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+    Wq, sw = cr.convrot_prepare_weight(to_torch_bf16(w), g)
+    guard = 4096
+    sentinel = 0x5A5A
+    buf = torch.full((guard + M * N + guard,), sentinel, dtype=torch.int16, device="cuda")
+    Y = buf[guard:guard + M * N].view(torch.bfloat16).view(M, N)
+    cr.convrot_linear(to_torch_bf16(x), Wq, sw, g, Y=Y)
+    torch.cuda.synchronize()
+    assert bool((buf[:guard] == sentinel).all()) and bool((buf[guard + M * N:] == sentinel).all())
+    ref = oracle.linear(oracle.bf16_to_f64(x), *oracle.prepare_weight(oracle.bf16_to_f64(w), g), g)
+    assert nrmse(bf16_tensor_to_f64(Y), ref) <= NRMSE_TOL
+
+
+def test_bounded_wait_reports_timeout_without_fault(cr):
+    import torch
+
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    cr.convrot_test_wait_timeout(ws, 5_000_000)  # 5 ms; nothing will complete the barrier
+    assert cr.convrot_read_device_status(ws) == 5
+    # the context is still usable and a normal call clears the word
+    d = synth.make_workload("tiny")
+    Wq, sw = cr.convrot_prepare_weight(to_torch_bf16(d["w"]), 256)
+    ws2 = torch.empty(cr.convrot_linear_workspace_bytes(64, 256, 256, 256), dtype=torch.uint8, device="cuda")
+    ws2[:4] = 5
+    cr.convrot_linear(to_torch_bf16(d["x"]), Wq, sw, 256, ws=ws2)
+    assert cr.convrot_read_device_status(ws2) == 0

@@ -1,0 +1,229 @@
+"""INT8 ConvRot linear layer for NVIDIA B200 (sm_100a).
+
+Python binding of libconvrot (include/convrot.h). Each function has the name
+of the C entry point it calls and only marshals arguments: torch tensors are
+passed as device pointers, the current CUDA stream as the stream. Outputs and
+workspaces that the caller does not pass are allocated with torch (the
+library itself never allocates). Every computation runs in the library's
+CUDA kernels; there is no CPU path.
+
+    Wq, s_w = convrot_prepare_weight(W, g=256)         # once per layer
+    Y = convrot_linear(X, Wq, s_w, g=256, bias=b)     # per call
+"""
+
+from __future__ import annotations
+
+from . import _lib
+
+__all__ = [
+    "ConvRotError",
+    "convrot_abi_version",
+    "convrot_status_string",
+    "convrot_prepare_weight",
+    "convrot_quant_act",
+    "convrot_linear_workspace_bytes",
+    "convrot_linear",
+    "convrot_gemm_dequant",
+    "convrot_gemm_s32",
+    "convrot_read_device_status",
+    "convrot_test_wait_timeout",
+    "ConvRotLinear",
+    "lib",
+]
+
+STATUS_NAMES = {0: "CONVROT_OK", 1: "CONVROT_ERR_INVALID_ARG", 2: "CONVROT_ERR_UNSUPPORTED",
+                3: "CONVROT_ERR_WORKSPACE", 4: "CONVROT_ERR_CUDA", 5: "CONVROT_ERR_DEVICE_TIMEOUT"}
+
+
+class ConvRotError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({convrot_status_string(status)})")
+
+
+def lib():
+    """The loaded ctypes library (raises ImportError if it is not built)."""
+    return _lib.load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise ConvRotError(status, where)
+
+
+def _stream_ptr(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _require(t, dtype, shape, name):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def convrot_abi_version() -> int:
+    return int(lib().convrot_abi_version())
+
+
+def convrot_status_string(status: int) -> str:
+    return lib().convrot_status_string(int(status)).decode()
+
+
+def convrot_prepare_weight(W, g: int = 256, Wq=None, w_scale=None, ws=None, stream=None):
+    """Rotate and quantise a bf16 weight [N,K]: returns (Wq int8 [N,K], w_scale float32 [1])."""
+    import torch
+
+    _require(W, torch.bfloat16, None, "W")
+    N, K = W.shape
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty((1,), dtype=torch.float32, device=W.device)
+    L = lib()
+    if ws is None:
+        ws = torch.empty((L.convrot_prepare_weight_workspace_bytes(),), dtype=torch.uint8, device=W.device)
+    _require(Wq, torch.int8, (N, K), "Wq")
+    _require(w_scale, torch.float32, (1,), "w_scale")
+    _check(L.convrot_prepare_weight(_ptr(W), N, K, g, _ptr(Wq), _ptr(w_scale), _ptr(ws), ws.numel(),
+                                    _stream_ptr(stream)), "convrot_prepare_weight")
+    return Wq, w_scale
+
+
+def convrot_quant_act(X, g: int = 256, Xq=None, x_scale=None, stream=None):
+    """Rotate + per-token quantise bf16 X [M,K]: returns (Xq int8 [M,K], x_scale float32 [M])."""
+    import torch
+
+    _require(X, torch.bfloat16, None, "X")
+    M, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if x_scale is None:
+        x_scale = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _require(Xq, torch.int8, (M, K), "Xq")
+    _require(x_scale, torch.float32, (M,), "x_scale")
+    _check(lib().convrot_quant_act(_ptr(X), M, K, g, _ptr(Xq), _ptr(x_scale), _stream_ptr(stream)),
+           "convrot_quant_act")
+    return Xq, x_scale
+
+
+def convrot_linear_workspace_bytes(M: int, N: int, K: int, g: int) -> int:
+    return int(lib().convrot_linear_workspace_bytes(M, N, K, g))
+
+
+def convrot_linear(X, Wq, w_scale, g: int = 256, bias=None, Y=None, ws=None, stream=None):
+    """Y [M,N] bf16 = ConvRot linear of bf16 X [M,K] with the prepared weight (Wq, w_scale)."""
+    import torch
+
+    _require(X, torch.bfloat16, None, "X")
+    M, K = X.shape
+    _require(Wq, torch.int8, None, "Wq")
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("Wq must be [N, K] with the K of X")
+    _require(w_scale, torch.float32, (1,), "w_scale")
+    if bias is not None:
+        _require(bias, torch.bfloat16, (N,), "bias")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    need = convrot_linear_workspace_bytes(M, N, K, g)
+    if ws is None:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=X.device)
+    _check(lib().convrot_linear(_ptr(X), M, K, g, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y), _ptr(ws),
+                                ws.numel(), _stream_ptr(stream)), "convrot_linear")
+    return Y
+
+
+def convrot_gemm_dequant(Xq, x_scale, Wq, w_scale, bias=None, Y=None, ws=None, stream=None):
+    """GEMM + epilogue on already-quantised codes: Y [M,N] bf16."""
+    import torch
+
+    _require(Xq, torch.int8, None, "Xq")
+    M, K = Xq.shape
+    _require(Wq, torch.int8, None, "Wq")
+    N = Wq.shape[0]
+    _require(x_scale, torch.float32, (M,), "x_scale")
+    _require(w_scale, torch.float32, (1,), "w_scale")
+    if bias is not None:
+        _require(bias, torch.bfloat16, (N,), "bias")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    L = lib()
+    if ws is None:
+        ws = torch.empty((L.convrot_gemm_workspace_bytes(),), dtype=torch.uint8, device=Xq.device)
+    _check(L.convrot_gemm_dequant(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, _ptr(bias), _ptr(Y),
+                                  _ptr(ws), ws.numel(), _stream_ptr(stream)), "convrot_gemm_dequant")
+    return Y
+
+
+def convrot_gemm_s32(Xq, Wq, acc=None, ws=None, stream=None):
+    """Raw int32 accumulators acc [M,N] = Xq Wq^T from the tcgen05 GEMM."""
+    import torch
+
+    _require(Xq, torch.int8, None, "Xq")
+    M, K = Xq.shape
+    _require(Wq, torch.int8, None, "Wq")
+    N = Wq.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    _require(acc, torch.int32, (M, N), "acc")
+    L = lib()
+    if ws is None:
+        ws = torch.empty((L.convrot_gemm_workspace_bytes(),), dtype=torch.uint8, device=Xq.device)
+    _check(L.convrot_gemm_s32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _ptr(ws), ws.numel(), _stream_ptr(stream)),
+           "convrot_gemm_s32")
+    return acc
+
+
+def convrot_read_device_status(ws, stream=None) -> int:
+    """Status word of a workspace (synchronises the stream): 0 or CONVROT_ERR_DEVICE_TIMEOUT (5)."""
+    return int(lib().convrot_read_device_status(_ptr(ws), _stream_ptr(stream)))
+
+
+def convrot_test_wait_timeout(ws, timeout_ns: int, stream=None) -> None:
+    _check(lib().convrot_test_wait_timeout(_ptr(ws), ws.numel(), int(timeout_ns), _stream_ptr(stream)),
+           "convrot_test_wait_timeout")
+
+
+class ConvRotLinear:
+    """A ConvRot linear layer: prepared int8 weight + optional bias, reusable workspace.
+
+    ``layer = ConvRotLinear(W, bias, g=256)`` rotates and quantises W once;
+    ``layer(X)`` runs convrot_linear on the current stream.
+    """
+
+    def __init__(self, W, bias=None, g: int = 256):
+        self.g = g
+        self.N, self.K = W.shape
+        self.Wq, self.w_scale = convrot_prepare_weight(W, g)
+        self.bias = bias
+        self._ws = None
+
+    def workspace(self, M: int):
+        import torch
+
+        need = convrot_linear_workspace_bytes(M, self.N, self.K, self.g)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty((need,), dtype=torch.uint8, device=self.Wq.device)
+        return self._ws
+
+    def __call__(self, X, Y=None, stream=None):
+        return convrot_linear(X, self.Wq, self.w_scale, self.g, self.bias, Y, self.workspace(X.shape[0]), stream)

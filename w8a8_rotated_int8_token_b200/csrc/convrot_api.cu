@@ -1,0 +1,225 @@
+// C ABI of libconvrot (declared in include/convrot.h): argument checks on the
+// host, workspace layout, and the launches of the rotation/quantisation and
+// GEMM kernels. Nothing here allocates device memory or synchronises, except
+// convrot_read_device_status.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "convrot.h"
+#include "gemm_i8.cuh"
+#include "rotate_quant.cuh"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
+
+// Workspace of convrot_linear: [status word | token scales | int8 codes].
+constexpr size_t kStatusBytes = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct LinearWs {
+  size_t scale_off, codes_off, total;
+};
+
+LinearWs linear_ws_layout(int64_t M, int64_t K) {
+  LinearWs w;
+  w.scale_off = kStatusBytes;
+  w.codes_off = align_up(w.scale_off + 4 * static_cast<size_t>(M), 1024);
+  w.total = align_up(w.codes_off + static_cast<size_t>(M) * static_cast<size_t>(K), 256);
+  return w;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+convrot_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA; }
+
+// Checks shared by every entry point that rotates rows of length K in groups of g.
+convrot_status check_rotation_shape(int64_t rows, int64_t K, int g) {
+  if (rows < 1 || K < 1) return CONVROT_ERR_INVALID_ARG;
+  if (g != 128 && g != 256) return CONVROT_ERR_UNSUPPORTED;
+  if (K % g != 0) return CONVROT_ERR_INVALID_ARG;
+  if (K > CONVROT_MAX_K) return CONVROT_ERR_UNSUPPORTED;
+  if (rows > (int64_t(1) << 31) - 1) return CONVROT_ERR_UNSUPPORTED;
+  return CONVROT_OK;
+}
+
+// Checks of the GEMM shape: TMA needs 16-byte row strides; coordinates are int32.
+convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int n_multiple) {
+  if (M < 1 || N < 1 || K < 1) return CONVROT_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % n_multiple != 0) return CONVROT_ERR_INVALID_ARG;
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (M > lim || N > lim || K > lim) return CONVROT_ERR_UNSUPPORTED;
+  return CONVROT_OK;
+}
+
+convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, int64_t M, int64_t N, int64_t K,
+                        const float* x_scale, const float* w_scale, const void* bias, int* status,
+                        cudaStream_t stream) {
+  convrot::GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.x_scale = x_scale;
+  p.w_scale = w_scale;
+  p.bias = static_cast<const uint16_t*>(bias);
+  p.status = status;
+  p.timeout_ns = kWaitTimeoutNs;
+  p.group_m = 0;
+  return from_cuda(convrot::launch_gemm_i8(epi, Xq, Wq, out, p, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int convrot_abi_version(void) { return kAbiVersion; }
+
+const char* convrot_status_string(int status) {
+  switch (status) {
+    case CONVROT_OK: return "ok";
+    case CONVROT_ERR_INVALID_ARG: return "invalid argument (null pointer, size, or alignment)";
+    case CONVROT_ERR_UNSUPPORTED: return "unsupported configuration (group size or size limit)";
+    case CONVROT_ERR_WORKSPACE: return "workspace null, misaligned or too small";
+    case CONVROT_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case CONVROT_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t convrot_prepare_weight_workspace_bytes(void) { return 256; }
+
+convrot_status convrot_prepare_weight(const void* W, int64_t N, int64_t K, int g, int8_t* Wq, float* w_scale,
+                                      void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  const convrot_status sh = check_rotation_shape(N, K, g);
+  if (sh != CONVROT_OK) return sh;
+  if (W == nullptr || Wq == nullptr || w_scale == nullptr) return CONVROT_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(w_scale, 4)) return CONVROT_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < convrot_prepare_weight_workspace_bytes())
+    return CONVROT_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned* amax = static_cast<unsigned*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return CONVROT_ERR_CUDA;
+  convrot::RotQuantParams p{};
+  p.src = static_cast<const uint16_t*>(W);
+  p.rows = N;
+  p.K = K;
+  p.dst = Wq;
+  p.scale = w_scale;
+  p.tensor_absmax = amax;
+  p.status_reset = nullptr;
+  e = convrot::launch_rotate_quant(g, convrot::kRqWeightAbsmax, p, s);
+  if (e != cudaSuccess) return CONVROT_ERR_CUDA;
+  return from_cuda(convrot::launch_rotate_quant(g, convrot::kRqWeightQuant, p, s));
+}
+
+convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int8_t* Xq, float* x_scale,
+                                 convrot_stream_t stream) {
+  const convrot_status sh = check_rotation_shape(M, K, g);
+  if (sh != CONVROT_OK) return sh;
+  if (X == nullptr || Xq == nullptr || x_scale == nullptr) return CONVROT_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(x_scale, 4)) return CONVROT_ERR_INVALID_ARG;
+  convrot::RotQuantParams p{};
+  p.src = static_cast<const uint16_t*>(X);
+  p.rows = M;
+  p.K = K;
+  p.dst = Xq;
+  p.scale = x_scale;
+  p.tensor_absmax = nullptr;
+  p.status_reset = nullptr;
+  return from_cuda(
+      convrot::launch_rotate_quant(g, convrot::kRqActivation, p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
+  if (check_rotation_shape(M, K, g) != CONVROT_OK || check_gemm_shape(M, N, K, 8) != CONVROT_OK) return 0;
+  return linear_ws_layout(M, K).total;
+}
+
+convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq, const float* w_scale,
+                              int64_t N, const void* bias, void* Y, void* ws, size_t ws_bytes,
+                              convrot_stream_t stream) {
+  convrot_status sh = check_rotation_shape(M, K, g);
+  if (sh != CONVROT_OK) return sh;
+  sh = check_gemm_shape(M, N, K, 8);
+  if (sh != CONVROT_OK) return sh;
+  if (X == nullptr || Wq == nullptr || w_scale == nullptr || Y == nullptr) return CONVROT_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(w_scale, 4) || !aligned(Y, 16) ||
+      (bias != nullptr && !aligned(bias, 16)))
+    return CONVROT_ERR_INVALID_ARG;
+  const LinearWs lay = linear_ws_layout(M, K);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(wsb);
+  float* x_scale = reinterpret_cast<float*>(wsb + lay.scale_off);
+  int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
+
+  convrot::RotQuantParams p{};
+  p.src = static_cast<const uint16_t*>(X);
+  p.rows = M;
+  p.K = K;
+  p.dst = Xq;
+  p.scale = x_scale;
+  p.tensor_absmax = nullptr;
+  p.status_reset = status;  // CTA 0 of the first kernel clears the status word of this call
+  if (convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return run_gemm(convrot::kEpiDequantBf16, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s);
+}
+
+size_t convrot_gemm_workspace_bytes(void) { return kStatusBytes; }
+
+convrot_status convrot_gemm_dequant(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale,
+                                    int64_t M, int64_t N, int64_t K, const void* bias, void* Y, void* ws,
+                                    size_t ws_bytes, convrot_stream_t stream) {
+  const convrot_status sh = check_gemm_shape(M, N, K, 8);
+  if (sh != CONVROT_OK) return sh;
+  if (Xq == nullptr || x_scale == nullptr || Wq == nullptr || w_scale == nullptr || Y == nullptr)
+    return CONVROT_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(x_scale, 4) || !aligned(w_scale, 4) ||
+      (bias != nullptr && !aligned(bias, 16)))
+    return CONVROT_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < kStatusBytes) return CONVROT_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return run_gemm(convrot::kEpiDequantBf16, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s);
+}
+
+convrot_status convrot_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
+                                void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  const convrot_status sh = check_gemm_shape(M, N, K, 4);
+  if (sh != CONVROT_OK) return sh;
+  if (Xq == nullptr || Wq == nullptr || acc == nullptr) return CONVROT_ERR_INVALID_ARG;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(acc, 16)) return CONVROT_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < kStatusBytes) return CONVROT_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return run_gemm(convrot::kEpiRawS32, Xq, Wq, acc, M, N, K, nullptr, nullptr, nullptr, status, s);
+}
+
+convrot_status convrot_read_device_status(const void* ws, convrot_stream_t stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return CONVROT_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  if (host == 0) return CONVROT_OK;
+  return host == CONVROT_ERR_DEVICE_TIMEOUT ? CONVROT_ERR_DEVICE_TIMEOUT : CONVROT_ERR_CUDA;
+}
+
+convrot_status convrot_test_wait_timeout(void* ws, size_t ws_bytes, int64_t timeout_ns, convrot_stream_t stream) {
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < kStatusBytes) return CONVROT_ERR_WORKSPACE;
+  if (timeout_ns < 1000 || timeout_ns > 1000000000) return CONVROT_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return from_cuda(convrot::launch_wait_timeout(status, static_cast<uint64_t>(timeout_ns), s));
+}
+
+}  // extern "C"
