@@ -154,6 +154,34 @@ CONVROT_API convrot_status convrot_gemm_s32(const int8_t* Xq, const int8_t* Wq,
                                 void* ws, size_t ws_bytes, convrot_stream_t stream);
 
 /*
+ * convrot_linear_noalloc -- convrot_linear without a caller-provided workspace,
+ * for callers that cannot allocate device memory: a plugin inside a host
+ * application that owns the device-memory budget and passes only input and
+ * output buffers, or a latency-critical loop where cudaMalloc/cudaFree could
+ * synchronise the device or fail. The pages describe no such entry point;
+ * it has no counterpart there.
+ *   Arguments as convrot_linear, minus the workspace. The scratch (status
+ *   word, token scales, int8 codes) is one built-in device array of
+ *   CONVROT_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds
+ *   until the process exits. A call needing more
+ *   (convrot_linear_workspace_bytes(M, N, K, g) > CONVROT_NOALLOC_SCRATCH_BYTES,
+ *   roughly M*K > 64 MiB) returns CONVROT_ERR_WORKSPACE and enqueues nothing.
+ *   device_status: NULL, or a device int that receives the call's status word
+ *   (0, or CONVROT_ERR_DEVICE_TIMEOUT) once the call has run on `stream`.
+ * Allocates nothing. The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current) and keeps it; make
+ * that first call before any stream capture begins. All calls share the array:
+ * calls that may overlap on the GPU (unordered streams, several host threads)
+ * race on it and must not be issued. Each call clears the status word and
+ * rewrites the codes and scales, so no result depends on an earlier call.
+ */
+#define CONVROT_NOALLOC_SCRATCH_BYTES (64u << 20)
+CONVROT_API convrot_status convrot_linear_noalloc(const void* X, int64_t M, int64_t K, int g,
+                                                  const int8_t* Wq, const float* w_scale, int64_t N,
+                                                  const void* bias, void* Y, int* device_status,
+                                                  convrot_stream_t stream);
+
+/*
  * convrot_read_device_status -- copy the status word of a workspace used by
  * convrot_linear / convrot_gemm_* back to the host and return it
  * (CONVROT_OK, or CONVROT_ERR_DEVICE_TIMEOUT if a bounded wait ran out).

@@ -32,6 +32,8 @@ SIGNATURES = {
                                     _c_void_p, _c_void_p, _size, _c_void_p]),
     "convrot_gemm_s32": (_int, [_c_void_p, _c_void_p, _i64, _i64, _i64, _c_void_p, _c_void_p, _size,
                                 _c_void_p]),
+    "convrot_linear_noalloc": (_int, [_c_void_p, _i64, _i64, _int, _c_void_p, _c_void_p, _i64, _c_void_p,
+                                      _c_void_p, _c_void_p, _c_void_p]),
     "convrot_read_device_status": (_int, [_c_void_p, _c_void_p]),
     "convrot_test_wait_timeout": (_int, [_c_void_p, _size, _i64, _c_void_p]),
 }
