@@ -111,7 +111,9 @@ CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K
  *   Y = bf16_rne( (Xq Wq^T) * (s_x[m] * s_w) + bias[n] ),  (Xq, s_x) = quant_act(X).
  * The int8 x int8 product accumulates exactly in int32 on the tcgen05 tensor
  * cores (InvokeAI "int8 Compute", second paragraph); dequantisation and the
- * bias are fused into the GEMM epilogue.
+ * bias are fused into the GEMM epilogue. For K <= 20480 the whole layer is one
+ * kernel: worker warps rotate and quantise the tokens while the tensor cores
+ * multiply the M-blocks already finished; above that it is two kernels.
  *   X        [M,K] bf16, device.   M >= 1, N >= 1, K % g == 0, K <= CONVROT_MAX_K,
  *                                   N % 8 == 0.
  *   Wq       [N,K] int8, device (from convrot_prepare_weight with the same g).
@@ -120,15 +122,35 @@ CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K
  *   Y        [M,N] bf16 out, device. Must not overlap any input.
  *   ws       device workspace, 256-byte aligned, ws_bytes >=
  *            convrot_linear_workspace_bytes(M, N, K, g). It holds the status
- *            word, the token scales and the int8 activation codes of this call;
- *            calls that may run at the same time need separate workspaces.
- * Enqueues two kernels (rotate+quantise, then GEMM+epilogue).
+ *            word, per-128-token readiness counters, the token scales and the
+ *            int8 activation codes of this call; calls that may run at the
+ *            same time need separate workspaces. Its contents need no
+ *            initialisation (counters carry a per-call tag).
  */
 CONVROT_API size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 CONVROT_API convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g,
                               const int8_t* Wq, const float* w_scale, int64_t N,
                               const void* bias, void* Y,
                               void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * convrot_linear_timed -- convrot_linear that also records caller-created CUDA
+ * events (cudaEvent_t, passed as void*) on `stream`: ev_start before its first
+ * launch, ev_mid after the rotate+quantise kernel (may be NULL; with the
+ * one-launch form it is recorded together with ev_end), ev_end after the
+ * GEMM. The layer's and each kernel's device time can then be read with
+ * cudaEventElapsedTime on the launching stream. ev_mid keeps the GEMM from
+ * overlapping the first kernel's tail.
+ */
+CONVROT_API convrot_status convrot_linear_timed(const void* X, int64_t M, int64_t K, int g,
+                                                const int8_t* Wq, const float* w_scale, int64_t N,
+                                                const void* bias, void* Y,
+                                                void* ws, size_t ws_bytes,
+                                                void* ev_start, void* ev_mid, void* ev_end,
+                                                convrot_stream_t stream);
+
+/* Kernel launches one convrot_linear call of this shape enqueues (1 or 2), 0 if invalid. */
+CONVROT_API int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g);
 
 /*
  * convrot_gemm_dequant -- the GEMM + epilogue half of convrot_linear, on codes

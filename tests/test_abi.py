@@ -52,8 +52,17 @@ def test_library_exports_nothing_else():
     assert exported == set(_declared_entry_points())
 
 
+def linear_ws_layout(M, K):
+    """Byte layout of convrot_linear's workspace, as include/convrot.h describes it."""
+    up = lambda v, a: (v + a - 1) // a * a  # noqa: E731
+    ready = 256
+    scale = up(ready + 8 * ((M + 127) // 128), 256)
+    codes = up(scale + 4 * M, 1024)
+    return {"ready": ready, "scale": scale, "codes": codes, "total": up(codes + M * K, 256)}
+
+
 def test_status_strings_and_version(L):
-    assert L.convrot_abi_version() == 1
+    assert L.convrot_abi_version() == 2
     for code in range(6):
         s = L.convrot_status_string(code)
         assert s and s != b"unknown status"
@@ -61,12 +70,11 @@ def test_status_strings_and_version(L):
 
 
 def test_workspace_sizes(L):
-    # [status 256 B | scales 4M, 1 KB aligned | codes M*K], 256-aligned
+    # [status 256 B | ready counters 8 B per 128 tokens | scales 4M | codes M*K]
     M, N, K = 4608, 9216, 3072
     need = L.convrot_linear_workspace_bytes(M, N, K, 256)
-    scale_end = 256 + 4 * M
-    codes_off = (scale_end + 1023) // 1024 * 1024
-    assert need == (codes_off + M * K + 255) // 256 * 256
+    assert need == linear_ws_layout(M, K)["total"]
+    assert need >= M * K + 4 * M + 8 * (M // 128) + 256
     assert L.convrot_linear_workspace_bytes(M, N, K, 64) == 0       # unsupported g
     assert L.convrot_linear_workspace_bytes(M, N, 3000, 256) == 0   # K % g != 0
     assert L.convrot_linear_workspace_bytes(M, 9212, K, 256) == 0   # N % 8 != 0
@@ -113,6 +121,11 @@ def test_other_entry_points_reject_bad_arguments_on_host(L):
     assert L.convrot_read_device_status(None, None) == 3
     assert L.convrot_test_wait_timeout(FAKE, 256, 10, None) == 1
     assert L.convrot_test_wait_timeout(FAKE, 256, 10**10, None) == 1
+    # the timed variant needs both events
+    assert L.convrot_linear_timed(FAKE, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30, None, None,
+                                  FAKE, None) == 1
+    assert L.convrot_linear_launch_count(4608, 9216, 3072, 256) in (1, 2)
+    assert L.convrot_linear_launch_count(4608, 9216, 3000, 256) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

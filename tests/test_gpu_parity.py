@@ -14,6 +14,7 @@ import pytest
 import oracle
 import synth
 from parity import (NRMSE_TOL, bf16_tensor_to_f64, check_codes, nrmse, to_torch_bf16)
+from test_abi import linear_ws_layout
 
 pytestmark = pytest.mark.gpu
 
@@ -225,9 +226,9 @@ def _linear_case(cr, d, rows=None):
     assert err <= NRMSE_TOL, f"{w.name}: NRMSE {err}"
     # the codes and token scales this call left in its workspace
     wsn = ws.cpu().numpy()
-    codes_off = (256 + 4 * M + 1023) // 1024 * 1024
-    sx_gpu = wsn[256:256 + 4 * M].view(np.float32)[rows]
-    xq_gpu = wsn[codes_off:codes_off + M * K].view(np.int8).reshape(M, K)[rows]
+    lay = linear_ws_layout(M, K)
+    sx_gpu = wsn[lay["scale"]:lay["scale"] + 4 * M].view(np.float32)[rows]
+    xq_gpu = wsn[lay["codes"]:lay["codes"] + M * K].view(np.int8).reshape(M, K)[rows]
     xr = oracle.rotate(xs, g)
     q_ref, s_ref = oracle.quantize_per_token(xr)
     check_codes(xq_gpu, sx_gpu, xr, q_ref, s_ref)
@@ -278,6 +279,47 @@ def test_zero_input_gives_zero_output_and_bias(cr):
     Yb = cr.convrot_linear(X, Wq, sw, 256, b)
     torch.cuda.synchronize()
     assert torch.equal(Yb.view(torch.int16), b.view(torch.int16).expand(130, -1))
+
+
+@pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256),   # largest K of the one-launch form
+                                     (129, 136, 20608, 128),   # two kernels (K above the fused limit)
+                                     (67, 264, 32768, 256),    # two kernels, largest K
+                                     (1, 16, 384, 128), (385, 520, 1024, 256)])
+def test_linear_fused_and_two_kernel_forms(cr, M, N, K, g):
+    rng = np.random.default_rng(M + N + K)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, rng.choice(K, max(1, K // 100), replace=False)] *= 50.0
+    d = {"workload": type("W", (), {"name": f"{M}x{K}x{N}", "g": g})(),
+         "x": synth.f32_to_bf16_bits(x),
+         "w": synth.f32_to_bf16_bits((rng.standard_normal((N, K)) * 0.02).astype(np.float32)),
+         "bias": synth.f32_to_bf16_bits((rng.standard_normal(N) * 0.01).astype(np.float32))}
+    _linear_case(cr, d)
+
+
+def test_linear_back_to_back_calls_on_one_workspace(cr):
+    """Consecutive calls reuse the workspace: later calls must not see earlier readiness counters."""
+    import torch
+
+    a = synth.make_workload("dit_qkv_1024")
+    b = synth.make_workload("tiny")
+    Wa, sa = cr.convrot_prepare_weight(to_torch_bf16(a["w"]), 256)
+    Wb, sb = cr.convrot_prepare_weight(to_torch_bf16(b["w"]), 256)
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(4608, 9216, 3072, 256), dtype=torch.uint8, device="cuda")
+    Xa = to_torch_bf16(a["x"])
+    Xb = to_torch_bf16(b["x"])
+    ref_a = cr.convrot_linear(Xa, Wa, sa, 256, to_torch_bf16(a["bias"]))
+    ref_b = cr.convrot_linear(Xb, Wb, sb, 256)
+    outs = []
+    for i in range(6):  # alternate layers on the same workspace, no synchronisation in between
+        if i % 2 == 0:
+            outs.append(("a", cr.convrot_linear(Xa, Wa, sa, 256, to_torch_bf16(a["bias"]), ws=ws)))
+        else:
+            outs.append(("b", cr.convrot_linear(Xb, Wb, sb, 256, ws=ws)))
+    torch.cuda.synchronize()
+    assert cr.convrot_read_device_status(ws) == 0
+    for tag, y in outs:
+        ref = ref_a if tag == "a" else ref_b
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
 
 
 @pytest.mark.parametrize("M,N,K", [(130, 264, 256), (1, 8, 128), (257, 1032, 384)])

@@ -27,6 +27,9 @@ SIGNATURES = {
     "convrot_linear_workspace_bytes": (_size, [_i64, _i64, _i64, _int]),
     "convrot_linear": (_int, [_c_void_p, _i64, _i64, _int, _c_void_p, _c_void_p, _i64, _c_void_p, _c_void_p,
                               _c_void_p, _size, _c_void_p]),
+    "convrot_linear_timed": (_int, [_c_void_p, _i64, _i64, _int, _c_void_p, _c_void_p, _i64, _c_void_p,
+                                    _c_void_p, _c_void_p, _size, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "convrot_linear_launch_count": (_int, [_i64, _i64, _i64, _int]),
     "convrot_gemm_workspace_bytes": (_size, []),
     "convrot_gemm_dequant": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _c_void_p,
                                     _c_void_p, _c_void_p, _size, _c_void_p]),

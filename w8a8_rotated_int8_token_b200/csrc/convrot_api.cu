@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "convrot.h"
@@ -13,24 +14,43 @@
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
+// The one-launch form (rotate+quantise worker warps inside the GEMM kernel) is
+// correct but, measured on the DiT QKV layer, its workers fall behind the
+// tensor cores (137 us vs 94 + 16 us for the two kernels), so the layer runs
+// as two kernels chained with programmatic dependent launch.
+constexpr bool kFusedLinear = false;
 
-// Workspace of convrot_linear: [status word | token scales | int8 codes].
+// Workspace of convrot_linear:
+// [status word | 256 B][M-block ready counters, 8 B each][token scales][int8 codes].
 constexpr size_t kStatusBytes = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct LinearWs {
-  size_t scale_off, codes_off, total;
+  size_t ready_off, scale_off, codes_off, total;
 };
 
 LinearWs linear_ws_layout(int64_t M, int64_t K) {
   LinearWs w;
-  w.scale_off = kStatusBytes;
+  w.ready_off = kStatusBytes;
+  const size_t mblocks = (static_cast<size_t>(M) + 127) / 128;
+  w.scale_off = align_up(w.ready_off + 8 * mblocks, 256);
   w.codes_off = align_up(w.scale_off + 4 * static_cast<size_t>(M), 1024);
   w.total = align_up(w.codes_off + static_cast<size_t>(M) * static_cast<size_t>(K), 256);
   return w;
+}
+
+// Epoch of a fused call: unique in the process, never 0, so that ready
+// counters left in a workspace by earlier calls never look finished.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> counter{0x5A17u};
+  uint32_t e;
+  do {
+    e = counter.fetch_add(1u, std::memory_order_relaxed) + 1u;
+  } while (e == 0u);
+  return e;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -112,6 +132,8 @@ convrot_status convrot_prepare_weight(const void* W, int64_t N, int64_t K, int g
   p.scale = w_scale;
   p.tensor_absmax = amax;
   p.status_reset = nullptr;
+  p.status = nullptr;
+  p.timeout_ns = kWaitTimeoutNs;
   e = convrot::launch_rotate_quant(g, convrot::kRqWeightAbsmax, p, s);
   if (e != cudaSuccess) return CONVROT_ERR_CUDA;
   return from_cuda(convrot::launch_rotate_quant(g, convrot::kRqWeightQuant, p, s));
@@ -131,6 +153,8 @@ convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int
   p.scale = x_scale;
   p.tensor_absmax = nullptr;
   p.status_reset = nullptr;
+  p.status = nullptr;
+  p.timeout_ns = kWaitTimeoutNs;
   return from_cuda(
       convrot::launch_rotate_quant(g, convrot::kRqActivation, p, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -140,9 +164,16 @@ size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
   return linear_ws_layout(M, K).total;
 }
 
-convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq, const float* w_scale,
-                              int64_t N, const void* bias, void* Y, void* ws, size_t ws_bytes,
-                              convrot_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// convrot_linear: one fused launch when the worker layout fits (K <= 20480),
+// else the rotate+quantise kernel followed by the GEMM. Events (may be null)
+// are recorded before and after the launches.
+convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq, const float* w_scale,
+                           int64_t N, const void* bias, void* Y, void* ws, size_t ws_bytes, cudaEvent_t ev0,
+                           cudaEvent_t ev1, cudaEvent_t ev2, cudaStream_t s) {
   convrot_status sh = check_rotation_shape(M, K, g);
   if (sh != CONVROT_OK) return sh;
   sh = check_gemm_shape(M, N, K, 8);
@@ -153,11 +184,35 @@ convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g, const 
     return CONVROT_ERR_INVALID_ARG;
   const LinearWs lay = linear_ws_layout(M, K);
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(wsb);
   float* x_scale = reinterpret_cast<float*>(wsb + lay.scale_off);
   int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
+
+  int tpr = 0, rpp = 0, cta_threads = 0;
+  if (kFusedLinear && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) {
+    // one launch: worker warps rotate + quantise while the GEMM consumes finished M-blocks
+    convrot::GemmParams gp{};
+    gp.M = static_cast<int>(M);
+    gp.N = static_cast<int>(N);
+    gp.K = static_cast<int>(K);
+    gp.x_scale = x_scale;
+    gp.w_scale = w_scale;
+    gp.bias = static_cast<const uint16_t*>(bias);
+    gp.status = status;
+    gp.timeout_ns = kWaitTimeoutNs;
+    gp.group_m = 0;
+    gp.X = static_cast<const uint16_t*>(X);
+    gp.Xq = Xq;
+    gp.x_scale_out = x_scale;
+    gp.ready = reinterpret_cast<unsigned long long*>(wsb + lay.ready_off);
+    gp.epoch = next_epoch();
+    if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (convrot::launch_linear_fused(g, Wq, Y, gp, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (ev2 != nullptr && cudaEventRecord(ev2, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    return CONVROT_OK;
+  }
 
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(X);
@@ -167,8 +222,42 @@ convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g, const 
   p.scale = x_scale;
   p.tensor_absmax = nullptr;
   p.status_reset = status;  // CTA 0 of the first kernel clears the status word of this call
+  p.status = status;
+  p.timeout_ns = kWaitTimeoutNs;
+  if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s) != cudaSuccess) return CONVROT_ERR_CUDA;
-  return run_gemm(convrot::kEpiDequantBf16, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s);
+  if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  const convrot_status st = run_gemm(convrot::kEpiDequantBf16, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s);
+  if (st != CONVROT_OK) return st;
+  if (ev2 != nullptr && cudaEventRecord(ev2, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return CONVROT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+convrot_status convrot_linear(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq, const float* w_scale,
+                              int64_t N, const void* bias, void* Y, void* ws, size_t ws_bytes,
+                              convrot_stream_t stream) {
+  return linear_impl(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, nullptr, nullptr, nullptr,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+convrot_status convrot_linear_timed(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq,
+                                    const float* w_scale, int64_t N, const void* bias, void* Y, void* ws,
+                                    size_t ws_bytes, void* ev_start, void* ev_mid, void* ev_end,
+                                    convrot_stream_t stream) {
+  if (ev_start == nullptr || ev_end == nullptr) return CONVROT_ERR_INVALID_ARG;
+  return linear_impl(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, static_cast<cudaEvent_t>(ev_start),
+                     static_cast<cudaEvent_t>(ev_mid), static_cast<cudaEvent_t>(ev_end),
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g) {
+  if (check_rotation_shape(M, K, g) != CONVROT_OK || check_gemm_shape(M, N, K, 8) != CONVROT_OK) return 0;
+  int tpr = 0, rpp = 0, cta_threads = 0;
+  return (kFusedLinear && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) ? 1 : 2;
 }
 
 size_t convrot_gemm_workspace_bytes(void) { return kStatusBytes; }

@@ -1,12 +1,14 @@
 // int8 x int8 -> int32 GEMM on the 5th-generation tensor cores (tcgen05,
 // kind::i8) with a fused epilogue, for Y = Xq Wq^T: both operands K-major.
+// In its fused form the same kernel also produces Xq: the whole ConvRot
+// linear layer in one launch.
 //
 // The int8-by-int8 product with int32 accumulation is the multiply step of
 // the ConvRot layer (InvokeAI "int8 Compute", second paragraph); the
 // epilogue applies the token and tensor scales and the bias and rounds to
 // bf16 (or, for exactness tests, stores the raw int32 accumulators).
 //
-// Structure: a persistent kernel, one CTA per SM, 6 warps.
+// Structure: a persistent kernel, one CTA per SM.
 //   warp 0, one lane : TMA producer. 128x128 (A) and 256x128 (B) int8 tiles,
 //                      128-byte swizzle, into a 4-stage shared-memory ring.
 //   warp 1           : allocates 512 TMEM columns; one lane issues
@@ -19,6 +21,17 @@
 //                      shared memory and writes them with TMA stores. Two
 //                      accumulators let the epilogue of tile i overlap the
 //                      MMAs of tile i+1.
+//   warps 6..        : (fused form only) rotate + quantise workers. The CTAs
+//                      together walk the token rows in order, a few rows per
+//                      CTA per pass, and write the int8 codes and token scales
+//                      of A. After each pass one thread publishes the rows it
+//                      finished in a per-M-block counter tagged with the call's
+//                      epoch (release); the producer acquires the counter of
+//                      an M-block before its first TMA load of that block, and
+//                      the epilogue before reading the block's token scales.
+//                      The workers never wait on the GEMM roles, so the GEMM
+//                      runs on the tensor cores while the rotation still runs
+//                      on the CUDA cores for later rows.
 // Tiles are visited in groups of `group_m` M-blocks so that the CTAs in flight
 // share A and B panels in L2. Every wait is bounded; a wait that runs out
 // records CONVROT_ERR_DEVICE_TIMEOUT (5) in the status word, every role
@@ -30,8 +43,10 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <cstdint>
 
+#include "fwht_dev.cuh"
 #include "gemm_i8.cuh"
 #include "ptx_sm100.cuh"
 
@@ -52,6 +67,7 @@ constexpr int CHUNK = 32;  // epilogue columns per TMEM load / TMA store
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = idesc_i8(BM, BN);
 constexpr int kTimeoutStatus = 5;
+constexpr int kFusedMaxThreads = 512;  // 6 GEMM warps + up to 10 rotate+quantise warps
 
 template <int EPI>
 struct Smem {
@@ -63,7 +79,8 @@ struct Smem {
   static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 8;
-  static constexpr int kBytes = kOffAbort + 8;
+  static constexpr int kOffRowMax = kOffAbort + 8;  // fused form: 2 x kMaxFusedRows row maxima
+  static constexpr int kBytes = kOffRowMax + 2 * kMaxFusedRows * 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
 };
 
@@ -83,15 +100,271 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* status) {
   atomicOr(status, kTimeoutStatus);
 }
 
+__device__ __forceinline__ uint64_t ld_acquire_u64(const unsigned long long* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float ld_relaxed_f32(const float* p) {
+  float v;
+  asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also ORs a predicate over the participating threads.
+__device__ __forceinline__ bool named_barrier_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %3, 0;\n\t"
+      "bar.red.or.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(threads), "r"(static_cast<uint32_t>(pred))
+      : "memory");
+  return r != 0;
+}
+
+// Rows of M-block mb that the fused workers must finish, tagged with the epoch.
+__device__ __forceinline__ uint64_t ready_target(const GemmParams& p, int mb) {
+  const int rows = (p.M - mb * BM) < BM ? (p.M - mb * BM) : BM;
+  return (static_cast<uint64_t>(p.epoch) << 32) | static_cast<uint64_t>(rows);
+}
+
+// Bounded wait until every row of M-block mb has been quantised in this call.
+__device__ __forceinline__ bool wait_block_ready(const GemmParams& p, int mb, volatile int* abort) {
+  const uint64_t target = ready_target(p, mb);
+  if (ld_acquire_u64(p.ready + mb) == target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_u64(p.ready + mb) == target) return true;
+    if ((it & 15u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (global_timer_ns() - t0 > p.timeout_ns) return false;
+    }
+  }
+}
+
+// Add n finished rows to M-block mb's counter for this epoch (a stale epoch
+// restarts the count). Called after a gpu-scope fence: release.
+__device__ __forceinline__ void publish_rows(const GemmParams& p, int mb, int n) {
+  unsigned long long* c = p.ready + mb;
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(c);
+  while (true) {
+    const unsigned long long nw = ((old >> 32) == p.epoch)
+                                      ? old + static_cast<unsigned long long>(n)
+                                      : ((static_cast<unsigned long long>(p.epoch) << 32) | static_cast<unsigned>(n));
+    const unsigned long long prev = atomicCAS(c, old, nw);
+    if (prev == old) break;
+    old = prev;
+  }
+}
+
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// One tile's epilogue for one warp: 8 chunks of 32 accumulator columns of the
+// warp's 32 TMEM lanes (rows row0..row0+31): load, scale + bias, pack, stage in
+// swizzled shared memory, TMA store. release() is called by lane 0 once the
+// accumulator has been read completely.
+template <int EPI, class Release>
+__device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmOut, const GemmParams& p, uint32_t t_row,
+                                              int row0, int n_base, float sc, uint8_t* ebuf0, int& chunk_count,
+                                              int lane, Release release) {
+  constexpr int kEpiBuf = (EPI == kEpiDequantBf16) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
+#pragma unroll 1
+  for (int c = 0; c < BN / CHUNK; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * CHUNK), r);
+    tmem_ld_wait();
+    if (c == BN / CHUNK - 1) {  // accumulator fully read: hand it back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) release();
+    }
+    const int n0 = n_base + c * CHUNK;
+    if (n0 >= p.N) continue;
+    uint8_t* ebuf = ebuf0 + (chunk_count & 1) * kEpiBuf;
+    if (lane == 0) bulk_wait_group_read<1>();  // the store that last read this buffer is done
+    __syncwarp();
+    if (EPI == kEpiDequantBf16) {
+      float bv[32];
+      if (p.bias != nullptr) {
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (n0 + 8 * pc < p.N) w = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * pc));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            bv[8 * pc + 2 * e] = __uint_as_float(ws[e] << 16);
+            bv[8 * pc + 2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) bv[e] = 0.0f;
+      }
+      uint32_t packed[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float y0 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e])), sc, bv[2 * e]);
+        const float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e + 1])), sc, bv[2 * e + 1]);
+        packed[e] = bf16x2(y0, y1);
+      }
+      // 32 rows x 64 bytes, 64-byte swizzle: 16-byte piece j of row r at piece j ^ ((r >> 1) & 3)
+      uint8_t* rowp = ebuf + lane * 64;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int pj = j ^ ((lane >> 1) & 3);
+        *reinterpret_cast<uint4*>(rowp + pj * 16) =
+            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+      }
+    } else {
+      // 32 rows x 128 bytes, 128-byte swizzle: piece j of row r at piece j ^ (r & 7)
+      uint8_t* rowp = ebuf + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int pj = j ^ (lane & 7);
+        *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmOut, ebuf, n0, row0);
+      bulk_commit_group();
+    }
+    ++chunk_count;
+  }
+}
+
+// Fused rotate + quantise worker (warps 6.. of the fused kernel): rows
+// [pass*rpp, pass*rpp + rpp) for pass = blockIdx.x, blockIdx.x + gridDim.x, ...
+// Same thread layout and arithmetic as the standalone rotate+quantise kernel
+// (64 elements per lane, g/64 lanes per group, f32x2 butterflies, shuffles
+// across the group's lanes), reading X straight from global memory.
+template <int G>
+__device__ __forceinline__ void quant_worker(const GemmParams& p, int qtid, int nq, unsigned* rmax2,
+                                             volatile int* abort) {
+  using namespace fwht;
+  constexpr int LG = G / 64;
+  constexpr int PIECE = G / 8;
+  const int tpr = p.q_threads_per_row;
+  const int rpp = p.q_rows_per_pass;
+  const int row_in_pass = qtid / tpr;
+  const int t = qtid - row_in_pass * tpr;
+  const int grp = t / LG;
+  const int l = t - grp * LG;
+  const bool lane_active = row_in_pass < rpp;
+  int pass = 0;
+  for (int64_t gp = blockIdx.x; gp * rpp < p.M; gp += gridDim.x, ++pass) {
+    const int64_t r0 = gp * rpp;
+    const int64_t row = r0 + row_in_pass;
+    const bool valid = lane_active && row < p.M;
+    unsigned* rmax = rmax2 + (pass & 1) * kMaxFusedRows;
+    if (qtid < rpp) rmax[qtid] = 0u;
+    const int64_t base = row * p.K + static_cast<int64_t>(grp) * G + 8 * l;
+    float2 v[4][8];
+    if (valid) {
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint16_t* src = p.X + base + j * PIECE;
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(raw[j].x), "=r"(raw[j].y), "=r"(raw[j].z), "=r"(raw[j].w)
+                     : "l"(src));
+      }
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const uint32_t aw[4] = {raw[jj].x, raw[jj].y, raw[jj].z, raw[jj].w};
+        const uint32_t bw[4] = {raw[jj + 4].x, raw[jj + 4].y, raw[jj + 4].z, raw[jj + 4].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          v[jj][2 * q] = make_float2(__uint_as_float(aw[q] << 16), __uint_as_float(bw[q] << 16));
+          v[jj][2 * q + 1] =
+              make_float2(__uint_as_float(aw[q] & 0xFFFF0000u), __uint_as_float(bw[q] & 0xFFFF0000u));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[jj][e] = make_float2(0.0f, 0.0f);
+    }
+    fwht_group<G>(v, l);
+    float m = 0.0f;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fmaxf(fabsf(v[jj][e].x), fabsf(v[jj][e].y)));
+#pragma unroll
+    for (int s = 1; s < LG; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+    named_barrier_sync(1, nq);  // rmax initialised
+    if (valid && l == 0) atomicMax(&rmax[row_in_pass], __float_as_uint(m));
+    named_barrier_sync(1, nq);
+    if (valid) {
+      const QuantScale qs = make_scale<G>(__uint_as_float(rmax[row_in_pass]));
+      if (t == 0) p.x_scale_out[row] = qs.s;
+      if (qs.pre != 1.0f) {
+        const float2 pre2 = make_float2(qs.pre, qs.pre);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[jj][e] = __fmul2_rn(v[jj][e], pre2);
+      }
+      const float2 ci2 = make_float2(qs.ci, qs.ci);
+      const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+      int8_t* dst = p.Xq + base;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        float2 r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __ffma2_rn(v[jj][e], ci2, magic2);
+        uint2 lo, hi;
+        lo.x = pack4(r[0].x, r[1].x, r[2].x, r[3].x);
+        lo.y = pack4(r[4].x, r[5].x, r[6].x, r[7].x);
+        hi.x = pack4(r[0].y, r[1].y, r[2].y, r[3].y);
+        hi.y = pack4(r[4].y, r[5].y, r[6].y, r[7].y);
+        *reinterpret_cast<uint2*>(dst + jj * PIECE) = lo;
+        *reinterpret_cast<uint2*>(dst + (jj + 4) * PIECE) = hi;
+      }
+    }
+    // the codes are read by TMA (async proxy) in other CTAs
+    fence_proxy_async_global();
+    // every worker's stores of this pass are done; all workers agree on stopping
+    // early when another role of the CTA has given up
+    const bool stop = named_barrier_or(1, nq, *abort != 0);
+    if (qtid == 0) {
+      __threadfence();
+      const int64_t r1 = (r0 + rpp) < p.M ? (r0 + rpp) : p.M;
+      for (int64_t r = r0; r < r1;) {
+        const int mb = static_cast<int>(r / BM);
+        const int64_t end = (static_cast<int64_t>(mb) + 1) * BM < r1 ? (static_cast<int64_t>(mb) + 1) * BM : r1;
+        publish_rows(p, mb, static_cast<int>(end - r));
+        r = end;
+      }
+    }
+    if (stop) break;
+  }
+}
+
 }  // namespace
 
-template <int EPI>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int EPI, int FG>
+__global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   using L = Smem<EPI>;
@@ -133,6 +406,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
+  // Everything above overlaps the previous kernel (programmatic launch); its
+  // outputs (and, fused, the workspace it may still read) are touched only
+  // after this point.
+  griddep_wait();
+  if (FG != 0 && blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0;
 
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
 
@@ -147,6 +425,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         int mb, nb;
         tile_coords(tile, p, mb, nb);
+        if (FG != 0) {
+          if (!wait_block_ready(p, mb, abort)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // the codes were written by generic stores
+        }
         for (int kb = 0; kb < p.num_k_blocks; ++kb) {
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort, p.timeout_ns)) {
             ok = false;
@@ -162,6 +447,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      // all of this CTA's loads are issued: the next kernel may start launching
+      griddep_launch_dependents();
       if (!ok) {
         raise_abort(abort, p.status);
         // let every copy already issued land before the CTA's shared memory goes away
@@ -213,7 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(drain);
       mbar_wait_bounded(drain, 0u, nullptr, p.timeout_ns);
     }
-  } else {
+  } else if (warp < 2 + EPI_WARPS) {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const float sw = (EPI == kEpiDequantBf16) ? __ldg(p.w_scale) : 0.0f;
@@ -234,73 +521,243 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row0 = mb * BM + q * 32;
       const int row = row0 + lane;
       float sc = 0.0f;
+      if (FG != 0) {
+        // the token scales of this block were written in this launch: acquire, then coherent loads
+        if (!wait_block_ready(p, mb, abort)) {
+          ok = false;
+          break;
+        }
+        sc = (row < p.M ? ld_relaxed_f32(p.x_scale + row) : 0.0f) * sw;
+      } else if (EPI == kEpiDequantBf16) {
+        sc = (row < p.M ? __ldg(p.x_scale + row) : 0.0f) * sw;
+      }
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
+      epilogue_tile<EPI>(&tmOut, p, t_row, row0, nb * BN, sc, ebuf0, chunk_count, lane,
+                         [&]() { mbar_arrive(&tmem_empty[b]); });
+    }
+    if (!ok && lane == 0) raise_abort(abort, p.status);
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ fused rotate + quantise
+    if constexpr (FG != 0) {
+      unsigned* rmax2 = reinterpret_cast<unsigned*>(smem + L::kOffRowMax);
+      quant_worker<FG>(p, static_cast<int>(threadIdx.x) - NUM_THREADS, static_cast<int>(blockDim.x) - NUM_THREADS,
+                       rmax2, abort);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ===================================================== CTA-pair (2-SM) form
+//
+// Two CTAs of a cluster compute a 256x256 tile together with
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=32): CTA r of the pair loads rows
+// r*128.. of the A tile and rows r*128.. of the B tile (its half of N) into its
+// own shared memory, so per SM the operand traffic is 32 KB per 128-byte K
+// step instead of 48 KB. The leader (rank 0) issues the MMAs; its full
+// barrier collects both CTAs' TMA bytes; tcgen05.commit multicasts stage and
+// accumulator completion to both CTAs; the follower's epilogue warps release
+// the accumulator by arriving on the leader's barrier. Each CTA holds its 128
+// rows x 256 columns of the accumulator (two buffers, 512 columns), and runs
+// the same epilogue as the single-SM form on them. No TMA multicast is used.
+
+constexpr int BN_HALF = BN / 2;
+constexpr int PAIR_STAGES = 6;
+constexpr int PA_STAGE_BYTES = BM * BK;       // 16 KB: this CTA's 128 rows of A
+constexpr int PB_STAGE_BYTES = BN_HALF * BK;  // 16 KB: this CTA's 128 rows of B
+constexpr uint32_t IDESC_PAIR = idesc_i8(2 * BM, BN);
+
+template <int EPI>
+struct PairSmem {
+  static constexpr int kStages = (EPI == kEpiDequantBf16) ? PAIR_STAGES : PAIR_STAGES - 1;
+  static constexpr int kEpiBuf = (EPI == kEpiDequantBf16) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kStages * PA_STAGE_BYTES;
+  static constexpr int kOffEpi = kStages * (PA_STAGE_BYTES + PB_STAGE_BYTES);
+  static constexpr int kOffBar = kOffEpi + EPI_WARPS * 2 * kEpiBuf;
+  // full[S], empty[S], tmem_full[2], tmem_empty[2], drain, teardown
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
+  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemPtr + 8;
+  static constexpr int kBytes = kOffAbort + 8;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+__device__ __forceinline__ void pair_tile_coords(int tile, const GemmParams& p, int& mb2, int& nb) {
+  const int per_group = p.group_m * p.num_n_blocks;
+  const int grp = tile / per_group;
+  const int first_m = grp * p.group_m;
+  const int rem_m = p.num_m_blocks - first_m;  // here: 256-row blocks
+  const int gsz = rem_m < p.group_m ? rem_m : p.group_m;
+  const int r = tile - grp * per_group;
+  mb2 = first_m + r % gsz;
+  nb = r / gsz;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+  using L = PairSmem<EPI>;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tmem_full = bars + 2 * S;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* drain = tmem_empty + 2;
+  uint64_t* teardown = drain + 1;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmOut);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 2 * EPI_WARPS);  // both CTAs' epilogue warps
+    }
+    mbar_init(drain, 1);
+    mbar_init(teardown, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_ptr, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  // both CTAs' barriers exist before any remote arrive or TMA completion targets them
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_ptr;
+  griddep_wait();
+
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // pair tiles
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        int mb2, nb;
+        pair_tile_coords(tile, p, mb2, nb);
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (PA_STAGE_BYTES + PB_STAGE_BYTES));
+          const uint32_t bar_leader = map_to_rank(&full[s], 0);
+          tma_load_2d_pair(smem + L::kOffA + s * PA_STAGE_BYTES, &tmA, bar_leader, kb * BK,
+                           mb2 * 2 * BM + static_cast<int>(rank) * BM);
+          tma_load_2d_pair(smem + L::kOffB + s * PB_STAGE_BYTES, &tmB, bar_leader, kb * BK,
+                           nb * BN + static_cast<int>(rank) * BN_HALF);
+          ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      griddep_launch_dependents();
+      if (!ok) raise_abort(abort, p.status);
+      // the last stages are released (MMAs done reading this CTA's operands and
+      // their commits delivered) before this CTA may go away
+      for (int64_t k = (issued > S ? issued - S : 0); k < issued; ++k)
+        mbar_wait_bounded(&empty[k % S], static_cast<uint32_t>((k / S) & 1), nullptr, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA (leader)
+    if (lane == 0 && leader) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++it) {
+        const int b = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (!mbar_wait_bounded(&tmem_empty[b], (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&full[s], ph, abort, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(smem + L::kOffA + s * PA_STAGE_BYTES);
+          const uint32_t b_base = smem_addr(smem + L::kOffB + s * PB_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            mma_i8_pair(d, smem_desc_k_sw128(a_base + k * UMMA_K), smem_desc_k_sw128(b_base + k * UMMA_K),
+                        IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair_mc(&empty[s], 0x3);  // the stage is free in both CTAs
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&tmem_full[b], 0x3);  // both halves of the accumulator are final
+      }
+      if (!ok) raise_abort(abort, p.status);
+      mma_commit_pair_mc(drain, 0x1);
+      mbar_wait_bounded(drain, 0u, nullptr, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------ epilogue (both)
+    const int q = warp & 3;
+    const float sw = (EPI == kEpiDequantBf16) ? __ldg(p.w_scale) : 0.0f;
+    uint8_t* ebuf0 = smem + L::kOffEpi + (q * 2) * L::kEpiBuf;
+    int chunk_count = 0;
+    int it = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+      int mb2, nb;
+      pair_tile_coords(tile, p, mb2, nb);
+      const int b = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      if (!mbar_wait_bounded(&tmem_full[b], use & 1u, abort, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row0 = mb2 * 2 * BM + static_cast<int>(rank) * BM + q * 32;
+      const int row = row0 + lane;
+      float sc = 0.0f;
       if (EPI == kEpiDequantBf16) sc = (row < p.M ? __ldg(p.x_scale + row) : 0.0f) * sw;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
-#pragma unroll 1
-      for (int c = 0; c < BN / CHUNK; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * CHUNK), r);
-        tmem_ld_wait();
-        if (c == BN / CHUNK - 1) {  // accumulator fully read: hand it back to the MMA warp
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tmem_empty[b]);
-        }
-        const int n0 = nb * BN + c * CHUNK;
-        if (n0 >= p.N) continue;
-        uint8_t* ebuf = ebuf0 + (chunk_count & 1) * L::kEpiBuf;
-        if (lane == 0) bulk_wait_group_read<1>();  // the store that last read this buffer is done
-        __syncwarp();
-        if (EPI == kEpiDequantBf16) {
-          float bv[32];
-          if (p.bias != nullptr) {
-#pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
-              uint4 w = make_uint4(0u, 0u, 0u, 0u);
-              if (n0 + 8 * pc < p.N) w = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * pc));
-              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                bv[8 * pc + 2 * e] = __uint_as_float(ws[e] << 16);
-                bv[8 * pc + 2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) bv[e] = 0.0f;
-          }
-          uint32_t packed[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float y0 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e])), sc, bv[2 * e]);
-            const float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e + 1])), sc, bv[2 * e + 1]);
-            packed[e] = bf16x2(y0, y1);
-          }
-          // 32 rows x 64 bytes, 64-byte swizzle: 16-byte piece j of row r at piece j ^ ((r >> 1) & 3)
-          uint8_t* rowp = ebuf + lane * 64;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int pj = j ^ ((lane >> 1) & 3);
-            *reinterpret_cast<uint4*>(rowp + pj * 16) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
-        } else {
-          // 32 rows x 128 bytes, 128-byte swizzle: piece j of row r at piece j ^ (r & 7)
-          uint8_t* rowp = ebuf + lane * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int pj = j ^ (lane & 7);
-            *reinterpret_cast<uint4*>(rowp + pj * 16) = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmOut, ebuf, n0, row0);
-          bulk_commit_group();
-        }
-        ++chunk_count;
-      }
+      const uint32_t release_addr = map_to_rank(&tmem_empty[b], 0);
+      epilogue_tile<EPI>(&tmOut, p, t_row, row0, nb * BN, sc, ebuf0, chunk_count, lane,
+                         [&]() { mbar_arrive_cluster(release_addr); });
     }
     if (!ok && lane == 0) raise_abort(abort, p.status);
     if (lane == 0) bulk_wait_group<0>();
@@ -309,8 +766,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   __syncthreads();
   if (warp == 1) {
+    // both CTAs are done with the pair's TMEM and with each other's barriers
+    if (lane == 0) {
+      mbar_arrive_cluster(map_to_rank(teardown, rank ^ 1u));
+      mbar_wait_bounded(teardown, 0u, nullptr, p.timeout_ns);
+    }
+    __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -342,14 +805,36 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int elem_bytes, const vo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr int kMaxDevices = 64;
+
+// SM count of the current device, looked up once per device.
 int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < kMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
-template <int EPI>
+// cudaFuncSetAttribute(max dynamic shared memory) once per device and kernel.
+template <class Kernel>
+cudaError_t ensure_smem_attr(Kernel kern, int bytes, std::atomic<int>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(bytes, std::memory_order_release);
+  return e;
+}
+
+template <int EPI, int FG>
 cudaError_t launch_impl(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
   CUtensorMap ta, tb, to;
   if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, p.K, p.M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -365,24 +850,105 @@ cudaError_t launch_impl(const int8_t* A, const int8_t* B, void* out, GemmParams 
   p.num_m_blocks = (p.M + BM - 1) / BM;
   p.num_n_blocks = (p.N + BN - 1) / BN;
   p.num_k_blocks = (p.K + BK - 1) / BK;
-  if (p.group_m <= 0) p.group_m = 16;
+  if (p.group_m <= 0) p.group_m = FG ? 4 : 16;
+  int threads = NUM_THREADS;
+  if (FG != 0) {
+    if (!fused_shape(p.K, &p.q_threads_per_row, &p.q_rows_per_pass, &threads)) return cudaErrorInvalidValue;
+  }
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int grid = tiles < sms ? tiles : sms;
   constexpr int smem = Smem<EPI>::kAlloc;
-  cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<int> attr_done[kMaxDevices];
+  cudaError_t e = ensure_smem_attr(gemm_i8_kernel<EPI, FG>, smem, attr_done);
   if (e != cudaSuccess) return e;
-  gemm_i8_kernel<EPI><<<grid, NUM_THREADS, smem, stream>>>(ta, tb, to, p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_kernel<EPI, FG>, ta, tb, to, p);
+}
+
+}  // namespace
+
+bool fused_shape(int64_t K, int* threads_per_row, int* rows_per_pass, int* cta_threads) {
+  if (K <= 0 || K % 128 != 0) return false;
+  const int64_t tpr = K / 64;
+  if (tpr > 32 * (kFusedMaxThreads - NUM_THREADS) / 32) return false;
+  int64_t rpp = 256 / tpr;
+  if (rpp < 1) rpp = 1;
+  if (rpp > kMaxFusedRows) rpp = kMaxFusedRows;
+  const int64_t workers = (rpp * tpr + 31) / 32 * 32;
+  if (NUM_THREADS + workers > kFusedMaxThreads) return false;
+  *threads_per_row = static_cast<int>(tpr);
+  *rows_per_pass = static_cast<int>(rpp);
+  *cta_threads = static_cast<int>(NUM_THREADS + workers);
+  return true;
+}
+
+namespace {
+
+template <int EPI>
+cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
+  CUtensorMap ta, tb, to;
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, p.K, p.M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, BN_HALF, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  bool ok_out;
+  if (EPI == kEpiDequantBf16)
+    ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  else
+    ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok_out) return cudaErrorInvalidValue;
+  p.num_m_blocks = (p.M + 2 * BM - 1) / (2 * BM);  // 256-row pair blocks
+  p.num_n_blocks = (p.N + BN - 1) / BN;
+  p.num_k_blocks = (p.K + BK - 1) / BK;
+  if (p.group_m <= 0) p.group_m = 8;
+  const int tiles = p.num_m_blocks * p.num_n_blocks;
+  const int sms = sm_count();
+  if (sms < 2) return cudaErrorInvalidDevice;
+  const int pairs = tiles < sms / 2 ? tiles : sms / 2;
+  constexpr int smem = PairSmem<EPI>::kAlloc;
+  static std::atomic<int> attr_done[kMaxDevices];
+  cudaError_t e = ensure_smem_attr(gemm_i8_pair_kernel<EPI>, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_pair_kernel<EPI>, ta, tb, to, p);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out, GemmParams p,
                            cudaStream_t stream) {
-  if (epi == kEpiDequantBf16) return launch_impl<kEpiDequantBf16>(A, B, out, p, stream);
-  if (epi == kEpiRawS32) return launch_impl<kEpiRawS32>(A, B, out, p, stream);
+  if (p.single_sm == 0) {
+    if (epi == kEpiDequantBf16) return launch_pair<kEpiDequantBf16>(A, B, out, p, stream);
+    if (epi == kEpiRawS32) return launch_pair<kEpiRawS32>(A, B, out, p, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (epi == kEpiDequantBf16) return launch_impl<kEpiDequantBf16, 0>(A, B, out, p, stream);
+  if (epi == kEpiRawS32) return launch_impl<kEpiRawS32, 0>(A, B, out, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_linear_fused(int g, const int8_t* Wq, void* Y, GemmParams p, cudaStream_t stream) {
+  if (g == 256) return launch_impl<kEpiDequantBf16, 256>(p.Xq, Wq, Y, p, stream);
+  if (g == 128) return launch_impl<kEpiDequantBf16, 128>(p.Xq, Wq, Y, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -20,12 +20,33 @@ struct GemmParams {
   int* status;            // status word: a timed-out wait ORs 5 into it
   uint64_t timeout_ns;    // bound of every device-side wait
   int group_m;            // M-blocks per raster group (0 = default)
+  int single_sm;          // 1: one-CTA tiles (128x256); 0: CTA-pair tiles (256x256, cta_group::2)
   int num_m_blocks, num_n_blocks, num_k_blocks;  // filled by the launcher
+  // fused form (launch_linear_fused): the kernel also rotates and quantises X
+  const uint16_t* X;              // [M,K] bf16 bits
+  int8_t* Xq;                     // [M,K] codes (the A operand)
+  float* x_scale_out;             // [M] token scales (same buffer as x_scale)
+  unsigned long long* ready;      // [num_m_blocks] epoch << 32 | rows quantised
+  uint32_t epoch;                 // unique per call, never 0
+  int q_threads_per_row, q_rows_per_pass;  // filled by the launcher
 };
+
+constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass
+
+// Worker layout of the fused kernel for a given K; false if K is not a
+// multiple of 128 or too large for one CTA's worker warps (then the layer runs
+// as two kernels).
+bool fused_shape(int64_t K, int* threads_per_row, int* rows_per_pass, int* cta_threads);
 
 // A = Xq [M,K] int8, B = Wq [N,K] int8, out = Y [M,N] bf16 or acc [M,N] int32.
 cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out, GemmParams p,
                            cudaStream_t stream);
+
+// The whole ConvRot linear layer in one launch: p.X is rotated and quantised
+// into p.Xq / p.x_scale_out by worker warps while the GEMM consumes finished
+// M-blocks. p.ready holds num_m_blocks counters; p.epoch must differ from
+// every earlier call's epoch on the same workspace.
+cudaError_t launch_linear_fused(int g, const int8_t* Wq, void* Y, GemmParams p, cudaStream_t stream);
 
 // One CTA waits on a barrier that nothing completes, for at most timeout_ns,
 // then ORs 5 into *status.

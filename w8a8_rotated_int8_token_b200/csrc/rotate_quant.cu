@@ -6,213 +6,229 @@
 // whole tensor, found by a first pass over all rows (InvokeAI "int8 Compute"
 // page: input rotated and quantised per token, weights int8_tensorwise).
 //
-// Thread layout. A token row of K elements is K/g groups. A group of g
-// elements is owned by LG = g/32 consecutive lanes, 32 elements per lane:
-// lane l of the group loads four 16-byte pieces at group offsets
-// j*(g/4) + 8*l (j = 0..3). With i = 64*j + 8*l + e (g = 256) the element
-// index bits split as e (bits 0-2, inside one 16-byte piece), l (lane bits)
-// and j (top two bits), so five butterfly stages run in registers and
-// log2(LG) stages (3 for g=256, 2 for g=128) run across lanes with shuffles. Each warp
-// load instruction covers LG*16-byte contiguous runs, fully coalesced.
-// A CTA holds `rpc` whole rows (K/32 threads per row); the row absmax is
-// reduced in shared memory. The transform is computed unnormalised in float32
-// and the 1/sqrt(g) factor is folded into the scale.
+// Thread layout. A token row of K elements is K/g groups. A group is owned by
+// LG = g/64 consecutive lanes, 64 elements per lane: lane l of the group loads
+// eight 16-byte pieces at group offsets j*(g/8) + 8*l (j = 0..7), so one warp
+// load instruction reads LG*16 contiguous bytes per group, fully coalesced.
+// The group index bits split as e (bits 0-2, inside a piece), l (log2 LG lane
+// bits) and j (top three bits): six butterfly stages run in registers and one
+// (g=128) or two (g=256) across lanes with shuffles.
+//
+// Arithmetic is packed: the 64 values live as 32 float2 pairs (piece j, piece
+// j+4), so every butterfly stage except the one on j's top bit is one f32x2
+// add or fma per two butterflies; that stage is done on scalars. The transform
+// is computed unnormalised in float32 and 1/sqrt(g) is folded into the scale.
+// A CTA handles `rpc` whole rows at a time (K/64 threads per row) and loops
+// over row blocks (persistent grid); one thread keeps kRqStages row blocks in
+// flight with bulk asynchronous copies into shared memory, so the memory
+// parallelism does not depend on how many warps fit. The row absmax is reduced
+// in shared memory.
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
+#include "fwht_dev.cuh"
+#include "ptx_sm100.cuh"
 #include "rotate_quant.cuh"
 
 namespace convrot {
 
-namespace {
+using namespace fwht;
 
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer (ties to even)
-
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint4 load_streaming(const uint16_t* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-// Unnormalised Walsh-Hadamard transform of one group held as v[j][e] by the
-// LG lanes of the group (see the file comment for the index split).
-template <int G>
-__device__ __forceinline__ void fwht_group(float (&v)[4][8], int l) {
-  // bits 0..2: inside each 16-byte piece
-#pragma unroll
-  for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if ((e & h) == 0) {
-          const float a = v[j][e], b = v[j][e + h];
-          v[j][e] = a + b;
-          v[j][e + h] = a - b;
-        }
-      }
-    }
-  }
-  // top two bits: across the four pieces of this lane
-#pragma unroll
-  for (int h = 1; h < 4; h <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if ((j & h) == 0) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a = v[j][e], b = v[j + h][e];
-          v[j][e] = a + b;
-          v[j + h][e] = a - b;
-        }
-      }
-    }
-  }
-  // middle bits: across the LG lanes of the group. The lower partner keeps
-  // a + b, the upper one b_partner - own = a - b.
-  constexpr int LG = G / 32;
-#pragma unroll
-  for (int m = 1; m < LG; m <<= 1) {
-    const float sgn = (l & m) ? -1.0f : 1.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float p = __shfl_xor_sync(0xFFFFFFFFu, v[j][e], m);
-        v[j][e] = fmaf(sgn, v[j][e], p);
-      }
-    }
-  }
-}
-
-// The scale of a row (or tensor) from the absmax of its unnormalised
-// transform, and the factor that maps an unnormalised value to code units.
-struct QuantScale {
-  float s;        // stored scale: float32(absmax(X R) / 127)
-  float ci;       // code = rne(u * ci) for an unnormalised value u (after `pre`)
-  float pre;      // 1, or 2^64 for rows whose scale is below 2^-100
-};
-
-template <int G>
-__device__ __forceinline__ QuantScale make_scale(float amax_u) {
-  // 1/sqrt(g) and 127*sqrt(g): exact for g = 256 (1/16 and 2032); nearest
-  // floats for g = 128. The scale takes one rounding for g = 256:
-  // s = absmax(X R)/127 = absmax_u / (127 sqrt(g)).
-  const float cg = (G == 256) ? 0.0625f : 0.0883883461356163f;
-  const float div = (G == 256) ? 2032.0f : 1436.8409423828125f;
-  QuantScale q;
-  q.s = amax_u / div;
-  q.pre = 1.0f;
-  if (q.s == 0.0f) {
-    q.ci = 0.0f;
-  } else if (q.s >= 0x1p-100f) {
-    q.ci = cg * (1.0f / q.s);
-  } else {  // tiny row: lift by 2^64 (exact) so that 1/s cannot overflow
-    q.pre = 0x1p64f;
-    q.ci = cg * (1.0f / (q.s * 0x1p64f));
-  }
-  return q;
-}
-
-__device__ __forceinline__ uint32_t pack4(float a, float b, float c, float d, float ci) {
-  // low byte of (u*ci + magic) is the two's-complement int8 code of rne(u*ci)
-  const uint32_t qa = __float_as_uint(fmaf(a, ci, kRoundMagic));
-  const uint32_t qb = __float_as_uint(fmaf(b, ci, kRoundMagic));
-  const uint32_t qc = __float_as_uint(fmaf(c, ci, kRoundMagic));
-  const uint32_t qd = __float_as_uint(fmaf(d, ci, kRoundMagic));
-  const uint32_t ab = __byte_perm(qa, qb, 0x0040);
-  const uint32_t cd = __byte_perm(qc, qd, 0x0040);
-  return __byte_perm(ab, cd, 0x5410);
-}
-
-}  // namespace
 
 template <int G, int MODE>
-__global__ void __launch_bounds__(1024) rotate_quant_kernel(RotQuantParams p) {
-  constexpr int LG = G / 32;
-  __shared__ unsigned row_max[kMaxRowsPerCta];
+__global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
+  constexpr int LG = G / 64;
+  constexpr int PIECE = G / 8;  // elements between consecutive pieces of a lane
+  extern __shared__ __align__(128) uint8_t stage_mem[];  // kRqStages x (rows_per_cta x K) bf16
+  __shared__ uint64_t full[kRqStages];
+  __shared__ unsigned row_max[2][kMaxRowsPerCta];
+  __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
-  const int row_in_cta = tid / p.threads_per_row;
+  const int rpc = p.rows_per_cta;
+  const int row_in_cta = tid / p.threads_per_row;  // >= rpc for the padding threads of the last warp
   const int t = tid - row_in_cta * p.threads_per_row;
   const int grp = t / LG;
   const int l = t - grp * LG;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * p.rows_per_cta + row_in_cta;
-  const bool valid = row < p.rows;
+  const bool lane_active = row_in_cta < rpc;
+  // Group k reads its pieces in the order j ^ (k mod F), F = 2 (g=256) or 4
+  // (g=128), so that the F groups sharing a 128-byte bank window hit
+  // different banks. The transform then comes out with piece r multiplied by
+  // (-1)^popcount(r & flip), which the quantisation multiplier undoes.
+  constexpr int F = (G == 256) ? 2 : 4;
+  const int flip = grp & (F - 1);
+  const int64_t nblocks = (p.rows + rpc - 1) / rpc;
+  const uint32_t stage_bytes = static_cast<uint32_t>(rpc) * static_cast<uint32_t>(p.K) * 2u;
 
-  if (tid < p.rows_per_cta) row_max[tid] = 0u;
+  if (tid == 0) {
+    for (int s = 0; s < kRqStages; ++s) mbar_init(&full[s], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // The input may be the previous kernel's output: wait for it (launches are
+  // programmatic), then let the next kernel start its prologue early.
+  griddep_wait();
+  griddep_launch_dependents();
   if (MODE == kRqActivation && p.status_reset != nullptr && blockIdx.x == 0 && tid == 0) *p.status_reset = 0;
 
-  float v[4][8];
-  const int64_t base = row * p.K + static_cast<int64_t>(grp) * G + 8 * l;
-  if (valid) {
-    uint4 raw[4];
+  // the producer (thread 0) keeps kRqStages row blocks of this CTA in flight
+  int64_t issued = 0;
+  auto issue = [&](int64_t it) {
+    const int64_t blk = blockIdx.x + it * gridDim.x;
+    if (blk >= nblocks) return;
+    const int64_t r0 = blk * rpc;
+    const int64_t nrows = (p.rows - r0) < rpc ? (p.rows - r0) : rpc;
+    const uint32_t bytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(p.K) * 2u;
+    const int slot = static_cast<int>(it % kRqStages);
+    mbar_arrive_expect_tx(&full[slot], bytes);
+    bulk_load(stage_mem + static_cast<size_t>(slot) * stage_bytes, p.src + r0 * p.K, bytes, &full[slot]);
+    issued = it + 1;
+  };
+  if (tid == 0)
+    for (int s = 0; s < kRqStages; ++s) issue(s);
+
+  int64_t it = 0;
+  bool timed_out = false;
+  for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x, ++it) {
+    const int slot = static_cast<int>(it % kRqStages);
+    const uint32_t ph = static_cast<uint32_t>((it / kRqStages) & 1);
+    const int64_t row = blk * rpc + row_in_cta;
+    const bool valid = lane_active && row < p.rows;
+    unsigned* rmax = row_max[it & 1];
+    if (tid < rpc) rmax[tid] = 0u;
+
+    const bool ok = mbar_wait_bounded(&full[slot], ph, &abort_flag, p.timeout_ns);
+    uint8_t* slot_mem = stage_mem + static_cast<size_t>(slot) * stage_bytes;
+    float2 v[4][8];
+    if (valid) {
+      const uint8_t* src =
+          slot_mem + (static_cast<size_t>(row_in_cta) * p.K + static_cast<size_t>(grp) * G + 8 * l) * 2;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) raw[j] = load_streaming(p.src + base + j * (G / 4));
+      for (int jj = 0; jj < 4; ++jj) {
+        const uint4 a = *reinterpret_cast<const uint4*>(src + ((jj ^ flip) * PIECE) * 2);
+        const uint4 b = *reinterpret_cast<const uint4*>(src + (((jj + 4) ^ flip) * PIECE) * 2);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+        for (int q = 0; q < 4; ++q) {
+          v[jj][2 * q] = make_float2(__uint_as_float(aw[q] << 16), __uint_as_float(bw[q] << 16));
+          v[jj][2 * q + 1] =
+              make_float2(__uint_as_float(aw[q] & 0xFFFF0000u), __uint_as_float(bw[q] & 0xFFFF0000u));
+        }
+      }
+    } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        v[j][2 * q] = bf16lo(w[q]);
-        v[j][2 * q + 1] = bf16hi(w[q]);
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[jj][e] = make_float2(0.0f, 0.0f);
+    }
+
+    float m = 0.0f;
+    float2 w[2][16];  // g = 256: the lane's values after the exchange
+    if constexpr (G == 256) {
+      fwht256_in_lane(v);
+      fwht256_exchange(v, w, slot_mem + static_cast<size_t>(tid >> 5) * 4096, (tid >> 2) & 7, l, lane_active);
+      fwht256_after_exchange(w);
+#pragma unroll
+      for (int b7 = 0; b7 < 2; ++b7)
+#pragma unroll
+        for (int q = 0; q < 16; ++q) m = fmaxf(m, fmaxf(fabsf(w[b7][q].x), fabsf(w[b7][q].y)));
+    } else {
+      fwht_group<G>(v, l);  // all lanes take part in the shuffles
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fmaxf(fabsf(v[jj][e].x), fabsf(v[jj][e].y)));
+    }
+#pragma unroll
+    for (int s = 1; s < LG; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+
+    // every thread has its data in registers: the slot may be refilled
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
+    if (tid == 0) issue(it + kRqStages);
+    // non-negative floats order like their bit patterns
+    if (valid && l == 0) atomicMax(&rmax[row_in_cta], __float_as_uint(m));
+    __syncthreads();
+
+    if (MODE == kRqWeightAbsmax) {
+      if (valid && t == 0) atomicMax(p.tensor_absmax, rmax[row_in_cta]);
+      continue;
+    }
+    const float amax_u =
+        (MODE == kRqActivation) ? __uint_as_float(rmax[row_in_cta]) : __uint_as_float(*p.tensor_absmax);
+    const QuantScale qs = make_scale<G>(amax_u);
+    if (MODE == kRqActivation) {
+      if (valid && t == 0) p.scale[row] = qs.s;
+    } else {
+      if (blk == 0 && tid == 0) *p.scale = qs.s;
+    }
+    if (!valid) continue;
+    const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+    int8_t* dst = p.dst + row * p.K + static_cast<int64_t>(grp) * G;
+    if constexpr (G == 256) {
+      // the lane holds elements 128*b7 + 32*l + (0..31); the piece-order flip
+      // of the input left them multiplied by (-1)^(flip & bit 5) = (-1)^(flip & l)
+      const float ci = (flip & l & 1) ? -qs.ci : qs.ci;
+      const float2 ci2 = make_float2(ci, ci);
+      const float2 pre2 = make_float2(qs.pre, qs.pre);
+      const bool lifted = qs.pre != 1.0f;
+#pragma unroll
+      for (int b7 = 0; b7 < 2; ++b7) {
+        uint32_t word[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float2 a = w[b7][2 * k], b = w[b7][2 * k + 1];
+          if (lifted) {  // tiny row: multiply by 2^64 first (exact), then by ci
+            a = __fmul2_rn(a, pre2);
+            b = __fmul2_rn(b, pre2);
+          }
+          const float2 ra = __ffma2_rn(a, ci2, magic2);
+          const float2 rb = __ffma2_rn(b, ci2, magic2);
+          word[k] = pack4(ra.x, ra.y, rb.x, rb.y);
+        }
+        int8_t* o = dst + 128 * b7 + 32 * l;
+        *reinterpret_cast<uint4*>(o) = make_uint4(word[0], word[1], word[2], word[3]);
+        *reinterpret_cast<uint4*>(o + 16) = make_uint4(word[4], word[5], word[6], word[7]);
+      }
+    } else {
+      if (qs.pre != 1.0f) {
+        const float2 pre2 = make_float2(qs.pre, qs.pre);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[jj][e] = __fmul2_rn(v[jj][e], pre2);
+      }
+      int8_t* d8 = dst + 8 * l;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const float cij = (__popc(jj & flip) & 1) ? -qs.ci : qs.ci;
+        const float2 ci2 = make_float2(cij, cij);
+        float2 r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __ffma2_rn(v[jj][e], ci2, magic2);
+        // piece jj from the .x halves, piece jj+4 from the .y halves
+        uint2 lo, hi;
+        lo.x = pack4(r[0].x, r[1].x, r[2].x, r[3].x);
+        lo.y = pack4(r[4].x, r[5].x, r[6].x, r[7].x);
+        hi.x = pack4(r[0].y, r[1].y, r[2].y, r[3].y);
+        hi.y = pack4(r[4].y, r[5].y, r[6].y, r[7].y);
+        *reinterpret_cast<uint2*>(d8 + jj * PIECE) = lo;
+        *reinterpret_cast<uint2*>(d8 + (jj + 4) * PIECE) = hi;
       }
     }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[j][e] = 0.0f;
   }
-
-  fwht_group<G>(v, l);  // all lanes take part in the shuffles
-
-  float m = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[j][e]));
-#pragma unroll
-  for (int s = 1; s < LG; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
-
-  __syncthreads();  // row_max initialised
-  // non-negative floats order like their bit patterns
-  if (valid && l == 0) atomicMax(&row_max[row_in_cta], __float_as_uint(m));
-  __syncthreads();
-
-  if (MODE == kRqWeightAbsmax) {
-    if (valid && t == 0) atomicMax(p.tensor_absmax, row_max[row_in_cta]);
-    return;
-  }
-
-  const float amax_u =
-      (MODE == kRqActivation) ? __uint_as_float(row_max[row_in_cta]) : __uint_as_float(*p.tensor_absmax);
-  const QuantScale qs = make_scale<G>(amax_u);
-  if (MODE == kRqActivation) {
-    if (valid && t == 0) p.scale[row] = qs.s;
-  } else {
-    if (blockIdx.x == 0 && tid == 0) *p.scale = qs.s;
-  }
-  if (!valid) return;
-  if (qs.pre != 1.0f) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[j][e] *= qs.pre;
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint2 out;
-    out.x = pack4(v[j][0], v[j][1], v[j][2], v[j][3], qs.ci);
-    out.y = pack4(v[j][4], v[j][5], v[j][6], v[j][7], qs.ci);
-    *reinterpret_cast<uint2*>(p.dst + base + j * (G / 4)) = out;
+  if (timed_out && tid == 0) {
+    if (p.status != nullptr) atomicOr(p.status, kRqTimeoutStatus);
+    // let the copies already issued land before the shared memory goes away
+    for (int64_t k = it; k < issued; ++k)
+      mbar_wait_bounded(&full[k % kRqStages], static_cast<uint32_t>((k / kRqStages) & 1), nullptr, p.timeout_ns);
   }
 }
 
@@ -220,37 +236,92 @@ __global__ void __launch_bounds__(1024) rotate_quant_kernel(RotQuantParams p) {
 
 bool rotquant_shape(int64_t K, int* threads_per_row, int* rows_per_cta) {
   if (K <= 0 || K % 128 != 0 || K > 32768) return false;
-  const int tpr = static_cast<int>(K / 32);
-  int rpc = (256 + tpr - 1) / tpr;
+  const int tpr = static_cast<int>(K / 64);
+  int rpc = (192 + tpr / 2) / tpr;
   if (rpc < 1) rpc = 1;
-  while ((rpc * tpr) % 32 != 0) ++rpc;
-  if (rpc * tpr > 1024 || rpc > kMaxRowsPerCta) return false;
+  if (rpc > kMaxRowsPerCta) rpc = kMaxRowsPerCta;
+  if ((rpc * tpr + 31) / 32 * 32 > kRotQuantMaxThreads) return false;
   *threads_per_row = tpr;
   *rows_per_cta = rpc;
   return true;
 }
+
+namespace {
+
+template <int G, int MODE>
+cudaError_t launch_typed(RotQuantParams p, cudaStream_t stream) {
+  void (*kern)(RotQuantParams) = rotate_quant_kernel<G, MODE>;
+  const int threads = (p.rows_per_cta * p.threads_per_row + 31) / 32 * 32;
+  const size_t smem = static_cast<size_t>(kRqStages) * p.rows_per_cta * p.K * 2;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  // per device and kernel: the largest dynamic shared memory set so far, and
+  // the occupancy found for the last (threads, smem) shape
+  constexpr int kDevs = 64;
+  static std::atomic<int> smem_set[kDevs];
+  static std::atomic<long long> occ_key[kDevs];
+  static std::atomic<int> occ_val[kDevs];
+  static std::atomic<int> sm_cache[kDevs];
+  const bool cacheable = dev >= 0 && dev < kDevs;
+  if (!cacheable || smem_set[dev].load(std::memory_order_acquire) < static_cast<int>(smem)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (cacheable) smem_set[dev].store(static_cast<int>(smem), std::memory_order_release);
+  }
+  const long long key = (static_cast<long long>(threads) << 32) | static_cast<long long>(smem);
+  int per_sm = 0;
+  if (cacheable && occ_key[dev].load(std::memory_order_acquire) == key) {
+    per_sm = occ_val[dev].load(std::memory_order_relaxed);
+  } else {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (cacheable) {
+      occ_val[dev].store(per_sm, std::memory_order_relaxed);
+      occ_key[dev].store(key, std::memory_order_release);
+    }
+  }
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  int sms = cacheable ? sm_cache[dev].load(std::memory_order_relaxed) : 0;
+  if (sms <= 0) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if (cacheable) sm_cache[dev].store(sms, std::memory_order_relaxed);
+  }
+  const int64_t nblocks = (p.rows + p.rows_per_cta - 1) / p.rows_per_cta;
+  const int64_t grid = nblocks < static_cast<int64_t>(sms) * per_sm ? nblocks : static_cast<int64_t>(sms) * per_sm;
+  // programmatic stream serialisation: the kernel waits for its predecessor
+  // itself (griddepcontrol.wait), so its launch can overlap the predecessor's tail
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+}  // namespace
 
 cudaError_t launch_rotate_quant(int g, int mode, RotQuantParams p, cudaStream_t stream) {
   int tpr = 0, rpc = 0;
   if (!rotquant_shape(p.K, &tpr, &rpc)) return cudaErrorInvalidValue;
   p.threads_per_row = tpr;
   p.rows_per_cta = rpc;
-  const int64_t ctas = (p.rows + rpc - 1) / rpc;
-  if (ctas > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(ctas));
-  const dim3 block(static_cast<unsigned>(rpc * tpr));
   if (g == 256) {
-    if (mode == kRqActivation) rotate_quant_kernel<256, kRqActivation><<<grid, block, 0, stream>>>(p);
-    else if (mode == kRqWeightAbsmax) rotate_quant_kernel<256, kRqWeightAbsmax><<<grid, block, 0, stream>>>(p);
-    else rotate_quant_kernel<256, kRqWeightQuant><<<grid, block, 0, stream>>>(p);
-  } else if (g == 128) {
-    if (mode == kRqActivation) rotate_quant_kernel<128, kRqActivation><<<grid, block, 0, stream>>>(p);
-    else if (mode == kRqWeightAbsmax) rotate_quant_kernel<128, kRqWeightAbsmax><<<grid, block, 0, stream>>>(p);
-    else rotate_quant_kernel<128, kRqWeightQuant><<<grid, block, 0, stream>>>(p);
-  } else {
-    return cudaErrorInvalidValue;
+    if (mode == kRqActivation) return launch_typed<256, kRqActivation>(p, stream);
+    if (mode == kRqWeightAbsmax) return launch_typed<256, kRqWeightAbsmax>(p, stream);
+    return launch_typed<256, kRqWeightQuant>(p, stream);
   }
-  return cudaGetLastError();
+  if (g == 128) {
+    if (mode == kRqActivation) return launch_typed<128, kRqActivation>(p, stream);
+    if (mode == kRqWeightAbsmax) return launch_typed<128, kRqWeightAbsmax>(p, stream);
+    return launch_typed<128, kRqWeightQuant>(p, stream);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace convrot

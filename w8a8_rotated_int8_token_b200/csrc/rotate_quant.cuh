@@ -14,6 +14,9 @@ enum RotQuantMode : int {
 };
 
 constexpr int kMaxRowsPerCta = 256;
+constexpr int kRqStages = 3;          // row blocks in flight per CTA
+constexpr int kRqTimeoutStatus = 5;   // CONVROT_ERR_DEVICE_TIMEOUT
+constexpr int kRotQuantMaxThreads = 512;  // K/64 threads per row: K <= 32768
 
 struct RotQuantParams {
   const uint16_t* src;      // [rows, K] bf16 bits
@@ -23,12 +26,15 @@ struct RotQuantParams {
   float* scale;             // [rows] (activation) or [1] (weight)
   unsigned* tensor_absmax;  // weight modes: float bits of the unnormalised absmax
   int* status_reset;        // activation mode: status word zeroed by CTA 0, or null
+  int* status;              // a timed-out wait ORs 5 into it (may be null)
+  uint64_t timeout_ns;      // bound of every device-side wait
   int threads_per_row;      // filled by launch_rotate_quant
   int rows_per_cta;         // filled by launch_rotate_quant
 };
 
-// Threads per row (K/32) and rows per CTA for a given K; false if K is not a
-// multiple of 128 or above 32768.
+// Threads per row (K/64) and rows per CTA for a given K; false if K is not a
+// multiple of 128 or above 32768. The CTA has rows*K/64 threads rounded up to
+// whole warps; the padding threads hold zeros.
 bool rotquant_shape(int64_t K, int* threads_per_row, int* rows_per_cta);
 
 cudaError_t launch_rotate_quant(int g, int mode, RotQuantParams p, cudaStream_t stream);
