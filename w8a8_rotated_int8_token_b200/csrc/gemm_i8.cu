@@ -568,7 +568,13 @@ __global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
 // the same epilogue as the single-SM form on them. No TMA multicast is used.
 
 constexpr int BN_HALF = BN / 2;
-constexpr int PAIR_STAGES = 6;
+#ifndef CONVROT_PAIR_STAGES
+#define CONVROT_PAIR_STAGES 6
+#endif
+#ifndef CONVROT_PAIR_GROUP_M
+#define CONVROT_PAIR_GROUP_M 8
+#endif
+constexpr int PAIR_STAGES = CONVROT_PAIR_STAGES;
 constexpr int PA_STAGE_BYTES = BM * BK;       // 16 KB: this CTA's 128 rows of A
 constexpr int PB_STAGE_BYTES = BN_HALF * BK;  // 16 KB: this CTA's 128 rows of B
 constexpr uint32_t IDESC_PAIR = idesc_i8(2 * BM, BN);
@@ -651,9 +657,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // pair tiles
+  if (warp == 0 && lane == 0 && pair < num_tiles) {
+    // the weight does not come from the previous kernel in a forward pass:
+    // start pulling this CTA's first B panel into L2 while that kernel finishes
+    int mb2, nb;
+    pair_tile_coords(pair, p, mb2, nb);
+    const int nk = p.num_k_blocks < 32 ? p.num_k_blocks : 32;
+    for (int kb = 0; kb < nk; ++kb) tma_prefetch_2d(&tmB, kb * BK, nb * BN + static_cast<int>(rank) * BN_HALF);
+  }
   griddep_wait();
 
-  const int num_tiles = p.num_m_blocks * p.num_n_blocks;  // pair tiles
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -774,6 +788,211 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// ===================================================== small-M (swap-AB) form
+//
+// For at most 128 tokens the layer is bound by streaming the int8 weight. The
+// MMA then takes the weight as its M side (128 weight rows per tile) and the
+// tokens as its N side (16..128): D[n][m] = sum_k Wq[n][k] Xq[m][k]. One CTA
+// per 128 weight rows streams its 128 x K panel through a deep TMA ring (the
+// activation codes are tiny and stay in L2); the panel is prefetched into L2
+// before waiting on the previous kernel, so the weight streams while the
+// rotate+quantise kernel runs. TMEM lane n holds weight row n, so the
+// epilogue writes Y[m][n] with 32 consecutive n per warp store.
+
+constexpr int SM_BW = 128;  // weight rows per tile
+
+template <int BNT>
+struct SmallSmem {
+  static constexpr int kW = SM_BW * BK;  // 16 KB
+  static constexpr int kX = BNT * BK;    // 2..16 KB
+  static constexpr int kFit = (200 * 1024) / (kW + kX);
+#ifdef CONVROT_SMALLM_STAGES
+  static constexpr int kStages = CONVROT_SMALLM_STAGES < kFit ? CONVROT_SMALLM_STAGES : kFit;
+#else
+  static constexpr int kStages = kFit > 10 ? 10 : kFit;
+#endif
+  static constexpr int kOffW = 0;
+  static constexpr int kOffX = kStages * kW;
+  static constexpr int kOffBar = kStages * (kW + kX);
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;
+  static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemPtr + 8;
+  static constexpr int kBytes = kOffAbort + 8;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int EPI, int BNT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_i8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                          void* __restrict__ out, const int8_t* __restrict__ Wq, const GemmParams p) {
+  using L = SmallSmem<BNT>;
+  constexpr int S = L::kStages;
+  constexpr uint32_t kIdesc = idesc_i8(SM_BW, BNT);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tmem_full = bars + 2 * S;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* drain = tmem_empty + 2;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = (p.N + SM_BW - 1) / SM_BW;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_ptr, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_ptr;
+  griddep_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int pending_phase[S];
+      for (int i = 0; i < S; ++i) pending_phase[i] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L::kW + L::kX);
+          tma_load_2d(smem + L::kOffW + s * L::kW, &tmW, &full[s], kb * BK, tile * SM_BW);
+          tma_load_2d(smem + L::kOffX + s * L::kX, &tmX, &full[s], kb * BK, 0);
+          pending_phase[s] = static_cast<int>(ph);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      griddep_launch_dependents();
+      if (!ok) {
+        raise_abort(abort, p.status);
+        for (int i = 0; i < S; ++i)
+          if (pending_phase[i] >= 0)
+            mbar_wait_bounded(&full[i], static_cast<uint32_t>(pending_phase[i]), nullptr, p.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int b = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (!mbar_wait_bounded(&tmem_empty[b], (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(b * 128);
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&full[s], ph, abort, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t w_base = smem_addr(smem + L::kOffW + s * L::kW);
+          const uint32_t x_base = smem_addr(smem + L::kOffX + s * L::kX);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            mma_i8(d, smem_desc_k_sw128(w_base + k * UMMA_K), smem_desc_k_sw128(x_base + k * UMMA_K), kIdesc,
+                   (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tmem_full[b]);
+      }
+      if (!ok) raise_abort(abort, p.status);
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0u, nullptr, p.timeout_ns);
+    }
+  } else {
+    const int q = warp & 3;
+    const float sw = (EPI == kEpiDequantBf16) ? __ldg(p.w_scale) : 0.0f;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int b = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int n = tile * SM_BW + q * 32 + lane;
+      float bn = 0.0f;
+      if (EPI == kEpiDequantBf16 && p.bias != nullptr && n < p.N) bn = __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16);
+      if (!mbar_wait_bounded(&tmem_full[b], use & 1u, abort, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * 128);
+#pragma unroll 1
+      for (int c = 0; c < BNT / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(c * 16), r);
+        tmem_ld_wait();
+        if (c == BNT / 16 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tmem_empty[b]);
+        }
+        if (n >= p.N) continue;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = c * 16 + j;
+          if (m >= p.M) break;
+          if (EPI == kEpiDequantBf16) {
+            const float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * sw, bn);
+            const __nv_bfloat16 h = __float2bfloat16_rn(y);
+            static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = h;
+          } else {
+            static_cast<int32_t*>(out)[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[j]);
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) raise_abort(abort, p.status);
+    __syncwarp();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
   }
 }
 
@@ -910,7 +1129,7 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
   p.num_m_blocks = (p.M + 2 * BM - 1) / (2 * BM);  // 256-row pair blocks
   p.num_n_blocks = (p.N + BN - 1) / BN;
   p.num_k_blocks = (p.K + BK - 1) / BK;
-  if (p.group_m <= 0) p.group_m = 8;
+  if (p.group_m <= 0) p.group_m = CONVROT_PAIR_GROUP_M;
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int sms = sm_count();
   if (sms < 2) return cudaErrorInvalidDevice;
@@ -934,8 +1153,53 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
 
 }  // namespace
 
+namespace {
+
+template <int EPI, int BNT>
+cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
+  CUtensorMap tw, tx;
+  if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, SM_BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, p.K, p.M, BK, BNT, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  p.num_k_blocks = (p.K + BK - 1) / BK;
+  const int tiles = (p.N + SM_BW - 1) / SM_BW;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = tiles < sms ? tiles : sms;
+  constexpr int smem = SmallSmem<BNT>::kAlloc;
+  static std::atomic<int> attr_done[kMaxDevices];
+  cudaError_t e = ensure_smem_attr(gemm_i8_smallm_kernel<EPI, BNT>, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_smallm_kernel<EPI, BNT>, tw, tx, out, B, p);
+}
+
+template <int EPI>
+cudaError_t launch_smallm(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
+  if (p.M <= 16) return launch_smallm_t<EPI, 16>(A, B, out, p, stream);
+  if (p.M <= 32) return launch_smallm_t<EPI, 32>(A, B, out, p, stream);
+  if (p.M <= 64) return launch_smallm_t<EPI, 64>(A, B, out, p, stream);
+  return launch_smallm_t<EPI, 128>(A, B, out, p, stream);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out, GemmParams p,
                            cudaStream_t stream) {
+  if (p.M <= kSmallM && p.single_sm == 0) {
+    if (epi == kEpiDequantBf16) return launch_smallm<kEpiDequantBf16>(A, B, out, p, stream);
+    if (epi == kEpiRawS32) return launch_smallm<kEpiRawS32>(A, B, out, p, stream);
+    return cudaErrorInvalidValue;
+  }
   if (p.single_sm == 0) {
     if (epi == kEpiDequantBf16) return launch_pair<kEpiDequantBf16>(A, B, out, p, stream);
     if (epi == kEpiRawS32) return launch_pair<kEpiRawS32>(A, B, out, p, stream);

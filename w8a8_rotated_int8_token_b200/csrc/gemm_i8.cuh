@@ -31,7 +31,8 @@ struct GemmParams {
   int q_threads_per_row, q_rows_per_pass;  // filled by the launcher
 };
 
-constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass
+constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass (fused form)
+constexpr int kSmallM = 64;  // up to this many tokens the GEMM runs in the weight-streaming (swap-AB) form
 
 // Worker layout of the fused kernel for a given K; false if K is not a
 // multiple of 128 or too large for one CTA's worker warps (then the layer runs
