@@ -19,11 +19,12 @@ __device__ __forceinline__ float2 bfly_diff(float2 a, float2 b) {
   return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 
-// Unnormalised Walsh-Hadamard transform of one group. p[jj][e] holds the
-// elements of pieces jj (.x) and jj+4 (.y) at in-piece position e.
-template <int G>
-__device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
-  // in-piece bits (e: 1, 2, 4), packed
+// The six butterfly stages of a group's transform on the index bits one lane
+// holds: p[jj][e] holds the elements of pieces jj (.x) and jj+4 (.y) at
+// in-piece position e, so the stages run on the in-piece bits (e: 1, 2, 4),
+// the two low piece bits (jj: 1, 2), packed as f32x2, and on the top piece
+// bit (.x against .y) on scalars.
+__device__ __forceinline__ void fwht_lane_local(float2 (&p)[4][8]) {
 #pragma unroll
   for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
@@ -38,7 +39,6 @@ __device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
       }
     }
   }
-  // piece bits 0 and 1, packed
 #pragma unroll
   for (int h = 1; h < 4; h <<= 1) {
 #pragma unroll
@@ -53,7 +53,6 @@ __device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
       }
     }
   }
-  // piece bit 2: the two halves of each pair
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
 #pragma unroll
@@ -62,8 +61,12 @@ __device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
       p[jj][e] = make_float2(a + b, a - b);
     }
   }
-  // lane bits: the lower partner keeps a + b, the upper one b_partner - own = a - b
-  constexpr int LG = G / 64;
+}
+
+// The stages on the lane bits of a group (LG = g/64 lanes), with shuffles:
+// the lower partner keeps a + b, the upper one b_partner - own = a - b.
+template <int LG>
+__device__ __forceinline__ void fwht_lane_shuffle(float2 (&p)[4][8], int l) {
 #pragma unroll
   for (int m = 1; m < LG; m <<= 1) {
     const float sgn = (l & m) ? -1.0f : 1.0f;
@@ -81,116 +84,86 @@ __device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
   }
 }
 
-// g = 256, first half: the five stages on the bits a lane holds in registers
-// (in-piece bits 0-2 and piece bits 5-6; bit 7 is the .x/.y half of a pair).
-__device__ __forceinline__ void fwht256_in_lane(float2 (&p)[4][8]) {
-#pragma unroll
-  for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if ((e & h) == 0) {
-          const float2 a = p[jj][e], b = p[jj][e + h];
-          p[jj][e] = bfly_sum(a, b);
-          p[jj][e + h] = bfly_diff(a, b);
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int h = 1; h < 4; h <<= 1) {
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      if ((jj & h) == 0) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float2 a = p[jj][e], b = p[jj + h][e];
-          p[jj][e] = bfly_sum(a, b);
-          p[jj + h][e] = bfly_diff(a, b);
-        }
-      }
-    }
-  }
+// Unnormalised Walsh-Hadamard transform of one group, all in registers and
+// shuffles; lane l of the group holds pieces jj, jj+4 at group offset 8l.
+template <int G>
+__device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
+  fwht_lane_local(p);
+  fwht_lane_shuffle<G / 64>(p, l);
 }
 
-// g = 256, the exchange: lane l of a group holds the elements whose bits 3-4
-// equal l; afterwards it holds those whose bits 5-6 equal l, as
-// w[b7][q] = (element 128*b7 + 32*l + 2*q, ... + 1), q = bits 1-4. The 4 KB of
-// shared memory the warp's own input came from are reused in two rounds, one
-// per value of bit 2, so that whole float2 pairs retire on both sides of each
-// round. In a round a group's 128 values form 32 16-byte chunks
-// c = bits 3-7 of the element index; chunk c is stored at
-// (c & ~7) | ((c ^ ((c >> 3) & 1) << 1 ^ 5 * (group & 1)) & 7), which keeps the
-// writes and the reads of a warp on all 32 banks (4 wavefronts each).
-__device__ __forceinline__ int xchg_chunk(int c, int gw5) {
-  return (c & ~7) | ((c ^ (((c >> 3) & 1) << 1) ^ gw5) & 7);
-}
+// g = 256 through shared memory instead of shuffles. Before the exchange
+// lane l (0..3) of a group holds the elements whose index bits 3-4 equal l;
+// the 8-byte pair p[jj][e] = (element 32jj + 8l + e, element 128 + the same).
+// Lane jj receives that pair: afterwards q[src][e] holds the pair of
+// elements 32*l + 8*src + e (and +128), so the lane owns two runs of 32
+// consecutive elements and index bits 3-4 are in registers.
+//
+// The transposition runs in four rounds (e in {2r, 2r+1}) through the 4 KB
+// of shared memory the warp's own input came from. In a round, the 16-byte
+// chunk that lane src sends to lane d of warp group gw sits at chunk index
+// 38*(gw/2) + (gw%2) + 10*d + 2*src: the two groups of a pair interleave on
+// even and odd chunks, so every 8-lane phase of a 16-byte store (fixed d) or
+// load (fixed src) touches 8 different bank quads, and every address is a
+// per-thread base plus a constant. A round spans 2432 bytes.
+constexpr int kX256RegionBytes = 4096;  // the input bytes of one warp: 32 lanes x 64 bf16 (see rotquant_slot_bytes)
 
-__device__ __forceinline__ void fwht256_exchange(const float2 (&p)[4][8], float2 (&w)[2][16], uint8_t* region,
-                                                 int gw, int l, bool active) {
-  float* blk = reinterpret_cast<float*>(region + gw * 512);
-  const int gw5 = (gw & 1) ? 5 : 0;
+__device__ __forceinline__ void fwht256_exchange(const float2 (&p)[4][8], float2 (&q)[4][8], uint8_t* warp_region,
+                                                 int gw, int l) {
+  uint8_t* const pair_base = warp_region + 16 * (38 * (gw >> 1) + (gw & 1));
+  uint8_t* const wr = pair_base + 32 * l;        // + 160 d
+  const uint8_t* const rd = pair_base + 160 * l;  // + 32 src
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {  // bit 2 of the element index
-    __syncwarp();  // the previous use of the region (input pieces or round 0) is finished
-    if (active) {
+  for (int r = 0; r < 4; ++r) {
+    __syncwarp();  // the warp's input loads, or the previous round's loads, are done
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {    // bits 5-6
-#pragma unroll
-        for (int b7 = 0; b7 < 2; ++b7) {
-          const int c = l + 4 * jj + 16 * b7;
-          float4 f;
-          f.x = b7 ? p[jj][4 * h + 0].y : p[jj][4 * h + 0].x;
-          f.y = b7 ? p[jj][4 * h + 1].y : p[jj][4 * h + 1].x;
-          f.z = b7 ? p[jj][4 * h + 2].y : p[jj][4 * h + 2].x;
-          f.w = b7 ? p[jj][4 * h + 3].y : p[jj][4 * h + 3].x;
-          *reinterpret_cast<float4*>(blk + 4 * xchg_chunk(c, gw5)) = f;
-        }
-      }
+    for (int d = 0; d < 4; ++d) {
+      const float2 a = p[d][2 * r], b = p[d][2 * r + 1];
+      *reinterpret_cast<float4*>(wr + 160 * d) = make_float4(a.x, a.y, b.x, b.y);
     }
     __syncwarp();
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {         // bits 3-4
+    for (int src = 0; src < 4; ++src) {
+      const float4 f = *reinterpret_cast<const float4*>(rd + 32 * src);
+      q[src][2 * r] = make_float2(f.x, f.y);
+      q[src][2 * r + 1] = make_float2(f.z, f.w);
+    }
+  }
+}
+
+// g = 256, the two stages left after the exchange (index bits 3-4, the first
+// index of q), packed.
+__device__ __forceinline__ void fwht256_after_exchange(float2 (&q)[4][8]) {
 #pragma unroll
-      for (int b7 = 0; b7 < 2; ++b7) {
-        const int q = 8 * (k >> 1) + 4 * (k & 1) + 2 * h;
-        if (active) {
-          const int c = k + 4 * l + 16 * b7;
-          const float4 f = *reinterpret_cast<const float4*>(blk + 4 * xchg_chunk(c, gw5));
-          w[b7][q] = make_float2(f.x, f.y);
-          w[b7][q + 1] = make_float2(f.z, f.w);
-        } else {
-          w[b7][q] = make_float2(0.0f, 0.0f);
-          w[b7][q + 1] = make_float2(0.0f, 0.0f);
+  for (int h = 1; h < 4; h <<= 1) {
+#pragma unroll
+    for (int src = 0; src < 4; ++src) {
+      if ((src & h) == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float2 a = q[src][e], b = q[src + h][e];
+          q[src][e] = bfly_sum(a, b);
+          q[src + h][e] = bfly_diff(a, b);
         }
       }
     }
   }
 }
 
-// g = 256, second half: stages on bits 3 (q bit 2), 4 (q bit 3) and 7.
-__device__ __forceinline__ void fwht256_after_exchange(float2 (&w)[2][16]) {
+// max |value| of a lane's 64 values, as a balanced tree (six dependent steps
+// instead of a 64-long chain).
+__device__ __forceinline__ float absmax64(const float2 (&w)[4][8]) {
+  float a[16];
 #pragma unroll
-  for (int h = 4; h < 16; h <<= 1) {
-#pragma unroll
-    for (int b7 = 0; b7 < 2; ++b7) {
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        if ((q & h) == 0) {
-          const float2 a = w[b7][q], b = w[b7][q + h];
-          w[b7][q] = bfly_sum(a, b);
-          w[b7][q + h] = bfly_diff(a, b);
-        }
-      }
-    }
+  for (int i = 0; i < 16; ++i) {
+    const float2 x = w[i >> 2][2 * (i & 3)], y = w[i >> 2][2 * (i & 3) + 1];
+    a[i] = fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(y.x), fabsf(y.y)));
   }
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const float2 a = w[0][q], b = w[1][q];
-    w[0][q] = bfly_sum(a, b);
-    w[1][q] = bfly_diff(a, b);
-  }
+  for (int n = 8; n >= 1; n >>= 1)
+#pragma unroll
+    for (int i = 0; i < n; ++i) a[i] = fmaxf(a[i], a[i + n]);
+  return a[0];
 }
 
 // The scale of a row (or tensor) from the absmax of its unnormalised

@@ -11,18 +11,22 @@
 // eight 16-byte pieces at group offsets j*(g/8) + 8*l (j = 0..7), so one warp
 // load instruction reads LG*16 contiguous bytes per group, fully coalesced.
 // The group index bits split as e (bits 0-2, inside a piece), l (log2 LG lane
-// bits) and j (top three bits): six butterfly stages run in registers and one
-// (g=128) or two (g=256) across lanes with shuffles.
+// bits) and j (top three bits): six butterfly stages run in registers. For
+// g = 128 the one stage on the lane bit uses shuffles. For g = 256 the lanes
+// of a group transpose their values through shared memory so that the two
+// lane bits come into registers (two more register stages); that costs one
+// 16-byte store and one 16-byte load per four values instead of two shuffles
+// per value.
 //
 // Arithmetic is packed: the 64 values live as 32 float2 pairs (piece j, piece
 // j+4), so every butterfly stage except the one on j's top bit is one f32x2
 // add or fma per two butterflies; that stage is done on scalars. The transform
 // is computed unnormalised in float32 and 1/sqrt(g) is folded into the scale.
-// A CTA handles `rpc` whole rows at a time (K/64 threads per row) and loops
-// over row blocks (persistent grid); one thread keeps kRqStages row blocks in
-// flight with bulk asynchronous copies into shared memory, so the memory
-// parallelism does not depend on how many warps fit. The row absmax is reduced
-// in shared memory.
+// A CTA handles `rpc` whole rows at a time (K/64 threads per row, about three
+// warps) and loops over row blocks (persistent grid, several CTAs per SM);
+// thread 0 streams the blocks into shared memory with bulk asynchronous
+// copies, the next block in flight while the current one is computed. The row
+// absmax is reduced in shared memory, with one CTA barrier per block.
 
 #include <cuda_runtime.h>
 
@@ -42,9 +46,11 @@ template <int G, int MODE>
 __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   constexpr int LG = G / 64;
   constexpr int PIECE = G / 8;  // elements between consecutive pieces of a lane
-  extern __shared__ __align__(128) uint8_t stage_mem[];  // kRqStages x (rows_per_cta x K) bf16
+  // kRqStages input slots of rows_per_cta x K bf16, each rounded up to whole
+  // 4 KB warp regions (g = 256 reuses a warp's region for its exchange)
+  extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ uint64_t full[kRqStages];
-  __shared__ unsigned row_max[2][kMaxRowsPerCta];
+  __shared__ unsigned row_max[3][kMaxRowsPerCta];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
@@ -61,13 +67,14 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   constexpr int F = (G == 256) ? 2 : 4;
   const int flip = grp & (F - 1);
   const int64_t nblocks = (p.rows + rpc - 1) / rpc;
-  const uint32_t stage_bytes = static_cast<uint32_t>(rpc) * static_cast<uint32_t>(p.K) * 2u;
+  const uint32_t stage_bytes = rotquant_slot_bytes(rpc, p.K);
 
   if (tid == 0) {
     for (int s = 0; s < kRqStages; ++s) mbar_init(&full[s], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
+  if (tid < rpc) row_max[0][tid] = 0u;
   __syncthreads();
   // The input may be the previous kernel's output: wait for it (launches are
   // programmatic), then let the next kernel start its prologue early.
@@ -75,7 +82,10 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   griddep_launch_dependents();
   if (MODE == kRqActivation && p.status_reset != nullptr && blockIdx.x == 0 && tid == 0) *p.status_reset = 0;
 
-  // the producer (thread 0) keeps kRqStages row blocks of this CTA in flight
+  // The producer (thread 0) loads row block it+1 as soon as block it has
+  // landed, so one block per CTA is in flight while the CTA computes: with a
+  // few CTAs per SM that covers the memory latency, and the first block of
+  // every CTA is not held up behind the later ones.
   int64_t issued = 0;
   auto issue = [&](int64_t it) {
     const int64_t blk = blockIdx.x + it * gridDim.x;
@@ -88,8 +98,8 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
     bulk_load(stage_mem + static_cast<size_t>(slot) * stage_bytes, p.src + r0 * p.K, bytes, &full[slot]);
     issued = it + 1;
   };
-  if (tid == 0)
-    for (int s = 0; s < kRqStages; ++s) issue(s);
+  static_assert(kRqStages >= 2, "the block after the current one needs its own slot");
+  if (tid == 0) issue(0);
 
   int64_t it = 0;
   bool timed_out = false;
@@ -98,10 +108,15 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
     const uint32_t ph = static_cast<uint32_t>((it / kRqStages) & 1);
     const int64_t row = blk * rpc + row_in_cta;
     const bool valid = lane_active && row < p.rows;
-    unsigned* rmax = row_max[it & 1];
-    if (tid < rpc) rmax[tid] = 0u;
+    // Row maxima rotate over three buffers: this block's, the next block's
+    // (cleared now, before this block's barrier), and the previous block's,
+    // which slower threads may still be reading.
+    unsigned* rmax = row_max[it % 3];
+    if (tid < rpc) row_max[(it + 1) % 3][tid] = 0u;
 
     const bool ok = mbar_wait_bounded(&full[slot], ph, &abort_flag, p.timeout_ns);
+    // the slot of block it+1 was released by the barrier of block it-1
+    if (tid == 0 && ok) issue(it + 1);
     uint8_t* slot_mem = stage_mem + static_cast<size_t>(slot) * stage_bytes;
     float2 v[4][8];
     if (valid) {
@@ -127,35 +142,33 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
         for (int e = 0; e < 8; ++e) v[jj][e] = make_float2(0.0f, 0.0f);
     }
 
-    float m = 0.0f;
-    float2 w[2][16];  // g = 256: the lane's values after the exchange
+    // transform; afterwards w holds the lane's values (layout per g below)
+    float2 w[4][8];
+    fwht_lane_local(v);
     if constexpr (G == 256) {
-      fwht256_in_lane(v);
-      fwht256_exchange(v, w, slot_mem + static_cast<size_t>(tid >> 5) * 4096, (tid >> 2) & 7, l, lane_active);
+      fwht256_exchange(v, w, slot_mem + static_cast<size_t>(tid >> 5) * kX256RegionBytes, (tid & 31) >> 2, l);
+      // the slot is refilled by an asynchronous copy after the barrier below
+      fence_proxy_async_smem();
       fwht256_after_exchange(w);
-#pragma unroll
-      for (int b7 = 0; b7 < 2; ++b7)
-#pragma unroll
-        for (int q = 0; q < 16; ++q) m = fmaxf(m, fmaxf(fabsf(w[b7][q].x), fabsf(w[b7][q].y)));
     } else {
-      fwht_group<G>(v, l);  // all lanes take part in the shuffles
+      fwht_lane_shuffle<LG>(v, l);
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fmaxf(fabsf(v[jj][e].x), fabsf(v[jj][e].y)));
+        for (int e = 0; e < 8; ++e) w[jj][e] = v[jj][e];
     }
+    float m = absmax64(w);
 #pragma unroll
     for (int s = 1; s < LG; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+    // non-negative floats order like their bit patterns
+    if (valid && l == 0) atomicMax(&rmax[row_in_cta], __float_as_uint(m));
 
-    // every thread has its data in registers: the slot may be refilled
+    // every thread has its input in registers (the slot may be refilled) and
+    // its row maximum posted; the CTA also agrees on a timed-out wait here
     if (__syncthreads_or(!ok)) {
       timed_out = true;
       break;
     }
-    if (tid == 0) issue(it + kRqStages);
-    // non-negative floats order like their bit patterns
-    if (valid && l == 0) atomicMax(&rmax[row_in_cta], __float_as_uint(m));
-    __syncthreads();
 
     if (MODE == kRqWeightAbsmax) {
       if (valid && t == 0) atomicMax(p.tensor_absmax, rmax[row_in_cta]);
@@ -170,41 +183,38 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
       if (blk == 0 && tid == 0) *p.scale = qs.s;
     }
     if (!valid) continue;
+    if (qs.pre != 1.0f) {  // tiny row: multiply by 2^64 first (exact), then by ci
+      const float2 pre2 = make_float2(qs.pre, qs.pre);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[jj][e] = __fmul2_rn(w[jj][e], pre2);
+    }
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
     int8_t* dst = p.dst + row * p.K + static_cast<int64_t>(grp) * G;
     if constexpr (G == 256) {
-      // the lane holds elements 128*b7 + 32*l + (0..31); the piece-order flip
-      // of the input left them multiplied by (-1)^(flip & bit 5) = (-1)^(flip & l)
+      // the lane holds elements 32*l + (0..31) (.x) and 128 + 32*l + (0..31)
+      // (.y), in the order w[src][e] = element 8*src + e of the run; the
+      // piece-order flip left them multiplied by (-1)^(flip & l)
       const float ci = (flip & l & 1) ? -qs.ci : qs.ci;
       const float2 ci2 = make_float2(ci, ci);
-      const float2 pre2 = make_float2(qs.pre, qs.pre);
-      const bool lifted = qs.pre != 1.0f;
+      uint32_t lo[8], hi[8];
 #pragma unroll
-      for (int b7 = 0; b7 < 2; ++b7) {
-        uint32_t word[8];
+      for (int src = 0; src < 4; ++src) {
+        float2 r[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float2 a = w[b7][2 * k], b = w[b7][2 * k + 1];
-          if (lifted) {  // tiny row: multiply by 2^64 first (exact), then by ci
-            a = __fmul2_rn(a, pre2);
-            b = __fmul2_rn(b, pre2);
-          }
-          const float2 ra = __ffma2_rn(a, ci2, magic2);
-          const float2 rb = __ffma2_rn(b, ci2, magic2);
-          word[k] = pack4(ra.x, ra.y, rb.x, rb.y);
-        }
-        int8_t* o = dst + 128 * b7 + 32 * l;
-        *reinterpret_cast<uint4*>(o) = make_uint4(word[0], word[1], word[2], word[3]);
-        *reinterpret_cast<uint4*>(o + 16) = make_uint4(word[4], word[5], word[6], word[7]);
+        for (int e = 0; e < 8; ++e) r[e] = __ffma2_rn(w[src][e], ci2, magic2);
+        lo[2 * src] = pack4(r[0].x, r[1].x, r[2].x, r[3].x);
+        lo[2 * src + 1] = pack4(r[4].x, r[5].x, r[6].x, r[7].x);
+        hi[2 * src] = pack4(r[0].y, r[1].y, r[2].y, r[3].y);
+        hi[2 * src + 1] = pack4(r[4].y, r[5].y, r[6].y, r[7].y);
       }
+      int8_t* o = dst + 32 * l;
+      *reinterpret_cast<uint4*>(o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(o + 16) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+      *reinterpret_cast<uint4*>(o + 128) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(o + 144) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
     } else {
-      if (qs.pre != 1.0f) {
-        const float2 pre2 = make_float2(qs.pre, qs.pre);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[jj][e] = __fmul2_rn(v[jj][e], pre2);
-      }
       int8_t* d8 = dst + 8 * l;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
@@ -212,7 +222,7 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
         const float2 ci2 = make_float2(cij, cij);
         float2 r[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) r[e] = __ffma2_rn(v[jj][e], ci2, magic2);
+        for (int e = 0; e < 8; ++e) r[e] = __ffma2_rn(w[jj][e], ci2, magic2);
         // piece jj from the .x halves, piece jj+4 from the .y halves
         uint2 lo, hi;
         lo.x = pack4(r[0].x, r[1].x, r[2].x, r[3].x);
@@ -237,7 +247,7 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
 bool rotquant_shape(int64_t K, int* threads_per_row, int* rows_per_cta) {
   if (K <= 0 || K % 128 != 0 || K > 32768) return false;
   const int tpr = static_cast<int>(K / 64);
-  int rpc = (192 + tpr / 2) / tpr;
+  int rpc = (96 + tpr / 2) / tpr;
   if (rpc < 1) rpc = 1;
   if (rpc > kMaxRowsPerCta) rpc = kMaxRowsPerCta;
   if ((rpc * tpr + 31) / 32 * 32 > kRotQuantMaxThreads) return false;
@@ -252,7 +262,7 @@ template <int G, int MODE>
 cudaError_t launch_typed(RotQuantParams p, cudaStream_t stream) {
   void (*kern)(RotQuantParams) = rotate_quant_kernel<G, MODE>;
   const int threads = (p.rows_per_cta * p.threads_per_row + 31) / 32 * 32;
-  const size_t smem = static_cast<size_t>(kRqStages) * p.rows_per_cta * p.K * 2;
+  const size_t smem = static_cast<size_t>(kRqStages) * rotquant_slot_bytes(p.rows_per_cta, p.K);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

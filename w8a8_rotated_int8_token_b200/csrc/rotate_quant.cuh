@@ -14,7 +14,7 @@ enum RotQuantMode : int {
 };
 
 constexpr int kMaxRowsPerCta = 256;
-constexpr int kRqStages = 3;          // row blocks in flight per CTA
+constexpr int kRqStages = 2;          // input slots per CTA: the block computed and the next one
 constexpr int kRqTimeoutStatus = 5;   // CONVROT_ERR_DEVICE_TIMEOUT
 constexpr int kRotQuantMaxThreads = 512;  // K/64 threads per row: K <= 32768
 
@@ -36,6 +36,13 @@ struct RotQuantParams {
 // multiple of 128 or above 32768. The CTA has rows*K/64 threads rounded up to
 // whole warps; the padding threads hold zeros.
 bool rotquant_shape(int64_t K, int* threads_per_row, int* rows_per_cta);
+
+// Bytes of one input slot: rows_per_cta rows of K bf16, rounded up to whole
+// 4 KB regions (one per warp of the CTA; 32 lanes x 64 bf16).
+__host__ __device__ inline uint32_t rotquant_slot_bytes(int rows_per_cta, int64_t K) {
+  const uint32_t bytes = static_cast<uint32_t>(rows_per_cta) * static_cast<uint32_t>(K) * 2u;
+  return (bytes + 4095u) / 4096u * 4096u;
+}
 
 cudaError_t launch_rotate_quant(int g, int mode, RotQuantParams p, cudaStream_t stream);
 
