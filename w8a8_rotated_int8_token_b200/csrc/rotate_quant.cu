@@ -101,27 +101,36 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   static_assert(kRqStages >= 2, "the block after the current one needs its own slot");
   if (tid == 0) issue(0);
 
+  // byte offset of the lane's first piece inside a slot (loop-invariant)
+  const uint32_t lane_off =
+      (static_cast<uint32_t>(row_in_cta) * static_cast<uint32_t>(p.K) + static_cast<uint32_t>(grp * G + 8 * l)) * 2u;
+
   int64_t it = 0;
+  int slot = 0;
+  uint32_t ph = 0;
+  int rsel = 0;  // which of the three row-maximum buffers this block uses
   bool timed_out = false;
   for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x, ++it) {
-    const int slot = static_cast<int>(it % kRqStages);
-    const uint32_t ph = static_cast<uint32_t>((it / kRqStages) & 1);
     const int64_t row = blk * rpc + row_in_cta;
     const bool valid = lane_active && row < p.rows;
     // Row maxima rotate over three buffers: this block's, the next block's
     // (cleared now, before this block's barrier), and the previous block's,
     // which slower threads may still be reading.
-    unsigned* rmax = row_max[it % 3];
-    if (tid < rpc) row_max[(it + 1) % 3][tid] = 0u;
+    const int rnext = (rsel == 2) ? 0 : rsel + 1;
+    unsigned* rmax = row_max[rsel];
+    if (tid < rpc) row_max[rnext][tid] = 0u;
 
     const bool ok = mbar_wait_bounded(&full[slot], ph, &abort_flag, p.timeout_ns);
     // the slot of block it+1 was released by the barrier of block it-1
     if (tid == 0 && ok) issue(it + 1);
     uint8_t* slot_mem = stage_mem + static_cast<size_t>(slot) * stage_bytes;
+    // Every lane loads, also those of rows past the end or of padding
+    // threads: their bytes lie inside the slot (stale but harmless) and only
+    // their stores are skipped. The first butterfly stage (top piece bit)
+    // is taken on the bf16 words as they arrive.
     float2 v[4][8];
-    if (valid) {
-      const uint8_t* src =
-          slot_mem + (static_cast<size_t>(row_in_cta) * p.K + static_cast<size_t>(grp) * G + 8 * l) * 2;
+    {
+      const uint8_t* src = slot_mem + lane_off;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const uint4 a = *reinterpret_cast<const uint4*>(src + ((jj ^ flip) * PIECE) * 2);
@@ -130,17 +139,16 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          v[jj][2 * q] = make_float2(__uint_as_float(aw[q] << 16), __uint_as_float(bw[q] << 16));
-          v[jj][2 * q + 1] =
-              make_float2(__uint_as_float(aw[q] & 0xFFFF0000u), __uint_as_float(bw[q] & 0xFFFF0000u));
+          v[jj][2 * q] = bfly_bf16_lo(aw[q], bw[q]);
+          v[jj][2 * q + 1] = bfly_bf16_hi(aw[q], bw[q]);
         }
       }
-    } else {
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[jj][e] = make_float2(0.0f, 0.0f);
     }
+    if (++slot == kRqStages) {
+      slot = 0;
+      ph ^= 1u;
+    }
+    rsel = rnext;
 
     // transform; afterwards w holds the lane's values (layout per g below)
     float2 w[4][8];
