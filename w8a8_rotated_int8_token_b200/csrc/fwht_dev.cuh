@@ -31,26 +31,6 @@ __device__ __forceinline__ void fwht_pair_stage(float2 (&p)[4][8]) {
   }
 }
 
-// The same stage taken straight from the bf16 input words: for a word pair
-// (wa of piece j, wb of piece j+4) it returns the butterflies of their low
-// (lo = true) or high halves. Only wb's half is widened to float32; wa's half
-// enters add/sub as bf16 (mixed-precision add.f32.bf16, exact widening), so a
-// butterfly of two bf16 inputs costs three instructions instead of four.
-__device__ __forceinline__ float2 bfly_bf16_lo(uint32_t wa, uint32_t wb) {
-  float s, d;
-  asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
-      "add.rn.f32.bf16 %0, h0, %3;\n\tsub.rn.f32.bf16 %1, h0, %3;\n\t}"
-      : "=f"(s), "=f"(d) : "r"(wa), "f"(__uint_as_float(wb << 16)));
-  return make_float2(s, d);
-}
-__device__ __forceinline__ float2 bfly_bf16_hi(uint32_t wa, uint32_t wb) {
-  float s, d;
-  asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
-      "add.rn.f32.bf16 %0, h1, %3;\n\tsub.rn.f32.bf16 %1, h1, %3;\n\t}"
-      : "=f"(s), "=f"(d) : "r"(wa), "f"(__uint_as_float(wb & 0xFFFF0000u)));
-  return make_float2(s, d);
-}
-
 // The five packed stages on the index bits a lane holds apart from the top
 // piece bit: p[jj][e] holds the elements of pieces jj (.x) and jj+4 (.y) at
 // in-piece position e; the stages run on e (1, 2, 4) and jj (1, 2) as f32x2.
@@ -110,8 +90,8 @@ __device__ __forceinline__ void fwht_lane_shuffle(float2 (&p)[4][8], int l) {
 // shuffles; lane l of the group holds pieces jj, jj+4 at group offset 8l.
 template <int G>
 __device__ __forceinline__ void fwht_group(float2 (&p)[4][8], int l) {
-  fwht_pair_stage(p);
   fwht_lane_local(p);
+  fwht_pair_stage(p);
   fwht_lane_shuffle<G / 64>(p, l);
 }
 

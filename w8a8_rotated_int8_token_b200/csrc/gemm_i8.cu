@@ -184,12 +184,18 @@ __device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmOut, const Ge
                                               int row0, int n_base, float sc, uint8_t* ebuf0, int& chunk_count,
                                               int lane, Release release) {
   constexpr int kEpiBuf = (EPI == kEpiDequantBf16) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
-#pragma unroll 1
-  for (int c = 0; c < BN / CHUNK; ++c) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(c * CHUNK), r);
-    tmem_ld_wait();
-    if (c == BN / CHUNK - 1) {  // accumulator fully read: hand it back to the MMA warp
+  constexpr int kChunks = BN / CHUNK;
+  // two register buffers: the load of chunk c+1 is in flight while chunk c
+  // is converted and stored
+  uint32_t buf[2][32];
+  tmem_ld_32x32b_x32(t_row, buf[0]);
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    uint32_t (&r)[32] = buf[c & 1];
+    tmem_ld_wait_regs(r);
+    if (c + 1 < kChunks) {
+      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((c + 1) * CHUNK), buf[(c + 1) & 1]);
+    } else {  // accumulator fully read: hand it back to the MMA warp
       tc_fence_before();
       __syncwarp();
       if (lane == 0) release();

@@ -126,8 +126,7 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
     uint8_t* slot_mem = stage_mem + static_cast<size_t>(slot) * stage_bytes;
     // Every lane loads, also those of rows past the end or of padding
     // threads: their bytes lie inside the slot (stale but harmless) and only
-    // their stores are skipped. The first butterfly stage (top piece bit)
-    // is taken on the bf16 words as they arrive.
+    // their stores are skipped.
     float2 v[4][8];
     {
       const uint8_t* src = slot_mem + lane_off;
@@ -139,8 +138,9 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          v[jj][2 * q] = bfly_bf16_lo(aw[q], bw[q]);
-          v[jj][2 * q + 1] = bfly_bf16_hi(aw[q], bw[q]);
+          v[jj][2 * q] = make_float2(__uint_as_float(aw[q] << 16), __uint_as_float(bw[q] << 16));
+          v[jj][2 * q + 1] =
+              make_float2(__uint_as_float(aw[q] & 0xFFFF0000u), __uint_as_float(bw[q] & 0xFFFF0000u));
         }
       }
     }
@@ -152,7 +152,11 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
 
     // transform; afterwards w holds the lane's values (layout per g below)
     float2 w[4][8];
+    // packed stages first, then the scalar one on the top piece bit: its
+    // results go straight to the 16-byte exchange stores (or the shuffles)
+    // without being re-paired
     fwht_lane_local(v);
+    fwht_pair_stage(v);
     if constexpr (G == 256) {
       fwht256_exchange(v, w, slot_mem + static_cast<size_t>(tid >> 5) * kX256RegionBytes, (tid & 31) >> 2, l);
       // the slot is refilled by an asynchronous copy after the barrier below
