@@ -35,6 +35,29 @@ N_SETS = 4  # rotating input/output sets per rank so that no step finds its data
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200
 
+# DRAM bytes per launch of the dominant kernel (the pair GEMM) on a workload,
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum). A
+# figure holds only for the kernel source it was taken on: the sha256 over
+# GEMM_SOURCES must match, otherwise the bench reports null.
+GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh", "fwht_dev.cuh"]
+GEMM_TRAFFIC = {
+    "dit_qkv_1024": {"bytes": 59430656 + 48917504,
+                     "sources_sha256": "ff470c56cf1c1a7484ad1b4ec2401cf7d68cd6981399e267c08053dcb8d056da"},
+}
+
+
+def gemm_traffic(config: str):
+    import hashlib
+
+    rec = GEMM_TRAFFIC.get(config)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "w8a8_rotated_int8_token_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return float(rec["bytes"]) if h.hexdigest() == rec["sources_sha256"] else None
+
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -419,7 +442,9 @@ def main():
                      "kernel": ("gemm_i8_pair_kernel (tcgen05.mma.cta_group::2 kind::i8, dequant/bias epilogue)"
                                 if launches == 2 else "gemm_i8_kernel with fused rotate+quantise workers"),
                      "achieved": dom_tops, "peak": int8_peak, "unit": "TOPS", "frac": dom_tops / int8_peak,
-                     "traffic": None, "us_per_launch": t_dom * 1e3,
+                     "traffic": gemm_traffic(args.config) if launches == 2 else None,
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
+                     "us_per_launch": t_dom * 1e3,
                      "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
                                     "(nominal int8:bf16 dense ratio)"},
         "layer_us_per_call_events": t_layer * 1e3,
