@@ -8,15 +8,20 @@ from .convrot_oracle import (  # noqa: F401
     QMAX,
     bf16_to_f64,
     dequant,
+    dequant_per_channel,
+    f16_to_f64,
+    gelu_erf,
     gemm_s32,
     hadamard,
     linear,
     nrmse,
     prepare_weight,
+    prepare_weight_per_channel,
     quant_act,
     quantize_per_token,
     quantize_tensorwise,
     rotate,
     rotation_matrix,
     to_bf16_rne,
+    to_f16_rne,
 )

@@ -29,6 +29,9 @@ Readings where the pages are silent (each listed in the design notes):
   * The weight scale is one float32 for the whole tensor; the activation scale
     is one float32 per token (row).
   * Dequantisation: y = acc * (s_x[m] * s_w) + bias[n].
+  * Variants: an FP16 compute dtype (X, bias and Y in fp16), one weight scale
+    per output channel, and an exact-erf GELU applied to y (the MLP
+    up-projection with its activation fused).
 
 Every step is written from its definition: the rotation is an explicit matrix
 product (no butterflies), the GEMM is a float64 matrix product of integer
@@ -46,6 +49,16 @@ QMAX = 127
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """bf16 values given as uint16 bit patterns, widened exactly to float64."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """IEEE fp16 values given as uint16 bit patterns, widened exactly to float64.
+
+    The layer's compute dtype may be FP16 as well as BF16 (InvokeAI "int8
+    Compute" page, "What stays on the default path": the kernels run in BF16
+    and FP16 only).
+    """
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
 def hadamard(g: int) -> np.ndarray:
@@ -129,6 +142,17 @@ def prepare_weight(w: np.ndarray, g: int) -> tuple[np.ndarray, np.float32]:
     return quantize_tensorwise(rotate(w, g))
 
 
+def prepare_weight_per_channel(w: np.ndarray, g: int) -> tuple[np.ndarray, np.ndarray]:
+    """W [N,K] -> (Wq int8 [N,K], s_w float32 [N]): rotate rows, one scale per output channel.
+
+    The "Row-wise" scaling of INT8 ConvRot in the format table of the ConvRot
+    article (section "Representative Model Formats and INT8 ConvRot"), read as
+    one scale per weight row (output channel): the same symmetric rule as the
+    per-token activation scale, applied to the rows of W R.
+    """
+    return quantize_per_token(rotate(w, g))
+
+
 def quant_act(x: np.ndarray, g: int) -> tuple[np.ndarray, np.ndarray]:
     """X [M,K] (float values) -> (Xq int8 [M,K], s_x float32 [M]): rotate tokens, then quantise."""
     return quantize_per_token(rotate(x, g))
@@ -154,6 +178,28 @@ def dequant(acc: np.ndarray, s_x: np.ndarray, s_w: float, bias: np.ndarray | Non
     return y
 
 
+def dequant_per_channel(acc: np.ndarray, s_x: np.ndarray, s_w: np.ndarray,
+                        bias: np.ndarray | None = None) -> np.ndarray:
+    """y[m, n] = acc[m, n] * (s_x[m] * s_w[n]) + bias[n], in float64 (per-output-channel weight scale)."""
+    y = np.asarray(acc, np.float64) * (np.asarray(s_x, np.float64)[:, None] * np.asarray(s_w, np.float64)[None, :])
+    if bias is not None:
+        y = y + np.asarray(bias, np.float64)[None, :]
+    return y
+
+
+def gelu_erf(y: np.ndarray) -> np.ndarray:
+    """GELU with the exact Gaussian CDF: y * Phi(y) = 0.5 * y * (1 + erf(y / sqrt(2))), float64.
+
+    The activation between the two MLP projections of the diffusion
+    transformers the pages measure; applied to the up projection's output
+    when it is fused into that layer.
+    """
+    from scipy.special import erf
+
+    y = np.asarray(y, np.float64)
+    return 0.5 * y * (1.0 + erf(y / np.sqrt(2.0)))
+
+
 def linear(x: np.ndarray, wq: np.ndarray, s_w: float, g: int,
            bias: np.ndarray | None = None) -> np.ndarray:
     """One ConvRot linear call: rotate + per-token quantise X, int8 GEMM, dequantise."""
@@ -171,6 +217,15 @@ def to_bf16_rne(y: np.ndarray) -> np.ndarray:
     """
     u = np.asarray(y, np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
     return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def to_f16_rne(y: np.ndarray) -> np.ndarray:
+    """Round float64 values to IEEE fp16 (nearest, ties to even); return uint16 bits.
+
+    NumPy's float64 -> float16 cast rounds to nearest even directly.
+    """
+    with np.errstate(over="ignore"):  # values past the fp16 range round to infinity
+        return np.asarray(y, np.float64).astype(np.float16).view(np.uint16)
 
 
 def nrmse(y: np.ndarray, ref: np.ndarray) -> float:

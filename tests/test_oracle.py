@@ -347,3 +347,79 @@ def test_nrmse_definition():
     ref = np.array([3.0, 4.0])
     assert oracle.nrmse(ref, ref) == 0.0
     assert oracle.nrmse(np.array([3.0, 4.0 + 0.5]), ref) == pytest.approx(0.1)
+
+
+# ---------------------------------------------------------------- variants
+# FP16 compute dtype, per-output-channel weight scale, exact-erf GELU.
+
+
+def _f16_from_definition(bits: int) -> float:
+    """IEEE binary16 decoded by hand: sign, 5-bit exponent (bias 15), 10-bit fraction."""
+    s = -1.0 if bits & 0x8000 else 1.0
+    e = (bits >> 10) & 0x1F
+    f = bits & 0x3FF
+    if e == 0:
+        return s * f * 2.0**-24
+    if e == 31:
+        return s * float("inf") if f == 0 else float("nan")
+    return s * (1.0 + f / 1024.0) * 2.0 ** (e - 15)
+
+
+@pytest.mark.parametrize("bits", [0x3C00, 0xC000, 0x7BFF, 0x0001, 0x03FF, 0x0400, 0x3555, 0x8000, 0x5640, 0xB4CD])
+def test_f16_widening_follows_the_format(bits):
+    got = float(oracle.f16_to_f64(np.array([bits], np.uint16))[0])
+    assert got == _f16_from_definition(bits)
+    assert np.signbit(got) == bool(bits & 0x8000)
+
+
+def test_to_f16_rne_ties_and_range():
+    # 1 + 2^-11 lies halfway between 1 and 1 + 2^-10: ties go to the even fraction (1.0)
+    cases = {1.0 + 2.0**-11: 0x3C00, 1.0 + 3 * 2.0**-11: 0x3C02, -2.5: 0xC100, 65504.0: 0x7BFF,
+             2.0**-24: 0x0001, 2.0**-25: 0x0000, 3 * 2.0**-25: 0x0002, 65520.0: 0x7C00}
+    got = oracle.to_f16_rne(np.array(list(cases), np.float64))
+    assert [int(b) for b in got] == list(cases.values())
+
+
+def test_gelu_closed_forms():
+    # Phi(1), Phi(2) of the standard normal CDF (tabulated constants)
+    phi1 = 0.8413447460685429
+    phi2 = 0.9772498680518208
+    y = oracle.gelu_erf(np.array([0.0, 1.0, -1.0, 2.0, -2.0, 12.0, -12.0]))
+    assert y[0] == 0.0
+    assert abs(y[1] - phi1) < 1e-15 and abs(y[2] - (-(1.0 - phi1))) < 1e-15
+    assert abs(y[3] - 2 * phi2) < 1e-15 and abs(y[4] - (-2 * (1.0 - phi2))) < 1e-15
+    assert y[5] == 12.0 and abs(y[6]) < 1e-30
+
+
+def test_gelu_odd_part_is_identity():
+    # y Phi(y) - (-y) Phi(-y) = y (Phi(y) + Phi(-y)) = y, for every y
+    x = np.random.default_rng(3).standard_normal(1000) * 4
+    np.testing.assert_allclose(oracle.gelu_erf(x) - oracle.gelu_erf(-x), x, rtol=0, atol=1e-14)
+
+
+def test_per_channel_weight_scale_follows_rows():
+    # rows that are power-of-two multiples of one row: identical codes, scales
+    # in the same ratios (a scale taken along the wrong axis breaks both)
+    rng = np.random.default_rng(4)
+    base = rng.standard_normal(256)
+    w = np.stack([base * 2.0**k for k in range(-3, 5)])
+    wq, sw = oracle.prepare_weight_per_channel(w, 256)
+    assert sw.dtype == np.float32 and sw.shape == (8,)
+    for n in range(1, 8):
+        assert np.array_equal(wq[n], wq[0])
+        assert sw[n] == np.float32(sw[0] * 2.0**n)
+    assert np.all(np.max(np.abs(wq.astype(np.int32)), axis=1) == 127)
+    # and the scale of a row is max |row of W R| / 127
+    wr = oracle.rotate(w, 256)
+    np.testing.assert_array_equal(sw, (np.max(np.abs(wr), axis=1) / 127).astype(np.float32))
+
+
+def test_dequant_per_channel_hand_case_and_tensorwise_limit():
+    acc = np.array([[1, 2], [3, 4]], np.int32)
+    y = oracle.dequant_per_channel(acc, np.array([1.0, 0.5]), np.array([2.0, 4.0]), np.array([0.5, -1.0]))
+    np.testing.assert_array_equal(y, [[2.5, 7.0], [3.5, 7.0]])
+    rng = np.random.default_rng(5)
+    acc = rng.integers(-1000, 1000, (5, 7)).astype(np.int32)
+    sx = rng.random(5).astype(np.float32)
+    np.testing.assert_array_equal(oracle.dequant_per_channel(acc, sx, np.full(7, 0.25, np.float32)),
+                                  oracle.dequant(acc, sx, np.float32(0.25)))

@@ -28,6 +28,13 @@ MUTATIONS = {
         "blocks = x.reshape(x.shape[:-1] + (g, K // g)).swapaxes(-1, -2)"),
     "weight_columns_reversed": ("np.asarray(wq, np.float64).T", "np.asarray(wq, np.float64)[:, ::-1].T"),
     "token_scale_not_float32": ("s = (amax / QMAX).astype(np.float32)", "s = (amax / QMAX)"),
+    "gelu_tanh_approximation": ("return 0.5 * y * (1.0 + erf(y / np.sqrt(2.0)))",
+                                "return 0.5 * y * (1.0 + np.tanh(0.7978845608028654 * (y + 0.044715 * y**3)))"),
+    "f16_read_as_bf16": ("return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)",
+                         "return bf16_to_f64(bits)"),
+    "per_channel_scale_tensorwise": ("    return quantize_per_token(rotate(w, g))\n",
+                                     "    q, s = quantize_tensorwise(rotate(w, g))\n    return q, np.full(q.shape[0], s)\n"),
+    "per_channel_scale_on_tokens_axis": ("np.asarray(s_w, np.float64)[None, :])", "np.asarray(s_w, np.float64)[:, None])"),
 }
 
 
