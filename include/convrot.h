@@ -111,9 +111,9 @@ CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K
  *   Y = bf16_rne( (Xq Wq^T) * (s_x[m] * s_w) + bias[n] ),  (Xq, s_x) = quant_act(X).
  * The int8 x int8 product accumulates exactly in int32 on the tcgen05 tensor
  * cores (InvokeAI "int8 Compute", second paragraph); dequantisation and the
- * bias are fused into the GEMM epilogue. For K <= 20480 the whole layer is one
- * kernel: worker warps rotate and quantise the tokens while the tensor cores
- * multiply the M-blocks already finished; above that it is two kernels.
+ * bias are fused into the GEMM epilogue. Two kernels (rotate+quantise, then
+ * the GEMM, chained with programmatic dependent launch);
+ * convrot_linear_launch_count reports the number for a shape.
  *   X        [M,K] bf16, device.   M >= 1, N >= 1, K % g == 0, K <= CONVROT_MAX_K,
  *                                   N % 8 == 0.
  *   Wq       [N,K] int8, device (from convrot_prepare_weight with the same g).
@@ -132,6 +132,58 @@ CONVROT_API convrot_status convrot_linear(const void* X, int64_t M, int64_t K, i
                               const int8_t* Wq, const float* w_scale, int64_t N,
                               const void* bias, void* Y,
                               void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * Variants of the layer: compute dtype, weight-scale granularity, activation.
+ *   CONVROT_DTYPE_F16: X, W, bias and Y are IEEE fp16 instead of bf16 (the
+ *     pages' kernels run in BF16 and FP16 only: InvokeAI "int8 Compute",
+ *     "What stays on the default path").
+ *   CONVROT_WSCALE_CHANNEL: one float32 weight scale per output channel (row
+ *     of W R), s_w[n] = max_k |(W R)[n,k]| / 127 -- the "Row-wise" scaling of
+ *     INT8 ConvRot in the format table of "Explanation of INT8 ConvRot"
+ *     (section "Representative Model Formats and INT8 ConvRot").
+ *   CONVROT_ACT_GELU_ERF: y -> y * Phi(y) = 0.5 y (1 + erf(y / sqrt(2))) applied
+ *     in float32 before the output rounding: the activation between the two
+ *     MLP projections of the diffusion transformers the pages measure, fused
+ *     into the up projection. The pages themselves describe no activation.
+ */
+typedef enum { CONVROT_DTYPE_BF16 = 0, CONVROT_DTYPE_F16 = 1 } convrot_dtype;
+typedef enum { CONVROT_WSCALE_TENSOR = 0, CONVROT_WSCALE_CHANNEL = 1 } convrot_wscale_mode;
+typedef enum { CONVROT_ACT_NONE = 0, CONVROT_ACT_GELU_ERF = 1 } convrot_activation;
+
+/*
+ * convrot_prepare_weight_ex -- convrot_prepare_weight with a dtype and a scale mode.
+ *   W        [N,K] in `dtype` (bf16 or fp16 bits), device.
+ *   wscale_mode  CONVROT_WSCALE_TENSOR: w_scale is 1 float (as convrot_prepare_weight);
+ *            CONVROT_WSCALE_CHANNEL: w_scale is [N] floats, 16-byte aligned, and
+ *            ws may be NULL (one kernel launch, no workspace).
+ * Other arguments and errors as convrot_prepare_weight; an unknown dtype or
+ * mode returns CONVROT_ERR_UNSUPPORTED.
+ */
+CONVROT_API convrot_status convrot_prepare_weight_ex(const void* W, int dtype, int64_t N, int64_t K, int g,
+                                                     int wscale_mode, int8_t* Wq, float* w_scale, void* ws,
+                                                     size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * convrot_quant_act_ex -- convrot_quant_act with X in `dtype` (bf16 or fp16).
+ */
+CONVROT_API convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t K, int g,
+                                                int8_t* Xq, float* x_scale, convrot_stream_t stream);
+
+/*
+ * convrot_linear_ex -- convrot_linear with the variants above:
+ *   Y = out_rne( act( (Xq Wq^T) * (s_x[m] * s_w[n or 0]) + bias[n] ) ).
+ *   dtype        type of X, bias and Y (CONVROT_DTYPE_BF16 or CONVROT_DTYPE_F16).
+ *   w_scale      1 float (CONVROT_WSCALE_TENSOR) or [N] floats, 16-byte aligned
+ *                (CONVROT_WSCALE_CHANNEL), from convrot_prepare_weight_ex.
+ *   activation   CONVROT_ACT_NONE or CONVROT_ACT_GELU_ERF.
+ * Other arguments, the workspace and the errors as convrot_linear. With bf16,
+ * a tensor scale and no activation it is exactly convrot_linear.
+ */
+CONVROT_API convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K, int g,
+                                             const int8_t* Wq, const float* w_scale, int wscale_mode, int64_t N,
+                                             const void* bias, int activation, void* Y, void* ws, size_t ws_bytes,
+                                             convrot_stream_t stream);
 
 /*
  * convrot_linear_timed -- convrot_linear that also records caller-created CUDA

@@ -62,7 +62,7 @@ def linear_ws_layout(M, K):
 
 
 def test_status_strings_and_version(L):
-    assert L.convrot_abi_version() == 2
+    assert L.convrot_abi_version() == 3
     for code in range(6):
         s = L.convrot_status_string(code)
         assert s and s != b"unknown status"
@@ -126,6 +126,34 @@ def test_other_entry_points_reject_bad_arguments_on_host(L):
                                   FAKE, None) == 1
     assert L.convrot_linear_launch_count(4608, 9216, 3072, 256) in (1, 2)
     assert L.convrot_linear_launch_count(4608, 9216, 3000, 256) == 0
+
+
+def test_variant_entry_points_reject_bad_arguments_on_host(L):
+    # convrot_linear_ex(X, dtype, M, K, g, Wq, w_scale, wscale_mode, N, bias, activation, Y, ws, ws_bytes, stream)
+    ok = (FAKE, 0, 64, 256, 256, FAKE, FAKE, 0, 256, None, 0, FAKE, FAKE, 1 << 30, None)
+
+    def call(**over):
+        a = list(ok)
+        names = ["X", "dtype", "M", "K", "g", "Wq", "w_scale", "mode", "N", "bias", "act", "Y", "ws", "ws_bytes", "s"]
+        for k, v in over.items():
+            a[names.index(k)] = v
+        return L.convrot_linear_ex(*a)
+
+    assert call(dtype=2) == 2                      # unknown dtype
+    assert call(mode=2) == 2                       # unknown scale mode
+    assert call(act=7) == 2                        # unknown activation
+    assert call(mode=1, w_scale=FAKE + 4) == 1     # per-channel scales need 16-byte alignment
+    assert call(g=64) == 2
+    assert call(Y=None) == 1
+    assert call(ws_bytes=100) == 3
+    # prepare_weight_ex(W, dtype, N, K, g, mode, Wq, w_scale, ws, ws_bytes, stream)
+    assert L.convrot_prepare_weight_ex(FAKE, 3, 8, 256, 256, 0, FAKE, FAKE, FAKE, 256, None) == 2
+    assert L.convrot_prepare_weight_ex(FAKE, 0, 8, 256, 256, 5, FAKE, FAKE, FAKE, 256, None) == 2
+    assert L.convrot_prepare_weight_ex(FAKE, 1, 8, 256, 256, 1, FAKE, FAKE + 4, None, 0, None) == 1
+    assert L.convrot_prepare_weight_ex(FAKE, 1, 8, 256, 256, 0, FAKE, FAKE, None, 0, None) == 3
+    # quant_act_ex(X, dtype, M, K, g, Xq, x_scale, stream)
+    assert L.convrot_quant_act_ex(FAKE, 9, 8, 256, 256, FAKE, FAKE, None) == 2
+    assert L.convrot_quant_act_ex(FAKE, 1, 8, 300, 256, FAKE, FAKE, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -23,6 +23,15 @@ __all__ = [
     "convrot_quant_act",
     "convrot_linear_workspace_bytes",
     "convrot_linear",
+    "convrot_prepare_weight_ex",
+    "convrot_quant_act_ex",
+    "convrot_linear_ex",
+    "DTYPE_BF16",
+    "DTYPE_F16",
+    "WSCALE_TENSOR",
+    "WSCALE_CHANNEL",
+    "ACT_NONE",
+    "ACT_GELU_ERF",
     "convrot_gemm_dequant",
     "convrot_gemm_s32",
     "convrot_read_device_status",
@@ -30,6 +39,11 @@ __all__ = [
     "ConvRotLinear",
     "lib",
 ]
+
+# convrot_dtype, convrot_wscale_mode, convrot_activation (include/convrot.h)
+DTYPE_BF16, DTYPE_F16 = 0, 1
+WSCALE_TENSOR, WSCALE_CHANNEL = 0, 1
+ACT_NONE, ACT_GELU_ERF = 0, 1
 
 STATUS_NAMES = {0: "CONVROT_OK", 1: "CONVROT_ERR_INVALID_ARG", 2: "CONVROT_ERR_UNSUPPORTED",
                 3: "CONVROT_ERR_WORKSPACE", 4: "CONVROT_ERR_CUDA", 5: "CONVROT_ERR_DEVICE_TIMEOUT"}
@@ -148,6 +162,93 @@ def convrot_linear(X, Wq, w_scale, g: int = 256, bias=None, Y=None, ws=None, str
         ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=X.device)
     _check(lib().convrot_linear(_ptr(X), M, K, g, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y), _ptr(ws),
                                 ws.numel(), _stream_ptr(stream)), "convrot_linear")
+    return Y
+
+
+def _dtype_code(t, name):
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float16:
+        return DTYPE_F16
+    raise TypeError(f"{name}: expected bfloat16 or float16, got {t.dtype}")
+
+
+def convrot_prepare_weight_ex(W, g: int = 256, wscale_mode: int = WSCALE_TENSOR, Wq=None, w_scale=None, ws=None,
+                              stream=None):
+    """Rotate and quantise a bf16 or fp16 weight [N,K]: returns (Wq int8 [N,K], w_scale float32 [1] or [N])."""
+    import torch
+
+    dtype = _dtype_code(W, "W")
+    _require(W, W.dtype, None, "W")
+    N, K = W.shape
+    ns = N if wscale_mode == WSCALE_CHANNEL else 1
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty((ns,), dtype=torch.float32, device=W.device)
+    L = lib()
+    if ws is None and wscale_mode != WSCALE_CHANNEL:
+        ws = torch.empty((L.convrot_prepare_weight_workspace_bytes(),), dtype=torch.uint8, device=W.device)
+    _require(Wq, torch.int8, (N, K), "Wq")
+    _require(w_scale, torch.float32, (ns,), "w_scale")
+    _check(L.convrot_prepare_weight_ex(_ptr(W), dtype, N, K, g, int(wscale_mode), _ptr(Wq), _ptr(w_scale), _ptr(ws),
+                                       0 if ws is None else ws.numel(), _stream_ptr(stream)),
+           "convrot_prepare_weight_ex")
+    return Wq, w_scale
+
+
+def convrot_quant_act_ex(X, g: int = 256, Xq=None, x_scale=None, stream=None):
+    """convrot_quant_act for a bf16 or fp16 X [M,K]."""
+    import torch
+
+    dtype = _dtype_code(X, "X")
+    _require(X, X.dtype, None, "X")
+    M, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if x_scale is None:
+        x_scale = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _require(Xq, torch.int8, (M, K), "Xq")
+    _require(x_scale, torch.float32, (M,), "x_scale")
+    _check(lib().convrot_quant_act_ex(_ptr(X), dtype, M, K, g, _ptr(Xq), _ptr(x_scale), _stream_ptr(stream)),
+           "convrot_quant_act_ex")
+    return Xq, x_scale
+
+
+def convrot_linear_ex(X, Wq, w_scale, g: int = 256, bias=None, activation: int = ACT_NONE, Y=None, ws=None,
+                      stream=None):
+    """ConvRot linear in the dtype of X (bf16 or fp16; bias and Y the same), with a
+    tensor (w_scale [1]) or per-output-channel (w_scale [N]) weight scale and an
+    optional exact-erf GELU on the output."""
+    import torch
+
+    dtype = _dtype_code(X, "X")
+    _require(X, X.dtype, None, "X")
+    M, K = X.shape
+    _require(Wq, torch.int8, None, "Wq")
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("Wq must be [N, K] with the K of X")
+    if w_scale.numel() == N and N != 1:
+        mode = WSCALE_CHANNEL
+    elif w_scale.numel() == 1:
+        mode = WSCALE_TENSOR
+    else:
+        raise ValueError("w_scale must hold 1 or N floats")
+    _require(w_scale, torch.float32, (w_scale.numel(),), "w_scale")
+    if bias is not None:
+        _require(bias, X.dtype, (N,), "bias")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _require(Y, X.dtype, (M, N), "Y")
+    need = convrot_linear_workspace_bytes(M, N, K, g)
+    if ws is None:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=X.device)
+    _check(lib().convrot_linear_ex(_ptr(X), dtype, M, K, g, _ptr(Wq), _ptr(w_scale), mode, N, _ptr(bias),
+                                   int(activation), _ptr(Y), _ptr(ws), ws.numel(), _stream_ptr(stream)),
+           "convrot_linear_ex")
     return Y
 
 

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
 // The one-launch form (rotate+quantise worker warps inside the GEMM kernel) is
 // correct but, measured on the DiT QKV layer, its workers fall behind the
@@ -76,10 +76,21 @@ convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int n_multiple)
   return CONVROT_OK;
 }
 
+// Options of the general dequant epilogue (convrot_linear_ex); the defaults
+// are convrot_linear's (bf16, one tensor scale, no activation).
+struct EpiOptions {
+  int out_f16 = 0;
+  int wscale_per_channel = 0;
+  int act = 0;
+  bool general() const { return out_f16 != 0 || wscale_per_channel != 0 || act != 0; }
+};
+
 convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, int64_t M, int64_t N, int64_t K,
                         const float* x_scale, const float* w_scale, const void* bias, int* status,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, EpiOptions opt = EpiOptions()) {
   convrot::GemmParams p{};
+  p.out_f16 = opt.out_f16;
+  p.wscale_per_channel = opt.wscale_per_channel;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -112,41 +123,59 @@ const char* convrot_status_string(int status) {
 
 size_t convrot_prepare_weight_workspace_bytes(void) { return 256; }
 
-convrot_status convrot_prepare_weight(const void* W, int64_t N, int64_t K, int g, int8_t* Wq, float* w_scale,
-                                      void* ws, size_t ws_bytes, convrot_stream_t stream) {
+convrot_status convrot_prepare_weight_ex(const void* W, int dtype, int64_t N, int64_t K, int g, int wscale_mode,
+                                         int8_t* Wq, float* w_scale, void* ws, size_t ws_bytes,
+                                         convrot_stream_t stream) {
   const convrot_status sh = check_rotation_shape(N, K, g);
   if (sh != CONVROT_OK) return sh;
+  if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
+  if (wscale_mode != CONVROT_WSCALE_TENSOR && wscale_mode != CONVROT_WSCALE_CHANNEL) return CONVROT_ERR_UNSUPPORTED;
   if (W == nullptr || Wq == nullptr || w_scale == nullptr) return CONVROT_ERR_INVALID_ARG;
-  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(w_scale, 4)) return CONVROT_ERR_INVALID_ARG;
-  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < convrot_prepare_weight_workspace_bytes())
-    return CONVROT_ERR_WORKSPACE;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(w_scale, wscale_mode == CONVROT_WSCALE_CHANNEL ? 16 : 4))
+    return CONVROT_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned* amax = static_cast<unsigned*>(ws);
-  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), s);
-  if (e != cudaSuccess) return CONVROT_ERR_CUDA;
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(W);
+  p.in_f16 = dtype == CONVROT_DTYPE_F16 ? 1 : 0;
   p.rows = N;
   p.K = K;
   p.dst = Wq;
   p.scale = w_scale;
-  p.tensor_absmax = amax;
   p.status_reset = nullptr;
   p.status = nullptr;
   p.timeout_ns = kWaitTimeoutNs;
+  if (wscale_mode == CONVROT_WSCALE_CHANNEL) {
+    // one scale per weight row: the per-row (activation) form of the kernel
+    p.tensor_absmax = nullptr;
+    return from_cuda(convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s));
+  }
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < convrot_prepare_weight_workspace_bytes())
+    return CONVROT_ERR_WORKSPACE;
+  unsigned* amax = static_cast<unsigned*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return CONVROT_ERR_CUDA;
+  p.tensor_absmax = amax;
   e = convrot::launch_rotate_quant(g, convrot::kRqWeightAbsmax, p, s);
   if (e != cudaSuccess) return CONVROT_ERR_CUDA;
   return from_cuda(convrot::launch_rotate_quant(g, convrot::kRqWeightQuant, p, s));
 }
 
-convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int8_t* Xq, float* x_scale,
-                                 convrot_stream_t stream) {
+convrot_status convrot_prepare_weight(const void* W, int64_t N, int64_t K, int g, int8_t* Wq, float* w_scale,
+                                      void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  return convrot_prepare_weight_ex(W, CONVROT_DTYPE_BF16, N, K, g, CONVROT_WSCALE_TENSOR, Wq, w_scale, ws, ws_bytes,
+                                   stream);
+}
+
+convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t K, int g, int8_t* Xq,
+                                    float* x_scale, convrot_stream_t stream) {
   const convrot_status sh = check_rotation_shape(M, K, g);
   if (sh != CONVROT_OK) return sh;
+  if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
   if (X == nullptr || Xq == nullptr || x_scale == nullptr) return CONVROT_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(x_scale, 4)) return CONVROT_ERR_INVALID_ARG;
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(X);
+  p.in_f16 = dtype == CONVROT_DTYPE_F16 ? 1 : 0;
   p.rows = M;
   p.K = K;
   p.dst = Xq;
@@ -157,6 +186,11 @@ convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int
   p.timeout_ns = kWaitTimeoutNs;
   return from_cuda(
       convrot::launch_rotate_quant(g, convrot::kRqActivation, p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int8_t* Xq, float* x_scale,
+                                 convrot_stream_t stream) {
+  return convrot_quant_act_ex(X, CONVROT_DTYPE_BF16, M, K, g, Xq, x_scale, stream);
 }
 
 size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
@@ -173,14 +207,14 @@ namespace {
 // are recorded before and after the launches.
 convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq, const float* w_scale,
                            int64_t N, const void* bias, void* Y, void* ws, size_t ws_bytes, cudaEvent_t ev0,
-                           cudaEvent_t ev1, cudaEvent_t ev2, cudaStream_t s) {
+                           cudaEvent_t ev1, cudaEvent_t ev2, cudaStream_t s, EpiOptions opt = EpiOptions()) {
   convrot_status sh = check_rotation_shape(M, K, g);
   if (sh != CONVROT_OK) return sh;
   sh = check_gemm_shape(M, N, K, 8);
   if (sh != CONVROT_OK) return sh;
   if (X == nullptr || Wq == nullptr || w_scale == nullptr || Y == nullptr) return CONVROT_ERR_INVALID_ARG;
-  if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(w_scale, 4) || !aligned(Y, 16) ||
-      (bias != nullptr && !aligned(bias, 16)))
+  if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(w_scale, opt.wscale_per_channel ? 16 : 4) ||
+      !aligned(Y, 16) || (bias != nullptr && !aligned(bias, 16)))
     return CONVROT_ERR_INVALID_ARG;
   const LinearWs lay = linear_ws_layout(M, K);
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE;
@@ -190,7 +224,7 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
 
   int tpr = 0, rpp = 0, cta_threads = 0;
-  if (kFusedLinear && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) {
+  if (kFusedLinear && !opt.general() && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) {
     // one launch: worker warps rotate + quantise while the GEMM consumes finished M-blocks
     convrot::GemmParams gp{};
     gp.M = static_cast<int>(M);
@@ -216,6 +250,7 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
 
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(X);
+  p.in_f16 = opt.out_f16;  // X, bias and Y share the compute dtype
   p.rows = M;
   p.K = K;
   p.dst = Xq;
@@ -227,7 +262,9 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return CONVROT_ERR_CUDA;
-  const convrot_status st = run_gemm(convrot::kEpiDequantBf16, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s);
+  const int epi = opt.act ? convrot::kEpiDequantGenGelu
+                           : (opt.general() ? convrot::kEpiDequantGen : convrot::kEpiDequantBf16);
+  const convrot_status st = run_gemm(epi, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s, opt);
   if (st != CONVROT_OK) return st;
   if (ev2 != nullptr && cudaEventRecord(ev2, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   return CONVROT_OK;
@@ -252,6 +289,20 @@ convrot_status convrot_linear_timed(const void* X, int64_t M, int64_t K, int g, 
   return linear_impl(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, static_cast<cudaEvent_t>(ev_start),
                      static_cast<cudaEvent_t>(ev_mid), static_cast<cudaEvent_t>(ev_end),
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K, int g, const int8_t* Wq,
+                                 const float* w_scale, int wscale_mode, int64_t N, const void* bias, int activation,
+                                 void* Y, void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
+  if (wscale_mode != CONVROT_WSCALE_TENSOR && wscale_mode != CONVROT_WSCALE_CHANNEL) return CONVROT_ERR_UNSUPPORTED;
+  if (activation != CONVROT_ACT_NONE && activation != CONVROT_ACT_GELU_ERF) return CONVROT_ERR_UNSUPPORTED;
+  EpiOptions opt;
+  opt.out_f16 = dtype == CONVROT_DTYPE_F16 ? 1 : 0;
+  opt.wscale_per_channel = wscale_mode == CONVROT_WSCALE_CHANNEL ? 1 : 0;
+  opt.act = activation == CONVROT_ACT_GELU_ERF ? 1 : 0;
+  return linear_impl(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, nullptr, nullptr, nullptr,
+                     reinterpret_cast<cudaStream_t>(stream), opt);
 }
 
 int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g) {

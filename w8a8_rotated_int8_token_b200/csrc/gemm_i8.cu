@@ -42,6 +42,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <atomic>
 #include <cstdint>
@@ -71,7 +72,7 @@ constexpr int kFusedMaxThreads = 512;  // 6 GEMM warps + up to 10 rotate+quantis
 
 template <int EPI>
 struct Smem {
-  static constexpr int kEpiBuf = (EPI == kEpiDequantBf16) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
+  static constexpr int kEpiBuf = epi_is_dequant(EPI) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = STAGES * A_STAGE_BYTES;
   static constexpr int kOffEpi = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES);
@@ -175,16 +176,103 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// One tile's epilogue for one warp: 8 chunks of 32 accumulator columns of the
-// warp's 32 TMEM lanes (rows row0..row0+31): load, scale + bias, pack, stage in
-// swizzled shared memory, TMA store. release() is called by lane 0 once the
-// accumulator has been read completely.
-template <int EPI, class Release>
+__device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// A 16-bit output-dtype value (bf16 or fp16 bits), widened exactly.
+__device__ __forceinline__ float out16_to_f32(uint32_t bits16, bool f16) {
+  return f16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(bits16)))
+             : __uint_as_float(bits16 << 16);
+}
+
+// erf(x) by the rational approximation of Abramowitz and Stegun, Handbook of
+// Mathematical Functions (1964), formula 7.1.26: for x >= 0,
+//   erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2),  t = 1/(1 + p x),
+// with |error| <= 1.5e-7; odd symmetry for x < 0. Branch-free, so a warp's
+// lanes never diverge on it (the epilogue applies it to every output).
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float e = 1.0f - poly * __expf(-ax * ax);
+  return copysignf(e, x);
+}
+
+// GELU with the Gaussian CDF: y * Phi(y) = 0.5 y (1 + erf(y / sqrt(2))).
+__device__ __forceinline__ float gelu_erf(float y) {
+  return 0.5f * y * (1.0f + erf_as7126(y * 0.70710678118654752f));
+}
+
+// The general epilogue for 32 consecutive output columns n0..n0+31 of one
+// row: y = acc * (sc * wv[e]) + bv[e] (then GELU), packed to the output dtype.
+// sc is x_scale[row] times the tensor weight scale, or x_scale[row] alone when
+// the weight scale is per channel (then wv holds w_scale[n]).
+template <bool GELU>
+__device__ __forceinline__ void dequant_gen32(const GemmParams& p, int n0, float sc, const uint32_t (&r)[32],
+                                              uint32_t (&packed)[16]) {
+  const bool f16 = p.out_f16 != 0;
+  float bv[32], wv[32];
+#pragma unroll
+  for (int pc = 0; pc < 4; ++pc) {
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (p.bias != nullptr && n0 + 8 * pc < p.N) w = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * pc));
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      bv[8 * pc + 2 * e] = out16_to_f32(ws[e] & 0xFFFFu, f16);
+      bv[8 * pc + 2 * e + 1] = out16_to_f32(ws[e] >> 16, f16);
+    }
+  }
+  if (p.wscale_per_channel) {
+#pragma unroll
+    for (int pc = 0; pc < 8; ++pc) {
+      float4 w = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (n0 + 4 * pc < p.N) w = __ldg(reinterpret_cast<const float4*>(p.w_scale + n0 + 4 * pc));
+      wv[4 * pc] = w.x;
+      wv[4 * pc + 1] = w.y;
+      wv[4 * pc + 2] = w.z;
+      wv[4 * pc + 3] = w.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) wv[e] = 1.0f;
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float y0 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e])), sc * wv[2 * e], bv[2 * e]);
+    float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e + 1])), sc * wv[2 * e + 1], bv[2 * e + 1]);
+    if (GELU) {
+      y0 = gelu_erf(y0);
+      y1 = gelu_erf(y1);
+    }
+    packed[e] = f16 ? f16x2(y0, y1) : bf16x2(y0, y1);
+  }
+}
+
+// The weight scale a row's multiplier carries: the tensor scale, or 1 when
+// the general epilogue applies a per-channel scale column by column.
+template <int EPI>
+__device__ __forceinline__ float epi_weight_scale(const GemmParams& p) {
+  if (EPI == kEpiDequantBf16) return __ldg(p.w_scale);
+  if (epi_is_general(EPI)) return p.wscale_per_channel ? 1.0f : __ldg(p.w_scale);
+  return 0.0f;
+}
+
+// One tile's epilogue for one warp: kChunks chunks of 32 accumulator columns
+// of the warp's 32 TMEM lanes (rows row0..row0+31), from t_row / n_base on:
+// load, scale + bias, pack, stage in swizzled shared memory, TMA store.
+// release() is called by lane 0 once the warp has read its columns.
+template <int EPI, int kChunks = BN / CHUNK, class Release>
 __device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmOut, const GemmParams& p, uint32_t t_row,
                                               int row0, int n_base, float sc, uint8_t* ebuf0, int& chunk_count,
                                               int lane, Release release) {
-  constexpr int kEpiBuf = (EPI == kEpiDequantBf16) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
-  constexpr int kChunks = BN / CHUNK;
+  constexpr int kEpiBuf = epi_is_dequant(EPI) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
   // two register buffers: the load of chunk c+1 is in flight while chunk c
   // is converted and stored
   uint32_t buf[2][32];
@@ -205,7 +293,17 @@ __device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmOut, const Ge
     uint8_t* ebuf = ebuf0 + (chunk_count & 1) * kEpiBuf;
     if (lane == 0) bulk_wait_group_read<1>();  // the store that last read this buffer is done
     __syncwarp();
-    if (EPI == kEpiDequantBf16) {
+    if (epi_is_general(EPI)) {
+      uint32_t packed[16];
+      dequant_gen32<EPI == kEpiDequantGenGelu>(p, n0, sc, r, packed);
+      uint8_t* rowp = ebuf + lane * 64;  // same 64-byte-swizzled staging as below
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int pj = j ^ ((lane >> 1) & 3);
+        *reinterpret_cast<uint4*>(rowp + pj * 16) =
+            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+      }
+    } else if (EPI == kEpiDequantBf16) {
       float bv[32];
       if (p.bias != nullptr) {
 #pragma unroll
@@ -509,7 +607,7 @@ __global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
   } else if (warp < 2 + EPI_WARPS) {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const float sw = (EPI == kEpiDequantBf16) ? __ldg(p.w_scale) : 0.0f;
+    const float sw = epi_weight_scale<EPI>(p);
     uint8_t* ebuf0 = smem + L::kOffEpi + (q * 2) * L::kEpiBuf;
     int chunk_count = 0;
     int it = 0;
@@ -534,7 +632,7 @@ __global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
           break;
         }
         sc = (row < p.M ? ld_relaxed_f32(p.x_scale + row) : 0.0f) * sw;
-      } else if (EPI == kEpiDequantBf16) {
+      } else if (epi_is_dequant(EPI)) {
         sc = (row < p.M ? __ldg(p.x_scale + row) : 0.0f) * sw;
       }
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
@@ -574,6 +672,11 @@ __global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
 // the same epilogue as the single-SM form on them. No TMA multicast is used.
 
 constexpr int BN_HALF = BN / 2;
+// Eight epilogue warps per CTA: two per TMEM lane quarter, each draining 128
+// of a tile's 256 accumulator columns, so that the epilogue of a tile (with
+// GELU the heaviest part of the kernel) stays shorter than the next tile's MMAs.
+constexpr int PAIR_EPI_WARPS = 8;
+constexpr int PAIR_THREADS = 64 + 32 * PAIR_EPI_WARPS;
 #ifndef CONVROT_PAIR_STAGES
 #define CONVROT_PAIR_STAGES 6
 #endif
@@ -587,12 +690,12 @@ constexpr uint32_t IDESC_PAIR = idesc_i8(2 * BM, BN);
 
 template <int EPI>
 struct PairSmem {
-  static constexpr int kStages = (EPI == kEpiDequantBf16) ? PAIR_STAGES : PAIR_STAGES - 1;
-  static constexpr int kEpiBuf = (EPI == kEpiDequantBf16) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
+  static constexpr int kStages = epi_is_dequant(EPI) ? PAIR_STAGES : PAIR_STAGES - 1;
+  static constexpr int kEpiBuf = epi_is_dequant(EPI) ? CHUNK * CHUNK * 2 : CHUNK * CHUNK * 4;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kStages * PA_STAGE_BYTES;
   static constexpr int kOffEpi = kStages * (PA_STAGE_BYTES + PB_STAGE_BYTES);
-  static constexpr int kOffBar = kOffEpi + EPI_WARPS * 2 * kEpiBuf;
+  static constexpr int kOffBar = kOffEpi + PAIR_EPI_WARPS * 2 * kEpiBuf;
   // full[S], empty[S], tmem_full[2], tmem_empty[2], drain, teardown
   static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
@@ -613,7 +716,7 @@ __device__ __forceinline__ void pair_tile_coords(int tile, const GemmParams& p, 
 }
 
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   using L = PairSmem<EPI>;
@@ -647,7 +750,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 2 * EPI_WARPS);  // both CTAs' epilogue warps
+      mbar_init(&tmem_empty[b], 2 * PAIR_EPI_WARPS);  // both CTAs' epilogue warps
     }
     mbar_init(drain, 1);
     mbar_init(teardown, 1);
@@ -754,9 +857,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------ epilogue (both)
-    const int q = warp & 3;
-    const float sw = (EPI == kEpiDequantBf16) ? __ldg(p.w_scale) : 0.0f;
-    uint8_t* ebuf0 = smem + L::kOffEpi + (q * 2) * L::kEpiBuf;
+    const int ew = warp - 2;   // 0..7
+    const int q = warp & 3;    // TMEM lane quarter this warp may access
+    const int half = ew >> 2;  // which 128 of the tile's 256 columns
+    const float sw = epi_weight_scale<EPI>(p);
+    uint8_t* ebuf0 = smem + L::kOffEpi + (ew * 2) * L::kEpiBuf;
     int chunk_count = 0;
     int it = 0;
     bool ok = true;
@@ -773,11 +878,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const int row0 = mb2 * 2 * BM + static_cast<int>(rank) * BM + q * 32;
       const int row = row0 + lane;
       float sc = 0.0f;
-      if (EPI == kEpiDequantBf16) sc = (row < p.M ? __ldg(p.x_scale + row) : 0.0f) * sw;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
+      if (epi_is_dequant(EPI)) sc = (row < p.M ? __ldg(p.x_scale + row) : 0.0f) * sw;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(b * BN + half * BN_HALF);
       const uint32_t release_addr = map_to_rank(&tmem_empty[b], 0);
-      epilogue_tile<EPI>(&tmOut, p, t_row, row0, nb * BN, sc, ebuf0, chunk_count, lane,
-                         [&]() { mbar_arrive_cluster(release_addr); });
+      epilogue_tile<EPI, BN_HALF / CHUNK>(&tmOut, p, t_row, row0, nb * BN + half * BN_HALF, sc, ebuf0, chunk_count,
+                                          lane, [&]() { mbar_arrive_cluster(release_addr); });
     }
     if (!ok && lane == 0) raise_abort(abort, p.status);
     if (lane == 0) bulk_wait_group<0>();
@@ -951,7 +1057,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     const int q = warp & 3;
-    const float sw = (EPI == kEpiDequantBf16) ? __ldg(p.w_scale) : 0.0f;
+    const float sw = epi_weight_scale<EPI>(p);
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -959,7 +1065,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       const int n = tile * SM_BW + q * 32 + lane;
       float bn = 0.0f;
-      if (EPI == kEpiDequantBf16 && p.bias != nullptr && n < p.N) bn = __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16);
+      float swn = sw;  // this thread's output channel's weight scale
+      if (epi_is_dequant(EPI) && n < p.N) {
+        if (p.bias != nullptr) bn = out16_to_f32(__ldg(p.bias + n), epi_is_general(EPI) && p.out_f16 != 0);
+        if (epi_is_general(EPI) && p.wscale_per_channel) swn = __ldg(p.w_scale + n);
+      }
       if (!mbar_wait_bounded(&tmem_full[b], use & 1u, abort, p.timeout_ns)) {
         ok = false;
         break;
@@ -985,6 +1095,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * sw, bn);
             const __nv_bfloat16 h = __float2bfloat16_rn(y);
             static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = h;
+          } else if (epi_is_general(EPI)) {
+            float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * swn, bn);
+            if (EPI == kEpiDequantGenGelu) y = gelu_erf(y);
+            if (p.out_f16)
+              static_cast<__half*>(out)[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(y);
+            else
+              static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(y);
           } else {
             static_cast<int32_t*>(out)[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[j]);
           }
@@ -1066,8 +1183,10 @@ cudaError_t launch_impl(const int8_t* A, const int8_t* B, void* out, GemmParams 
       !encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   bool ok_out;
-  if (EPI == kEpiDequantBf16)
-    ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (epi_is_dequant(EPI))
+    ok_out = encode_2d(&to, (epi_is_general(EPI) && p.out_f16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   else
     ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok_out) return cudaErrorInvalidValue;
@@ -1127,8 +1246,10 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
       !encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, BN_HALF, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   bool ok_out;
-  if (EPI == kEpiDequantBf16)
-    ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (epi_is_dequant(EPI))
+    ok_out = encode_2d(&to, (epi_is_general(EPI) && p.out_f16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   else
     ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok_out) return cudaErrorInvalidValue;
@@ -1149,7 +1270,7 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(PAIR_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
@@ -1203,15 +1324,21 @@ cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out,
                            cudaStream_t stream) {
   if (p.M <= kSmallM && p.single_sm == 0) {
     if (epi == kEpiDequantBf16) return launch_smallm<kEpiDequantBf16>(A, B, out, p, stream);
+    if (epi == kEpiDequantGen) return launch_smallm<kEpiDequantGen>(A, B, out, p, stream);
+    if (epi == kEpiDequantGenGelu) return launch_smallm<kEpiDequantGenGelu>(A, B, out, p, stream);
     if (epi == kEpiRawS32) return launch_smallm<kEpiRawS32>(A, B, out, p, stream);
     return cudaErrorInvalidValue;
   }
   if (p.single_sm == 0) {
     if (epi == kEpiDequantBf16) return launch_pair<kEpiDequantBf16>(A, B, out, p, stream);
+    if (epi == kEpiDequantGen) return launch_pair<kEpiDequantGen>(A, B, out, p, stream);
+    if (epi == kEpiDequantGenGelu) return launch_pair<kEpiDequantGenGelu>(A, B, out, p, stream);
     if (epi == kEpiRawS32) return launch_pair<kEpiRawS32>(A, B, out, p, stream);
     return cudaErrorInvalidValue;
   }
   if (epi == kEpiDequantBf16) return launch_impl<kEpiDequantBf16, 0>(A, B, out, p, stream);
+  if (epi == kEpiDequantGen) return launch_impl<kEpiDequantGen, 0>(A, B, out, p, stream);
+  if (epi == kEpiDequantGenGelu) return launch_impl<kEpiDequantGenGelu, 0>(A, B, out, p, stream);
   if (epi == kEpiRawS32) return launch_impl<kEpiRawS32, 0>(A, B, out, p, stream);
   return cudaErrorInvalidValue;
 }

@@ -10,13 +10,23 @@ namespace convrot {
 enum GemmEpilogue : int {
   kEpiDequantBf16 = 0,  // Y = bf16_rne(float(acc) * (x_scale[m] * w_scale) + bias[n])
   kEpiRawS32 = 1,       // acc as int32
+  // Y = out_rne(float(acc) * (x_scale[m] * w_scale[n or 0]) + bias[n]) with the
+  // run-time options below (per-channel weight scale, fp16 output and bias)
+  kEpiDequantGen = 2,
+  kEpiDequantGenGelu = 3,  // the same followed by GELU (exact erf)
 };
+
+// true for the epilogues that write a 2-byte dequantised output
+__host__ __device__ constexpr bool epi_is_dequant(int epi) { return epi != kEpiRawS32; }
+__host__ __device__ constexpr bool epi_is_general(int epi) { return epi == kEpiDequantGen || epi == kEpiDequantGenGelu; }
 
 struct GemmParams {
   int M, N, K;
   const float* x_scale;   // [M]   (dequant epilogue)
   const float* w_scale;   // [1]   (dequant epilogue)
-  const uint16_t* bias;   // [N] bf16 bits or null
+  const uint16_t* bias;   // [N] bf16 (fp16 with out_f16) bits or null
+  int wscale_per_channel; // kEpiDequantGen(Gelu): w_scale holds N floats (one per output channel)
+  int out_f16;            // kEpiDequantGen(Gelu): Y and bias are IEEE fp16 instead of bf16
   int* status;            // status word: a timed-out wait ORs 5 into it
   uint64_t timeout_ns;    // bound of every device-side wait
   int group_m;            // M-blocks per raster group (0 = default)

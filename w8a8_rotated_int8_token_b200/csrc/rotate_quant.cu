@@ -28,6 +28,7 @@
 // copies, the next block in flight while the current one is computed. The row
 // absmax is reduced in shared memory, with one CTA barrier per block.
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -42,7 +43,19 @@ namespace convrot {
 using namespace fwht;
 
 
-template <int G, int MODE>
+// bf16 (F16IN false) or IEEE fp16 (true) input words: two elements each,
+// widened exactly to float32 (low half first).
+template <bool F16IN>
+__device__ __forceinline__ float2 widen2(uint32_t w) {
+  if (F16IN) {
+    __half2 h;
+    *reinterpret_cast<uint32_t*>(&h) = w;
+    return __half22float2(h);
+  }
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+template <int G, int MODE, bool F16IN>
 __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   constexpr int LG = G / 64;
   constexpr int PIECE = G / 8;  // elements between consecutive pieces of a lane
@@ -138,9 +151,9 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          v[jj][2 * q] = make_float2(__uint_as_float(aw[q] << 16), __uint_as_float(bw[q] << 16));
-          v[jj][2 * q + 1] =
-              make_float2(__uint_as_float(aw[q] & 0xFFFF0000u), __uint_as_float(bw[q] & 0xFFFF0000u));
+          const float2 fa = widen2<F16IN>(aw[q]), fb = widen2<F16IN>(bw[q]);
+          v[jj][2 * q] = make_float2(fa.x, fb.x);
+          v[jj][2 * q + 1] = make_float2(fa.y, fb.y);
         }
       }
     }
@@ -270,9 +283,9 @@ bool rotquant_shape(int64_t K, int* threads_per_row, int* rows_per_cta) {
 
 namespace {
 
-template <int G, int MODE>
+template <int G, int MODE, bool F16IN>
 cudaError_t launch_typed(RotQuantParams p, cudaStream_t stream) {
-  void (*kern)(RotQuantParams) = rotate_quant_kernel<G, MODE>;
+  void (*kern)(RotQuantParams) = rotate_quant_kernel<G, MODE, F16IN>;
   const int threads = (p.rows_per_cta * p.threads_per_row + 31) / 32 * 32;
   const size_t smem = static_cast<size_t>(kRqStages) * rotquant_slot_bytes(p.rows_per_cta, p.K);
   int dev = 0;
@@ -328,21 +341,20 @@ cudaError_t launch_typed(RotQuantParams p, cudaStream_t stream) {
 
 }  // namespace
 
+template <int G, bool F16IN>
+cudaError_t launch_mode(int mode, RotQuantParams p, cudaStream_t stream) {
+  if (mode == kRqActivation) return launch_typed<G, kRqActivation, F16IN>(p, stream);
+  if (mode == kRqWeightAbsmax) return launch_typed<G, kRqWeightAbsmax, F16IN>(p, stream);
+  return launch_typed<G, kRqWeightQuant, F16IN>(p, stream);
+}
+
 cudaError_t launch_rotate_quant(int g, int mode, RotQuantParams p, cudaStream_t stream) {
   int tpr = 0, rpc = 0;
   if (!rotquant_shape(p.K, &tpr, &rpc)) return cudaErrorInvalidValue;
   p.threads_per_row = tpr;
   p.rows_per_cta = rpc;
-  if (g == 256) {
-    if (mode == kRqActivation) return launch_typed<256, kRqActivation>(p, stream);
-    if (mode == kRqWeightAbsmax) return launch_typed<256, kRqWeightAbsmax>(p, stream);
-    return launch_typed<256, kRqWeightQuant>(p, stream);
-  }
-  if (g == 128) {
-    if (mode == kRqActivation) return launch_typed<128, kRqActivation>(p, stream);
-    if (mode == kRqWeightAbsmax) return launch_typed<128, kRqWeightAbsmax>(p, stream);
-    return launch_typed<128, kRqWeightQuant>(p, stream);
-  }
+  if (g == 256) return p.in_f16 ? launch_mode<256, true>(mode, p, stream) : launch_mode<256, false>(mode, p, stream);
+  if (g == 128) return p.in_f16 ? launch_mode<128, true>(mode, p, stream) : launch_mode<128, false>(mode, p, stream);
   return cudaErrorInvalidValue;
 }
 

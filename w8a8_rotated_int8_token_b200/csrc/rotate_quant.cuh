@@ -19,7 +19,8 @@ constexpr int kRqTimeoutStatus = 5;   // CONVROT_ERR_DEVICE_TIMEOUT
 constexpr int kRotQuantMaxThreads = 512;  // K/64 threads per row: K <= 32768
 
 struct RotQuantParams {
-  const uint16_t* src;      // [rows, K] bf16 bits
+  const uint16_t* src;      // [rows, K] bf16 bits (IEEE fp16 bits with in_f16)
+  int in_f16;               // 0: bf16 input, 1: fp16 input
   int64_t rows;
   int64_t K;
   int8_t* dst;              // [rows, K] codes (unused in kRqWeightAbsmax)
