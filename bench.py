@@ -8,6 +8,7 @@ g=256, with bias.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
     python bench.py --impl reference ...   # the CPU oracle as the reference arm
+    python bench.py --dtype f16 --wscale channel --act gelu   # a layer variant (convrot_linear_ex)
 
 Under torchrun (N > 1) every rank runs an independent replica of the same
 workload on its own GPU (the layer has no cross-GPU step); the value is the
@@ -41,8 +42,8 @@ INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B2
 # GEMM_SOURCES must match, otherwise the bench reports null.
 GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh", "fwht_dev.cuh"]
 GEMM_TRAFFIC = {
-    "dit_qkv_1024": {"bytes": 59430656 + 48917504,
-                     "sources_sha256": "ff470c56cf1c1a7484ad1b4ec2401cf7d68cd6981399e267c08053dcb8d056da"},
+    "dit_qkv_1024": {"bytes": 60029696 + 49044224,
+                     "sources_sha256": "93c2b5d64aa264a58d36511b1cfe83357739fedb0b849c8efb702d162d86e95f"},
 }
 
 
@@ -69,6 +70,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    # layer variants (convrot_linear_ex); the defaults are the headline layer
+    ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16", help="dtype of X, W, bias and Y")
+    ap.add_argument("--wscale", choices=["tensor", "channel"], default="tensor", help="weight-scale granularity")
+    ap.add_argument("--act", choices=["none", "gelu"], default="none", help="activation fused into the epilogue")
     return ap.parse_args()
 
 
@@ -272,11 +277,21 @@ def main():
     M, K, N, g = w.M, w.K, w.N, w.g
     L = cr.lib()
 
+    variant = (args.dtype, args.wscale, args.act) != ("bf16", "tensor", "none")
+    io_dtype = torch.bfloat16 if args.dtype == "bf16" else torch.float16
+    dt_code = cr.DTYPE_BF16 if args.dtype == "bf16" else cr.DTYPE_F16
+    ws_mode = cr.WSCALE_TENSOR if args.wscale == "tensor" else cr.WSCALE_CHANNEL
+    act_code = cr.ACT_NONE if args.act == "none" else cr.ACT_GELU_ERF
+
     def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        return t if io_dtype == torch.bfloat16 else t.to(io_dtype)  # the same values in fp16
 
     W = to_dev(d["w"])
-    Wq0, sw = cr.convrot_prepare_weight(W, g)
+    if variant:
+        Wq0, sw = cr.convrot_prepare_weight_ex(W, g, ws_mode)
+    else:
+        Wq0, sw = cr.convrot_prepare_weight(W, g)
     del W
     bias = None if d["bias"] is None else to_dev(d["bias"])
     X0 = to_dev(d["x"])
@@ -285,7 +300,7 @@ def main():
     for i in range(N_SETS):
         sets.append({
             "X": X0.clone(), "Wq": Wq0.clone(),
-            "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+            "Y": torch.empty((M, N), dtype=io_dtype, device=dev),
             "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=dev),
         })
     del X0
@@ -296,8 +311,12 @@ def main():
 
     def step(i):
         s = sets[i % N_SETS]
-        st = L.convrot_linear(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw_ptr, N, b_ptr, s["Y"].data_ptr(),
-                              s["ws"].data_ptr(), ws_bytes, sp)
+        if variant:
+            st = L.convrot_linear_ex(s["X"].data_ptr(), dt_code, M, K, g, s["Wq"].data_ptr(), sw_ptr, ws_mode, N,
+                                     b_ptr, act_code, s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, sp)
+        else:
+            st = L.convrot_linear(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw_ptr, N, b_ptr,
+                                  s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, sp)
         if st != 0:
             raise cr.ConvRotError(st, "convrot_linear")
 
@@ -340,17 +359,20 @@ def main():
         if st != 0:
             raise cr.ConvRotError(st, "convrot_linear_timed")
 
-    for i in range(args.warmup):
-        timed_step(i, ev[i % len(ev)])
-    torch.cuda.synchronize(dev)
-    barrier()
-    for i in range(args.steps):
-        timed_step(i, ev[i])
-    torch.cuda.synchronize(dev)
-    barrier()
-    t_layer = max_over_ranks(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
-    t_first = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
-    t_second = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    if not variant:
+        for i in range(args.warmup):
+            timed_step(i, ev[i % len(ev)])
+        torch.cuda.synchronize(dev)
+        barrier()
+        for i in range(args.steps):
+            timed_step(i, ev[i])
+        torch.cuda.synchronize(dev)
+        barrier()
+        t_layer = max_over_ranks(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
+        t_first = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+        t_second = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    # (variants: no per-launch events; the GEMM's time is the layer's minus the
+    # standalone rotate+quantise kernel's, below)
 
     # ---- the two stages as standalone kernels, each timed alone back to back (context)
     xq = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(N_SETS)]
@@ -359,7 +381,11 @@ def main():
 
     def q_only(i):
         j = i % N_SETS
-        L.convrot_quant_act(sets[j]["X"].data_ptr(), M, K, g, xq[j].data_ptr(), xsc[j].data_ptr(), sp)
+        if variant:
+            L.convrot_quant_act_ex(sets[j]["X"].data_ptr(), dt_code, M, K, g, xq[j].data_ptr(), xsc[j].data_ptr(),
+                                   sp)
+        else:
+            L.convrot_quant_act(sets[j]["X"].data_ptr(), M, K, g, xq[j].data_ptr(), xsc[j].data_ptr(), sp)
 
     def g_only(i):
         j = i % N_SETS
@@ -381,28 +407,35 @@ def main():
 
     n_alone = max(1, min(args.steps, 200))
     t_q = time_loop(q_only, n_alone)
-    t_g = time_loop(g_only, n_alone)
+    t_g = None if variant else time_loop(g_only, n_alone)
     del xq, xsc
+    if variant:
+        t_layer = t_ms / args.steps
+        t_first = t_q
+        t_second = t_layer - t_q
 
     peaks, peak_src = load_peaks()
     int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
     layer_tops = ops / (t_layer * 1e-3) / 1e12
-    gemm_tops = ops / (t_g * 1e-3) / 1e12
+    gemm_tops = None if t_g is None else ops / (t_g * 1e-3) / 1e12
     q_bytes = 3.0 * M * K + 4.0 * M
     q_gbs = q_bytes / (t_q * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        xh = [torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16)).view(torch.bfloat16).pin_memory()
-              for _ in range(2)]
-        yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        xh = [torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16)).view(torch.bfloat16).to(io_dtype)
+              .pin_memory() for _ in range(2)]
+        yh = [torch.empty((M, N), dtype=io_dtype).pin_memory() for _ in range(2)]
         e2e_steps = max(1, min(args.steps, 200))
 
         def e2e_step(i):
             s = sets[i % N_SETS]
             s["X"].copy_(xh[i % 2], non_blocking=True)
-            cr.convrot_linear(s["X"], s["Wq"], sw, g, bias, Y=s["Y"], ws=s["ws"])
+            if variant:
+                cr.convrot_linear_ex(s["X"], s["Wq"], sw, g, bias, act_code, Y=s["Y"], ws=s["ws"])
+            else:
+                cr.convrot_linear(s["X"], s["Wq"], sw, g, bias, Y=s["Y"], ws=s["ws"])
             yh[i % 2].copy_(s["Y"], non_blocking=True)
 
         for i in range(min(args.warmup, 5)):
@@ -422,7 +455,8 @@ def main():
 
     cpu = None
     parity = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    # the oracle leg reproduces the headline layer; variants report none
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         y_all = sets[(args.steps - 1) % N_SETS]["Y"].float().cpu().numpy().astype(np.float64)
         cpu, parity = cpu_oracle_leg(d, args.cpu_seconds, y_all)
 
@@ -442,9 +476,11 @@ def main():
                      "kernel": ("gemm_i8_pair_kernel (tcgen05.mma.cta_group::2 kind::i8, dequant/bias epilogue)"
                                 if launches == 2 else "gemm_i8_kernel with fused rotate+quantise workers"),
                      "achieved": dom_tops, "peak": int8_peak, "unit": "TOPS", "frac": dom_tops / int8_peak,
-                     "traffic": gemm_traffic(args.config) if launches == 2 else None,
+                     "traffic": gemm_traffic(args.config) if launches == 2 and not variant else None,
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "us_per_launch": t_dom * 1e3,
+                     "us_source": ("layer time minus the standalone rotate+quantise kernel" if variant
+                                   else "CUDA events around the GEMM launch inside each step"),
                      "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
                                     "(nominal int8:bf16 dense ratio)"},
         "layer_us_per_call_events": t_layer * 1e3,
@@ -455,15 +491,20 @@ def main():
             "rotate_quant_kernel (standalone, timed alone)": {
                 "us": t_q * 1e3, "bound": "hbm", "achieved": q_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "frac": q_gbs / peaks["hbm_gbs"], "algorithmic_bytes": q_bytes},
-            "gemm_i8_kernel (GEMM + epilogue only, timed alone incl. 4-byte status memset)": {
-                "us": t_g * 1e3, "bound": "tensor", "achieved": gemm_tops, "unit": "TOPS", "peak": int8_peak,
-                "frac": gemm_tops / int8_peak, "ops": ops},
         },
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
     }
+    if variant:  # no per-launch events in a variant run: only the standalone timing is real
+        del out["kernels"]["rotate_quant_kernel (first launch of the step, events)"]
+    if t_g is not None:
+        out["kernels"]["gemm_i8_kernel (GEMM + epilogue only, timed alone incl. 4-byte status memset)"] = {
+            "us": t_g * 1e3, "bound": "tensor", "achieved": gemm_tops, "unit": "TOPS", "peak": int8_peak,
+            "frac": gemm_tops / int8_peak, "ops": ops}
+    if variant:
+        out["config"]["variant"] = {"io_dtype": args.dtype, "weight_scale": args.wscale, "activation": args.act}
     if parity is not None:
         out["parity_nrmse_vs_oracle_sample"] = parity
     print(json.dumps(out), flush=True)
