@@ -77,6 +77,24 @@ def parse_args():
     return ap.parse_args()
 
 
+def reduce_max(v: float, device) -> float:
+    """The maximum of v over the ranks of the default process group (v itself
+    with one rank): every multi-rank time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(ops_per_step: float, steps: int, world: int, t_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks over the (max-over-ranks) time."""
+    return ops_per_step * steps * world / (t_ms * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -266,11 +284,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dev)
 
     d = synth.make_workload(args.config)
     w = d["workload"]
@@ -341,7 +355,7 @@ def main():
         if st != 0:
             raise cr.ConvRotError(st, "device status after the timed region")
     ops = 2.0 * M * N * K
-    value = ops * args.steps * world / (t_ms * 1e-3) / 1e12
+    value = job_tops(ops, args.steps, world, t_ms)
 
     # ---- the layer kernel timed per launch: events recorded around each call on its stream
     launches = L.convrot_linear_launch_count(M, N, K, g)
@@ -449,7 +463,7 @@ def main():
         torch.cuda.synchronize(dev)
         barrier()
         t_e2e = max_over_ranks(ev0.elapsed_time(ev1))
-        e2e = {"value": ops * e2e_steps * world / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_tops(ops, e2e_steps, world, t_e2e), "unit": UNIT,
                "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(yh[0].numel() * 2),
                "steps": e2e_steps, "ms_per_step": t_e2e / e2e_steps}
 
