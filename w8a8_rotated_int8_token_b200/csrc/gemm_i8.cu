@@ -775,8 +775,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     const int nk = p.num_k_blocks < 32 ? p.num_k_blocks : 32;
     for (int kb = 0; kb < nk; ++kb) tma_prefetch_2d(&tmB, kb * BK, nb * BN + static_cast<int>(rank) * BN_HALF);
   }
-  griddep_wait();
-
+  // Only the activation codes and token scales come from the previous kernel
+  // (the rotate+quantise launch, which releases this one only after its own
+  // predecessor has finished): the producer waits for it before its first A
+  // load, the epilogue before its first token scale; the weight loads of the
+  // first S stages go out before that wait.
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -785,6 +788,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
       uint32_t ph = 0;
       int64_t issued = 0;
       bool ok = true;
+      auto load_a = [&](int st, int kb, int mb2) {
+        tma_load_2d_pair(smem + L::kOffA + st * PA_STAGE_BYTES, &tmA, map_to_rank(&full[st], 0), kb * BK,
+                         mb2 * 2 * BM + static_cast<int>(rank) * BM);
+      };
+      int early_s[S], early_kb[S], early_mb[S];
+      int n_early = 0;
+      bool waited = false;
+      auto release_early = [&]() {  // wait for the previous kernel, then the A loads held back
+        griddep_wait();
+        waited = true;
+        for (int i = 0; i < n_early; ++i) load_a(early_s[i], early_kb[i], early_mb[i]);
+      };
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         int mb2, nb;
         pair_tile_coords(tile, p, mb2, nb);
@@ -795,10 +810,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
           }
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * (PA_STAGE_BYTES + PB_STAGE_BYTES));
           const uint32_t bar_leader = map_to_rank(&full[s], 0);
-          tma_load_2d_pair(smem + L::kOffA + s * PA_STAGE_BYTES, &tmA, bar_leader, kb * BK,
-                           mb2 * 2 * BM + static_cast<int>(rank) * BM);
           tma_load_2d_pair(smem + L::kOffB + s * PB_STAGE_BYTES, &tmB, bar_leader, kb * BK,
                            nb * BN + static_cast<int>(rank) * BN_HALF);
+          if (waited) {
+            load_a(s, kb, mb2);
+          } else {
+            early_s[n_early] = s;
+            early_kb[n_early] = kb;
+            early_mb[n_early] = mb2;
+            if (++n_early == S) release_early();
+          }
           ++issued;
           if (++s == S) {
             s = 0;
@@ -806,6 +827,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
           }
         }
       }
+      if (!waited) release_early();  // fewer than S stages in all, or a timed-out wait
       griddep_launch_dependents();
       if (!ok) raise_abort(abort, p.status);
       // the last stages are released (MMAs done reading this CTA's operands and
@@ -857,6 +879,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------ epilogue (both)
+    griddep_wait();            // the token scales come from the previous kernel
     const int ew = warp - 2;   // 0..7
     const int q = warp & 3;    // TMEM lane quarter this warp may access
     const int half = ew >> 2;  // which 128 of the tile's 256 columns
@@ -981,7 +1004,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
-  griddep_wait();
+  // The weight stream does not depend on the previous kernel (see the pair
+  // kernel): the weight loads of the first S stages go out before the wait,
+  // the activation-code loads and the token scales after it.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -990,6 +1015,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int pending_phase[S];
       for (int i = 0; i < S; ++i) pending_phase[i] = -1;
       bool ok = true;
+      int early_s[S], early_kb[S];
+      int n_early = 0;
+      bool waited = false;
+      auto release_early = [&]() {
+        griddep_wait();
+        waited = true;
+        for (int i = 0; i < n_early; ++i)
+          tma_load_2d(smem + L::kOffX + early_s[i] * L::kX, &tmX, &full[early_s[i]], early_kb[i] * BK, 0);
+      };
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < p.num_k_blocks; ++kb) {
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort, p.timeout_ns)) {
@@ -998,7 +1032,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           mbar_arrive_expect_tx(&full[s], L::kW + L::kX);
           tma_load_2d(smem + L::kOffW + s * L::kW, &tmW, &full[s], kb * BK, tile * SM_BW);
-          tma_load_2d(smem + L::kOffX + s * L::kX, &tmX, &full[s], kb * BK, 0);
+          if (waited) {
+            tma_load_2d(smem + L::kOffX + s * L::kX, &tmX, &full[s], kb * BK, 0);
+          } else {
+            early_s[n_early] = s;
+            early_kb[n_early] = kb;
+            if (++n_early == S) release_early();
+          }
           pending_phase[s] = static_cast<int>(ph);
           if (++s == S) {
             s = 0;
@@ -1006,6 +1046,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      if (!waited) release_early();
       griddep_launch_dependents();
       if (!ok) {
         raise_abort(abort, p.status);
@@ -1056,6 +1097,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_bounded(drain, 0u, nullptr, p.timeout_ns);
     }
   } else {
+    griddep_wait();  // the token scales come from the previous kernel
     const int q = warp & 3;
     const float sw = epi_weight_scale<EPI>(p);
     int it = 0;
