@@ -14,6 +14,7 @@ from .convrot_oracle import (  # noqa: F401
     gemm_s32,
     hadamard,
     linear,
+    linear_ex,
     nrmse,
     prepare_weight,
     prepare_weight_per_channel,

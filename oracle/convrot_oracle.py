@@ -200,6 +200,24 @@ def gelu_erf(y: np.ndarray) -> np.ndarray:
     return 0.5 * y * (1.0 + erf(y / np.sqrt(2.0)))
 
 
+def linear_ex(x: np.ndarray, wq: np.ndarray, s_w, g: int, bias: np.ndarray | None = None,
+              addend: np.ndarray | None = None, gelu: bool = False) -> np.ndarray:
+    """The layer with its variants, float64: rotate + per-token quantise X, int8 GEMM,
+    dequantise with a tensor (scalar s_w) or per-output-channel (s_w [N]) weight
+    scale, add the bias, add `addend` [M,N] (a term computed beside the int8
+    layer, as a LoRA is: InvokeAI "int8 Compute", after the list in "What stays
+    on the default path": applied beside the int8 layer in the compute
+    precision, never quantised), then GELU if asked.
+    """
+    xq, s_x = quant_act(x, g)
+    acc = gemm_s32(xq, wq)
+    s_w = np.asarray(s_w)
+    y = dequant_per_channel(acc, s_x, s_w, bias) if s_w.ndim == 1 and s_w.size > 1 else dequant(acc, s_x, s_w, bias)
+    if addend is not None:
+        y = y + np.asarray(addend, np.float64)
+    return gelu_erf(y) if gelu else y
+
+
 def linear(x: np.ndarray, wq: np.ndarray, s_w: float, g: int,
            bias: np.ndarray | None = None) -> np.ndarray:
     """One ConvRot linear call: rotate + per-token quantise X, int8 GEMM, dequantise."""

@@ -423,3 +423,36 @@ def test_dequant_per_channel_hand_case_and_tensorwise_limit():
     sx = rng.random(5).astype(np.float32)
     np.testing.assert_array_equal(oracle.dequant_per_channel(acc, sx, np.full(7, 0.25, np.float32)),
                                   oracle.dequant(acc, sx, np.float32(0.25)))
+
+
+def test_linear_ex_reduces_to_its_parts():
+    # the composed variant equals its definition step by step, and with no
+    # options it is exactly the plain layer
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((5, 256))
+    w = rng.standard_normal((8, 256)) * 0.02
+    b = rng.standard_normal(8) * 0.01
+    z = rng.standard_normal((5, 8)) * 0.05
+    wq, sw = oracle.prepare_weight(w, 256)
+    np.testing.assert_array_equal(oracle.linear_ex(x, wq, sw, 256, b), oracle.linear(x, wq, sw, 256, b))
+    y0 = oracle.linear(x, wq, sw, 256, b)
+    np.testing.assert_array_equal(oracle.linear_ex(x, wq, sw, 256, b, addend=z), y0 + z)
+    np.testing.assert_array_equal(oracle.linear_ex(x, wq, sw, 256, b, addend=z, gelu=True), oracle.gelu_erf(y0 + z))
+    wqc, swc = oracle.prepare_weight_per_channel(w, 256)
+    xq, sx = oracle.quant_act(x, 256)
+    ref = oracle.gemm_s32(xq, wqc) * (sx[:, None].astype(np.float64) * swc[None, :].astype(np.float64)) + b
+    np.testing.assert_array_equal(oracle.linear_ex(x, wqc, swc, 256, b), ref)
+
+
+def test_addend_hand_case():
+    # one token, one output: x = 4 e_0 in a 256-group -> codes 127 * sign pattern / 127 ...
+    # built so the accumulator is known: x rotated is c/16 * H[0,:] = all +c/16, so s_x = c/(16*127)
+    # and every code is 127; a weight row equal to e_0 rotates to all +1/16, codes 127, s_w = 1/(16*127)
+    x = np.zeros((1, 256))
+    x[0, 0] = 4.0
+    w = np.zeros((1, 256))
+    w[0, 0] = 1.0
+    wq, sw = oracle.prepare_weight(w, 256)
+    y = oracle.linear_ex(x, wq, sw, 256, bias=np.array([0.5]), addend=np.array([[-0.25]]))
+    # acc = 256 * 127^2; y = acc * s_x * s_w + 0.5 - 0.25 = x . w + 0.25 = 4.25 (to float32 rounding of the scales)
+    assert abs(y[0, 0] - 4.25) < 1e-6

@@ -34,6 +34,7 @@ MUTATIONS = {
                          "return bf16_to_f64(bits)"),
     "per_channel_scale_tensorwise": ("    return quantize_per_token(rotate(w, g))\n",
                                      "    q, s = quantize_tensorwise(rotate(w, g))\n    return q, np.full(q.shape[0], s)\n"),
+    "addend_dropped": ("        y = y + np.asarray(addend, np.float64)\n", "        y = y\n"),
     "per_channel_scale_on_tokens_axis": ("np.asarray(s_w, np.float64)[None, :])", "np.asarray(s_w, np.float64)[:, None])"),
 }
 
