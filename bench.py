@@ -326,8 +326,9 @@ def main():
     def step(i):
         s = sets[i % N_SETS]
         if variant:
-            st = L.convrot_linear_ex(s["X"].data_ptr(), dt_code, M, K, g, s["Wq"].data_ptr(), sw_ptr, ws_mode, N,
-                                     b_ptr, act_code, s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, sp)
+            st = L.convrot_linear_ex(s["X"].data_ptr(), dt_code, M, K, 0, g, s["Wq"].data_ptr(), sw_ptr, ws_mode,
+                                     N, b_ptr, None, act_code, s["Y"].data_ptr(), 0, s["ws"].data_ptr(), ws_bytes,
+                                     sp)
         else:
             st = L.convrot_linear(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw_ptr, N, b_ptr,
                                   s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, sp)
@@ -396,8 +397,8 @@ def main():
     def q_only(i):
         j = i % N_SETS
         if variant:
-            L.convrot_quant_act_ex(sets[j]["X"].data_ptr(), dt_code, M, K, g, xq[j].data_ptr(), xsc[j].data_ptr(),
-                                   sp)
+            L.convrot_quant_act_ex(sets[j]["X"].data_ptr(), dt_code, M, K, 0, g, xq[j].data_ptr(),
+                                   xsc[j].data_ptr(), sp)
         else:
             L.convrot_quant_act(sets[j]["X"].data_ptr(), M, K, g, xq[j].data_ptr(), xsc[j].data_ptr(), sp)
 

@@ -165,25 +165,36 @@ CONVROT_API convrot_status convrot_prepare_weight_ex(const void* W, int dtype, i
                                                      size_t ws_bytes, convrot_stream_t stream);
 
 /*
- * convrot_quant_act_ex -- convrot_quant_act with X in `dtype` (bf16 or fp16).
+ * convrot_quant_act_ex -- convrot_quant_act with X in `dtype` (bf16 or fp16)
+ * and a row stride: row m of X starts ldx elements after row m-1 (ldx >= K,
+ * a multiple of 8; 0 means K). Xq and x_scale stay dense.
  */
-CONVROT_API convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t K, int g,
-                                                int8_t* Xq, float* x_scale, convrot_stream_t stream);
+CONVROT_API convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t K, int64_t ldx,
+                                                int g, int8_t* Xq, float* x_scale, convrot_stream_t stream);
 
 /*
- * convrot_linear_ex -- convrot_linear with the variants above:
- *   Y = out_rne( act( (Xq Wq^T) * (s_x[m] * s_w[n or 0]) + bias[n] ) ).
- *   dtype        type of X, bias and Y (CONVROT_DTYPE_BF16 or CONVROT_DTYPE_F16).
+ * convrot_linear_ex -- convrot_linear with the variants above, an addend and row strides:
+ *   Y = out_rne( act( (Xq Wq^T) * (s_x[m] * s_w[n or 0]) + bias[n] + addend[m,n] ) ).
+ *   dtype        type of X, bias, addend and Y (CONVROT_DTYPE_BF16 or CONVROT_DTYPE_F16).
+ *   ldx          row stride of X in elements (>= K, a multiple of 8; 0 = K).
  *   w_scale      1 float (CONVROT_WSCALE_TENSOR) or [N] floats, 16-byte aligned
  *                (CONVROT_WSCALE_CHANNEL), from convrot_prepare_weight_ex.
+ *   addend       [M, ldy] in `dtype`, 16-byte aligned, or NULL: a term computed
+ *                beside the int8 layer in the compute precision and never
+ *                quantised -- how the pages apply a LoRA to an int8 layer
+ *                (InvokeAI "int8 Compute", after the list in "What stays on
+ *                the default path") -- added in float32 before the activation
+ *                and the single output rounding. It may not overlap Y.
  *   activation   CONVROT_ACT_NONE or CONVROT_ACT_GELU_ERF.
+ *   ldy          row stride of Y and of addend in elements (>= N, a multiple of 8; 0 = N).
  * Other arguments, the workspace and the errors as convrot_linear. With bf16,
- * a tensor scale and no activation it is exactly convrot_linear.
+ * dense rows, a tensor scale, no addend and no activation it is exactly
+ * convrot_linear.
  */
-CONVROT_API convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K, int g,
+CONVROT_API convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K, int64_t ldx, int g,
                                              const int8_t* Wq, const float* w_scale, int wscale_mode, int64_t N,
-                                             const void* bias, int activation, void* Y, void* ws, size_t ws_bytes,
-                                             convrot_stream_t stream);
+                                             const void* bias, const void* addend, int activation, void* Y,
+                                             int64_t ldy, void* ws, size_t ws_bytes, convrot_stream_t stream);
 
 /*
  * convrot_linear_timed -- convrot_linear that also records caller-created CUDA

@@ -62,7 +62,7 @@ def linear_ws_layout(M, K):
 
 
 def test_status_strings_and_version(L):
-    assert L.convrot_abi_version() == 3
+    assert L.convrot_abi_version() == 4
     for code in range(6):
         s = L.convrot_status_string(code)
         assert s and s != b"unknown status"
@@ -129,12 +129,14 @@ def test_other_entry_points_reject_bad_arguments_on_host(L):
 
 
 def test_variant_entry_points_reject_bad_arguments_on_host(L):
-    # convrot_linear_ex(X, dtype, M, K, g, Wq, w_scale, wscale_mode, N, bias, activation, Y, ws, ws_bytes, stream)
-    ok = (FAKE, 0, 64, 256, 256, FAKE, FAKE, 0, 256, None, 0, FAKE, FAKE, 1 << 30, None)
+    # convrot_linear_ex(X, dtype, M, K, ldx, g, Wq, w_scale, wscale_mode, N, bias, addend, activation, Y, ldy,
+    #                   ws, ws_bytes, stream)
+    names = ["X", "dtype", "M", "K", "ldx", "g", "Wq", "w_scale", "mode", "N", "bias", "addend", "act", "Y", "ldy",
+             "ws", "ws_bytes", "s"]
+    ok = [FAKE, 0, 64, 256, 0, 256, FAKE, FAKE, 0, 256, None, None, 0, FAKE, 0, FAKE, 1 << 30, None]
 
     def call(**over):
         a = list(ok)
-        names = ["X", "dtype", "M", "K", "g", "Wq", "w_scale", "mode", "N", "bias", "act", "Y", "ws", "ws_bytes", "s"]
         for k, v in over.items():
             a[names.index(k)] = v
         return L.convrot_linear_ex(*a)
@@ -143,6 +145,11 @@ def test_variant_entry_points_reject_bad_arguments_on_host(L):
     assert call(mode=2) == 2                       # unknown scale mode
     assert call(act=7) == 2                        # unknown activation
     assert call(mode=1, w_scale=FAKE + 4) == 1     # per-channel scales need 16-byte alignment
+    assert call(addend=FAKE + 8) == 1              # misaligned addend
+    assert call(ldx=200) == 1                      # ldx < K
+    assert call(ldx=260) == 1                      # ldx not a multiple of 8
+    assert call(ldy=255) == 1                      # ldy < N
+    assert call(ldy=260) == 1                      # ldy not a multiple of 8
     assert call(g=64) == 2
     assert call(Y=None) == 1
     assert call(ws_bytes=100) == 3
@@ -151,9 +158,10 @@ def test_variant_entry_points_reject_bad_arguments_on_host(L):
     assert L.convrot_prepare_weight_ex(FAKE, 0, 8, 256, 256, 5, FAKE, FAKE, FAKE, 256, None) == 2
     assert L.convrot_prepare_weight_ex(FAKE, 1, 8, 256, 256, 1, FAKE, FAKE + 4, None, 0, None) == 1
     assert L.convrot_prepare_weight_ex(FAKE, 1, 8, 256, 256, 0, FAKE, FAKE, None, 0, None) == 3
-    # quant_act_ex(X, dtype, M, K, g, Xq, x_scale, stream)
-    assert L.convrot_quant_act_ex(FAKE, 9, 8, 256, 256, FAKE, FAKE, None) == 2
-    assert L.convrot_quant_act_ex(FAKE, 1, 8, 300, 256, FAKE, FAKE, None) == 1
+    # quant_act_ex(X, dtype, M, K, ldx, g, Xq, x_scale, stream)
+    assert L.convrot_quant_act_ex(FAKE, 9, 8, 256, 0, 256, FAKE, FAKE, None) == 2
+    assert L.convrot_quant_act_ex(FAKE, 1, 8, 300, 0, 256, FAKE, FAKE, None) == 1
+    assert L.convrot_quant_act_ex(FAKE, 1, 8, 256, 100, 256, FAKE, FAKE, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -1,8 +1,9 @@
 """Parity of the layer's variants with the CPU oracle, on a B200, through the C ABI.
 
 Variants (convrot_*_ex): the FP16 compute dtype (X, W, bias and Y in fp16),
-one weight scale per output channel, and the exact-erf GELU fused into the
-epilogue. Each case runs in the same launch configuration as the default
+one weight scale per output channel, the exact-erf GELU fused into the
+epilogue, an addend computed beside the int8 layer (a LoRA's output), and
+strided rows of X, Y and the addend. Each case runs in the same launch configuration as the default
 layer (CTA-pair GEMM for M > 64, the weight-streaming GEMM for M <= 64) and is
 compared with the oracle's float64 result on sampled token rows.
 """
@@ -206,3 +207,58 @@ def test_gelu_epilogue_against_the_exact_function(cr, name, M):
     bound = 0.5 * ulp + 0.5 * np.abs(oracle.f16_to_f64(bb)) * 2e-7 + 1e-7 * np.abs(ref)
     for m in (0, M // 2, M - 1):
         assert np.all(np.abs(y[m] - ref) <= bound + 1e-12), np.max(np.abs(y[m] - ref) - bound)
+
+
+@pytest.mark.parametrize("name,dtype,act", [("tiny", BF16, NONE), ("dit_qkv_1024", F16, GELU),
+                                            ("textenc_m16", BF16, GELU), ("textenc_m128", F16, NONE)])
+def test_strided_rows_and_addend_match_oracle(cr, name, dtype, act):
+    # X and Y live inside wider row-major buffers (row strides K + 64 and N + 40),
+    # the addend shares Y's stride; the oracle sees the dense values
+    import torch
+
+    d = synth.make_workload(name)
+    g = d["workload"].g
+    xb = _as_dtype_bits(d["x"], dtype)
+    wb = _as_dtype_bits(d["w"], dtype)
+    bb = None if d["bias"] is None else _as_dtype_bits(d["bias"], dtype)
+    M, K = xb.shape
+    N = wb.shape[0]
+    rng = np.random.default_rng(21)
+    zb = _as_dtype_bits(synth.f32_to_bf16_bits((rng.standard_normal((M, N)) * 0.05).astype(np.float32)), dtype)
+    Wq, sw = cr.convrot_prepare_weight_ex(_to_torch(wb, dtype), g, TENSOR)
+    ldx, ldy = K + 64, N + 40
+    Xbig = _to_torch(np.zeros((M, ldx), np.uint16), dtype)
+    Xbig[:, :K] = _to_torch(xb, dtype)
+    Ybig = torch.full((M, ldy), float("nan"), dtype=Xbig.dtype, device="cuda")
+    Zbig = torch.zeros((M, ldy), dtype=Xbig.dtype, device="cuda")
+    Zbig[:, :N] = _to_torch(zb, dtype)
+    X, Y, Z = Xbig[:, :K], Ybig[:, :N], Zbig[:, :N]
+    bias = None if bb is None else _to_torch(bb, dtype)
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, N, K, g), dtype=torch.uint8, device="cuda")
+    cr.convrot_linear_ex(X, Wq, sw, g, bias, act, Y=Y, ws=ws, addend=Z)
+    assert cr.convrot_read_device_status(ws) == 0
+    torch.cuda.synchronize()
+    # the padding columns of Y were not written
+    assert torch.isnan(Ybig[:, N:]).all()
+    rows = _rows_sample(M)
+    wq_ref, sw_ref = oracle.prepare_weight(_to_f64(wb, dtype), g)
+    ref = oracle.linear_ex(_to_f64(xb[rows], dtype), wq_ref, sw_ref, g, None if bb is None else _to_f64(bb, dtype),
+                           addend=_to_f64(zb[rows], dtype), gelu=(act == GELU))
+    y = _from_torch(Y.contiguous(), dtype)[rows]
+    err = nrmse(y, ref)
+    assert err <= NRMSE_TOL, f"{name}: NRMSE {err}"
+
+
+def test_strided_quant_act_is_the_dense_one(cr):
+    import torch
+
+    d = synth.make_workload("dit_qkv_1024")
+    g = d["workload"].g
+    X = _to_torch(d["x"], BF16)
+    M, K = X.shape
+    Xbig = torch.zeros((M, K + 136), dtype=X.dtype, device="cuda")
+    Xbig[:, :K] = X
+    q0, s0 = cr.convrot_quant_act(X, g)
+    q1, s1 = cr.convrot_quant_act_ex(Xbig[:, :K], g)
+    torch.cuda.synchronize()
+    assert torch.equal(q0, q1) and torch.equal(s0, s1)

@@ -199,34 +199,43 @@ def convrot_prepare_weight_ex(W, g: int = 256, wscale_mode: int = WSCALE_TENSOR,
     return Wq, w_scale
 
 
+def _rows_view(t, name):
+    """(rows, cols, row stride in elements) of a 2-D tensor whose rows may be strided."""
+    import torch
+
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D CUDA tensor with contiguous rows")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
 def convrot_quant_act_ex(X, g: int = 256, Xq=None, x_scale=None, stream=None):
-    """convrot_quant_act for a bf16 or fp16 X [M,K]."""
+    """convrot_quant_act for a bf16 or fp16 X [M,K] whose rows may be strided."""
     import torch
 
     dtype = _dtype_code(X, "X")
-    _require(X, X.dtype, None, "X")
-    M, K = X.shape
+    M, K, ldx = _rows_view(X, "X")
     if Xq is None:
         Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
     if x_scale is None:
         x_scale = torch.empty((M,), dtype=torch.float32, device=X.device)
     _require(Xq, torch.int8, (M, K), "Xq")
     _require(x_scale, torch.float32, (M,), "x_scale")
-    _check(lib().convrot_quant_act_ex(_ptr(X), dtype, M, K, g, _ptr(Xq), _ptr(x_scale), _stream_ptr(stream)),
+    _check(lib().convrot_quant_act_ex(_ptr(X), dtype, M, K, ldx, g, _ptr(Xq), _ptr(x_scale), _stream_ptr(stream)),
            "convrot_quant_act_ex")
     return Xq, x_scale
 
 
 def convrot_linear_ex(X, Wq, w_scale, g: int = 256, bias=None, activation: int = ACT_NONE, Y=None, ws=None,
-                      stream=None):
-    """ConvRot linear in the dtype of X (bf16 or fp16; bias and Y the same), with a
-    tensor (w_scale [1]) or per-output-channel (w_scale [N]) weight scale and an
-    optional exact-erf GELU on the output."""
+                      stream=None, addend=None):
+    """ConvRot linear in the dtype of X (bf16 or fp16; bias, addend and Y the same), with a
+    tensor (w_scale [1]) or per-output-channel (w_scale [N]) weight scale, an optional
+    addend [M,N] (a term computed beside the int8 layer, e.g. a LoRA's output) and an
+    optional exact-erf GELU. X, Y and addend may have strided rows (Y and addend share
+    one row stride)."""
     import torch
 
     dtype = _dtype_code(X, "X")
-    _require(X, X.dtype, None, "X")
-    M, K = X.shape
+    M, K, ldx = _rows_view(X, "X")
     _require(Wq, torch.int8, None, "Wq")
     N = Wq.shape[0]
     if Wq.shape[1] != K:
@@ -242,13 +251,18 @@ def convrot_linear_ex(X, Wq, w_scale, g: int = 256, bias=None, activation: int =
         _require(bias, X.dtype, (N,), "bias")
     if Y is None:
         Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
-    _require(Y, X.dtype, (M, N), "Y")
+    if Y.dtype != X.dtype or tuple(Y.shape) != (M, N):
+        raise ValueError(f"Y must be [{M}, {N}] {X.dtype}")
+    _, _, ldy = _rows_view(Y, "Y")
+    if addend is not None:
+        if addend.dtype != X.dtype or tuple(addend.shape) != (M, N) or _rows_view(addend, "addend")[2] != ldy:
+            raise ValueError("addend must be [M, N] in the dtype of X, with the row stride of Y")
     need = convrot_linear_workspace_bytes(M, N, K, g)
     if ws is None:
         ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=X.device)
-    _check(lib().convrot_linear_ex(_ptr(X), dtype, M, K, g, _ptr(Wq), _ptr(w_scale), mode, N, _ptr(bias),
-                                   int(activation), _ptr(Y), _ptr(ws), ws.numel(), _stream_ptr(stream)),
-           "convrot_linear_ex")
+    _check(lib().convrot_linear_ex(_ptr(X), dtype, M, K, ldx, g, _ptr(Wq), _ptr(w_scale), mode, N, _ptr(bias),
+                                   _ptr(addend), int(activation), _ptr(Y), ldy, _ptr(ws), ws.numel(),
+                                   _stream_ptr(stream)), "convrot_linear_ex")
     return Y
 
 

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
 // The one-launch form (rotate+quantise worker warps inside the GEMM kernel) is
 // correct but, measured on the DiT QKV layer, its workers fall behind the
@@ -82,7 +82,12 @@ struct EpiOptions {
   int out_f16 = 0;
   int wscale_per_channel = 0;
   int act = 0;
-  bool general() const { return out_f16 != 0 || wscale_per_channel != 0 || act != 0; }
+  const void* addend = nullptr;  // [M, ldy] in the output dtype, added before the activation
+  int64_t ldx = 0;               // row strides in elements (0 = dense)
+  int64_t ldy = 0;
+  bool general() const {
+    return out_f16 != 0 || wscale_per_channel != 0 || act != 0 || addend != nullptr || ldy != 0;
+  }
 };
 
 convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, int64_t M, int64_t N, int64_t K,
@@ -91,6 +96,8 @@ convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, 
   convrot::GemmParams p{};
   p.out_f16 = opt.out_f16;
   p.wscale_per_channel = opt.wscale_per_channel;
+  p.addend = static_cast<const uint16_t*>(opt.addend);
+  p.ldy = opt.ldy;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -166,18 +173,20 @@ convrot_status convrot_prepare_weight(const void* W, int64_t N, int64_t K, int g
                                    stream);
 }
 
-convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t K, int g, int8_t* Xq,
-                                    float* x_scale, convrot_stream_t stream) {
+convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t K, int64_t ldx, int g,
+                                    int8_t* Xq, float* x_scale, convrot_stream_t stream) {
   const convrot_status sh = check_rotation_shape(M, K, g);
   if (sh != CONVROT_OK) return sh;
   if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
   if (X == nullptr || Xq == nullptr || x_scale == nullptr) return CONVROT_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(x_scale, 4)) return CONVROT_ERR_INVALID_ARG;
+  if (ldx != 0 && (ldx < K || ldx % 8 != 0)) return CONVROT_ERR_INVALID_ARG;
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(X);
   p.in_f16 = dtype == CONVROT_DTYPE_F16 ? 1 : 0;
   p.rows = M;
   p.K = K;
+  p.ldx = ldx;
   p.dst = Xq;
   p.scale = x_scale;
   p.tensor_absmax = nullptr;
@@ -190,7 +199,7 @@ convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t
 
 convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int8_t* Xq, float* x_scale,
                                  convrot_stream_t stream) {
-  return convrot_quant_act_ex(X, CONVROT_DTYPE_BF16, M, K, g, Xq, x_scale, stream);
+  return convrot_quant_act_ex(X, CONVROT_DTYPE_BF16, M, K, 0, g, Xq, x_scale, stream);
 }
 
 size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
@@ -214,7 +223,10 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   if (sh != CONVROT_OK) return sh;
   if (X == nullptr || Wq == nullptr || w_scale == nullptr || Y == nullptr) return CONVROT_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(w_scale, opt.wscale_per_channel ? 16 : 4) ||
-      !aligned(Y, 16) || (bias != nullptr && !aligned(bias, 16)))
+      !aligned(Y, 16) || (bias != nullptr && !aligned(bias, 16)) ||
+      (opt.addend != nullptr && !aligned(opt.addend, 16)))
+    return CONVROT_ERR_INVALID_ARG;
+  if ((opt.ldx != 0 && (opt.ldx < K || opt.ldx % 8 != 0)) || (opt.ldy != 0 && (opt.ldy < N || opt.ldy % 8 != 0)))
     return CONVROT_ERR_INVALID_ARG;
   const LinearWs lay = linear_ws_layout(M, K);
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE;
@@ -224,7 +236,7 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
 
   int tpr = 0, rpp = 0, cta_threads = 0;
-  if (kFusedLinear && !opt.general() && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) {
+  if (kFusedLinear && !opt.general() && opt.ldx == 0 && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) {
     // one launch: worker warps rotate + quantise while the GEMM consumes finished M-blocks
     convrot::GemmParams gp{};
     gp.M = static_cast<int>(M);
@@ -253,6 +265,7 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   p.in_f16 = opt.out_f16;  // X, bias and Y share the compute dtype
   p.rows = M;
   p.K = K;
+  p.ldx = opt.ldx;
   p.dst = Xq;
   p.scale = x_scale;
   p.tensor_absmax = nullptr;
@@ -291,9 +304,10 @@ convrot_status convrot_linear_timed(const void* X, int64_t M, int64_t K, int g, 
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
-convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K, int g, const int8_t* Wq,
-                                 const float* w_scale, int wscale_mode, int64_t N, const void* bias, int activation,
-                                 void* Y, void* ws, size_t ws_bytes, convrot_stream_t stream) {
+convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K, int64_t ldx, int g,
+                                 const int8_t* Wq, const float* w_scale, int wscale_mode, int64_t N,
+                                 const void* bias, const void* addend, int activation, void* Y, int64_t ldy,
+                                 void* ws, size_t ws_bytes, convrot_stream_t stream) {
   if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
   if (wscale_mode != CONVROT_WSCALE_TENSOR && wscale_mode != CONVROT_WSCALE_CHANNEL) return CONVROT_ERR_UNSUPPORTED;
   if (activation != CONVROT_ACT_NONE && activation != CONVROT_ACT_GELU_ERF) return CONVROT_ERR_UNSUPPORTED;
@@ -301,6 +315,9 @@ convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K,
   opt.out_f16 = dtype == CONVROT_DTYPE_F16 ? 1 : 0;
   opt.wscale_per_channel = wscale_mode == CONVROT_WSCALE_CHANNEL ? 1 : 0;
   opt.act = activation == CONVROT_ACT_GELU_ERF ? 1 : 0;
+  opt.addend = addend;
+  opt.ldx = (ldx == K) ? 0 : ldx;
+  opt.ldy = (ldy == N) ? 0 : ldy;
   return linear_impl(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, nullptr, nullptr, nullptr,
                      reinterpret_cast<cudaStream_t>(stream), opt);
 }

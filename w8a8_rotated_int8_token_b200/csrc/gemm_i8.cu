@@ -214,8 +214,8 @@ __device__ __forceinline__ float gelu_erf(float y) {
 // sc is x_scale[row] times the tensor weight scale, or x_scale[row] alone when
 // the weight scale is per channel (then wv holds w_scale[n]).
 template <bool GELU>
-__device__ __forceinline__ void dequant_gen32(const GemmParams& p, int n0, float sc, const uint32_t (&r)[32],
-                                              uint32_t (&packed)[16]) {
+__device__ __forceinline__ void dequant_gen32(const GemmParams& p, int row, int n0, float sc,
+                                              const uint32_t (&r)[32], uint32_t (&packed)[16]) {
   const bool f16 = p.out_f16 != 0;
   float bv[32], wv[32];
 #pragma unroll
@@ -242,6 +242,21 @@ __device__ __forceinline__ void dequant_gen32(const GemmParams& p, int n0, float
   } else {
 #pragma unroll
     for (int e = 0; e < 32; ++e) wv[e] = 1.0f;
+  }
+  if (p.addend != nullptr && row < p.M) {  // this row's 32 addend values join the bias
+    const int64_t ld = p.ldy ? p.ldy : p.N;
+    const uint16_t* a = p.addend + static_cast<int64_t>(row) * ld + n0;
+#pragma unroll
+    for (int pc = 0; pc < 4; ++pc) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (n0 + 8 * pc < p.N) w = __ldg(reinterpret_cast<const uint4*>(a + 8 * pc));
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bv[8 * pc + 2 * e] += out16_to_f32(ws[e] & 0xFFFFu, f16);
+        bv[8 * pc + 2 * e + 1] += out16_to_f32(ws[e] >> 16, f16);
+      }
+    }
   }
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
@@ -295,7 +310,7 @@ __device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmOut, const Ge
     __syncwarp();
     if (epi_is_general(EPI)) {
       uint32_t packed[16];
-      dequant_gen32<EPI == kEpiDequantGenGelu>(p, n0, sc, r, packed);
+      dequant_gen32<EPI == kEpiDequantGenGelu>(p, row0 + lane, n0, sc, r, packed);
       uint8_t* rowp = ebuf + lane * 64;  // same 64-byte-swizzled staging as below
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -1138,12 +1153,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const __nv_bfloat16 h = __float2bfloat16_rn(y);
             static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = h;
           } else if (epi_is_general(EPI)) {
-            float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * swn, bn);
+            const int64_t at = static_cast<int64_t>(m) * (p.ldy ? p.ldy : p.N) + n;
+            float bias_add = bn;
+            if (p.addend != nullptr) bias_add += out16_to_f32(__ldg(p.addend + at), p.out_f16 != 0);
+            float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * swn, bias_add);
             if (EPI == kEpiDequantGenGelu) y = gelu_erf(y);
             if (p.out_f16)
-              static_cast<__half*>(out)[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(y);
+              static_cast<__half*>(out)[at] = __float2half_rn(y);
             else
-              static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(y);
+              static_cast<__nv_bfloat16*>(out)[at] = __float2bfloat16_rn(y);
           } else {
             static_cast<int32_t*>(out)[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[j]);
           }
@@ -1177,12 +1195,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// A 2-D tiled tensor map; row_elems = distance between rows in elements (0 = inner).
 bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
-               uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+               uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz,
+               uint64_t row_elems = 0) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+  const cuuint64_t strides[1] = {(row_elems ? row_elems : inner) * static_cast<uint64_t>(elem_bytes)};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return enc(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -1228,7 +1248,7 @@ cudaError_t launch_impl(const int8_t* A, const int8_t* B, void* out, GemmParams 
   if (epi_is_dequant(EPI))
     ok_out = encode_2d(&to, (epi_is_general(EPI) && p.out_f16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                       2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+                       2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B, static_cast<uint64_t>(p.ldy));
   else
     ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok_out) return cudaErrorInvalidValue;
@@ -1291,7 +1311,7 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
   if (epi_is_dequant(EPI))
     ok_out = encode_2d(&to, (epi_is_general(EPI) && p.out_f16) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                       2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+                       2, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B, static_cast<uint64_t>(p.ldy));
   else
     ok_out = encode_2d(&to, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, out, p.N, p.M, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok_out) return cudaErrorInvalidValue;

@@ -27,6 +27,8 @@ struct GemmParams {
   const uint16_t* bias;   // [N] bf16 (fp16 with out_f16) bits or null
   int wscale_per_channel; // kEpiDequantGen(Gelu): w_scale holds N floats (one per output channel)
   int out_f16;            // kEpiDequantGen(Gelu): Y and bias are IEEE fp16 instead of bf16
+  const uint16_t* addend; // kEpiDequantGen(Gelu): [M, ldy] term added before the activation, or null
+  int64_t ldy;            // row stride of Y (and addend) in elements (>= N); 0 = N
   int* status;            // status word: a timed-out wait ORs 5 into it
   uint64_t timeout_ns;    // bound of every device-side wait
   int group_m;            // M-blocks per raster group (0 = default)

@@ -105,10 +105,17 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
     if (blk >= nblocks) return;
     const int64_t r0 = blk * rpc;
     const int64_t nrows = (p.rows - r0) < rpc ? (p.rows - r0) : rpc;
-    const uint32_t bytes = static_cast<uint32_t>(nrows) * static_cast<uint32_t>(p.K) * 2u;
+    const uint32_t row_bytes = static_cast<uint32_t>(p.K) * 2u;
+    const uint32_t bytes = static_cast<uint32_t>(nrows) * row_bytes;
     const int slot = static_cast<int>(it % kRqStages);
+    uint8_t* const dst = stage_mem + static_cast<size_t>(slot) * stage_bytes;
     mbar_arrive_expect_tx(&full[slot], bytes);
-    bulk_load(stage_mem + static_cast<size_t>(slot) * stage_bytes, p.src + r0 * p.K, bytes, &full[slot]);
+    if (p.ldx == 0 || p.ldx == p.K) {  // dense rows: one copy for the block
+      bulk_load(dst, p.src + r0 * p.K, bytes, &full[slot]);
+    } else {  // strided rows: one copy per row, packed densely in the slot
+      for (int64_t r = 0; r < nrows; ++r)
+        bulk_load(dst + r * row_bytes, p.src + (r0 + r) * p.ldx, row_bytes, &full[slot]);
+    }
     issued = it + 1;
   };
   static_assert(kRqStages >= 2, "the block after the current one needs its own slot");

@@ -23,6 +23,7 @@ struct RotQuantParams {
   int in_f16;               // 0: bf16 input, 1: fp16 input
   int64_t rows;
   int64_t K;
+  int64_t ldx;              // row stride of src in elements (>= K, a multiple of 8); 0 = K
   int8_t* dst;              // [rows, K] codes (unused in kRqWeightAbsmax)
   float* scale;             // [rows] (activation) or [1] (weight)
   unsigned* tensor_absmax;  // weight modes: float bits of the unnormalised absmax
