@@ -39,11 +39,12 @@ INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B2
 # DRAM bytes per launch of the dominant kernel (the pair GEMM) on a workload,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum). A
 # figure holds only for the kernel source it was taken on: the sha256 over
-# GEMM_SOURCES must match, otherwise the bench reports null.
-GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh", "fwht_dev.cuh"]
+# GEMM_SOURCES (the files the pair kernel is compiled from) must match,
+# otherwise the bench reports null.
+GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh"]
 GEMM_TRAFFIC = {
-    "dit_qkv_1024": {"bytes": 60029696 + 49044224,
-                     "sources_sha256": "93c2b5d64aa264a58d36511b1cfe83357739fedb0b849c8efb702d162d86e95f"},
+    "dit_qkv_1024": {"bytes": 60552192 + 48752640,
+                     "sources_sha256": "db12ebca48b98470125439c244b8752a705b51805c9ee1deac0ac4520bf7ccfc"},
 }
 
 

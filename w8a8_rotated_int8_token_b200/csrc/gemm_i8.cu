@@ -8,7 +8,11 @@
 // epilogue applies the token and tensor scales and the bias and rounds to
 // bf16 (or, for exactness tests, stores the raw int32 accumulators).
 //
-// Structure: a persistent kernel, one CTA per SM.
+// Three forms share the roles below: the CTA-pair kernel (256x256 tiles on two
+// SMs, the layer's GEMM for M > 64), the weight-streaming kernel (M <= 64) and
+// the single-SM kernel described here (also the one-launch fused form).
+//
+// Structure of the single-SM form: a persistent kernel, one CTA per SM.
 //   warp 0, one lane : TMA producer. 128x128 (A) and 256x128 (B) int8 tiles,
 //                      128-byte swizzle, into a 4-stage shared-memory ring.
 //   warp 1           : allocates 512 TMEM columns; one lane issues
@@ -684,7 +688,8 @@ __global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
 // accumulator completion to both CTAs; the follower's epilogue warps release
 // the accumulator by arriving on the leader's barrier. Each CTA holds its 128
 // rows x 256 columns of the accumulator (two buffers, 512 columns), and runs
-// the same epilogue as the single-SM form on them. No TMA multicast is used.
+// the same epilogue routine as the single-SM form on them, split over eight
+// warps of 128 columns each. No TMA multicast is used.
 
 constexpr int BN_HALF = BN / 2;
 // Eight epilogue warps per CTA: two per TMEM lane quarter, each draining 128
