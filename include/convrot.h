@@ -134,6 +134,23 @@ CONVROT_API convrot_status convrot_linear(const void* X, int64_t M, int64_t K, i
                               void* ws, size_t ws_bytes, convrot_stream_t stream);
 
 /*
+ * convrot_linear_one_launch -- the same layer as convrot_linear in ONE kernel
+ * launch: worker warps of the GEMM kernel rotate and quantise the tokens
+ * block by block and release each 128-token block to the tensor cores through
+ * a per-call tagged counter in the workspace, while the tensor cores already
+ * multiply the finished blocks (single-SM 128x256 tiles). For callers for whom
+ * a launch costs more than the slower schedule: on the DiT QKV layer it
+ * measured slower than the two-kernel convrot_linear (137 against 110 us).
+ * Same arguments, workspace and errors as convrot_linear, plus
+ * CONVROT_ERR_UNSUPPORTED when K > 20480 (the worker warps of one CTA hold a
+ * token) or K % 128 != 0.
+ */
+CONVROT_API convrot_status convrot_linear_one_launch(const void* X, int64_t M, int64_t K, int g,
+                                                     const int8_t* Wq, const float* w_scale, int64_t N,
+                                                     const void* bias, void* Y, void* ws, size_t ws_bytes,
+                                                     convrot_stream_t stream);
+
+/*
  * Variants of the layer: compute dtype, weight-scale granularity, activation.
  *   CONVROT_DTYPE_F16: X, W, bias and Y are IEEE fp16 instead of bf16 (the
  *     pages' kernels run in BF16 and FP16 only: InvokeAI "int8 Compute",
@@ -199,9 +216,8 @@ CONVROT_API convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M
 /*
  * convrot_linear_timed -- convrot_linear that also records caller-created CUDA
  * events (cudaEvent_t, passed as void*) on `stream`: ev_start before its first
- * launch, ev_mid after the rotate+quantise kernel (may be NULL; with the
- * one-launch form it is recorded together with ev_end), ev_end after the
- * GEMM. The layer's and each kernel's device time can then be read with
+ * launch, ev_mid after the rotate+quantise kernel (may be NULL), ev_end
+ * after the GEMM. The layer's and each kernel's device time can then be read with
  * cudaEventElapsedTime on the launching stream. ev_mid keeps the GEMM from
  * overlapping the first kernel's tail.
  */

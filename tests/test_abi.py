@@ -62,7 +62,7 @@ def linear_ws_layout(M, K):
 
 
 def test_status_strings_and_version(L):
-    assert L.convrot_abi_version() == 4
+    assert L.convrot_abi_version() == 5
     for code in range(6):
         s = L.convrot_status_string(code)
         assert s and s != b"unknown status"
@@ -124,7 +124,10 @@ def test_other_entry_points_reject_bad_arguments_on_host(L):
     # the timed variant needs both events
     assert L.convrot_linear_timed(FAKE, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30, None, None,
                                   FAKE, None) == 1
-    assert L.convrot_linear_launch_count(4608, 9216, 3072, 256) in (1, 2)
+    assert L.convrot_linear_launch_count(4608, 9216, 3072, 256) == 2
+    # the one-launch form: K beyond what one CTA's worker warps hold
+    assert L.convrot_linear_one_launch(FAKE, 64, 20608, 128, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 40, None) == 2
+    assert L.convrot_linear_one_launch(FAKE, 64, 256, 256, FAKE, FAKE, 256, None, None, FAKE, 1 << 30, None) == 1
     assert L.convrot_linear_launch_count(4608, 9216, 3000, 256) == 0
 
 

@@ -200,7 +200,7 @@ def test_gemm_dequant_on_identical_codes(cr):
 # ------------------------------------------------------------ end to end
 
 
-def _linear_case(cr, d, rows=None):
+def _linear_case(cr, d, rows=None, one_launch=False):
     import torch
 
     w = d["workload"]
@@ -212,7 +212,8 @@ def _linear_case(cr, d, rows=None):
     M, K = d["x"].shape
     N = d["w"].shape[0]
     ws = torch.empty(cr.convrot_linear_workspace_bytes(M, N, K, g), dtype=torch.uint8, device="cuda")
-    Y = cr.convrot_linear(X, Wq, sw, g, bias, ws=ws)
+    layer = cr.convrot_linear_one_launch if one_launch else cr.convrot_linear
+    Y = layer(X, Wq, sw, g, bias, ws=ws)
     status = cr.convrot_read_device_status(ws)
     assert status == 0
     if rows is None:
@@ -281,22 +282,48 @@ def test_zero_input_gives_zero_output_and_bias(cr):
     assert torch.equal(Yb.view(torch.int16), b.view(torch.int16).expand(130, -1))
 
 
-@pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256),   # largest K of the one-launch form
-                                     (129, 136, 20608, 128),   # two kernels (K above the fused limit)
-                                     (67, 264, 32768, 256),    # two kernels, largest K
-                                     (1, 16, 384, 128), (385, 520, 1024, 256)])
-def test_linear_fused_and_two_kernel_forms(cr, M, N, K, g):
+def _random_layer(M, N, K, g):
     rng = np.random.default_rng(M + N + K)
     x = rng.standard_normal((M, K)).astype(np.float32)
     x[:, rng.choice(K, max(1, K // 100), replace=False)] *= 50.0
-    d = {"workload": type("W", (), {"name": f"{M}x{K}x{N}", "g": g})(),
-         "x": synth.f32_to_bf16_bits(x),
-         "w": synth.f32_to_bf16_bits((rng.standard_normal((N, K)) * 0.02).astype(np.float32)),
-         "bias": synth.f32_to_bf16_bits((rng.standard_normal(N) * 0.01).astype(np.float32))}
-    _linear_case(cr, d)
+    return {"workload": type("W", (), {"name": f"{M}x{K}x{N}", "g": g})(),
+            "x": synth.f32_to_bf16_bits(x),
+            "w": synth.f32_to_bf16_bits((rng.standard_normal((N, K)) * 0.02).astype(np.float32)),
+            "bias": synth.f32_to_bf16_bits((rng.standard_normal(N) * 0.01).astype(np.float32))}
 
 
-def test_linear_back_to_back_calls_on_one_workspace(cr):
+@pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256), (129, 136, 20608, 128),
+                                     (67, 264, 32768, 256),    # largest K
+                                     (1, 16, 384, 128), (385, 520, 1024, 256)])
+def test_linear_ragged_and_large_k(cr, M, N, K, g):
+    _linear_case(cr, _random_layer(M, N, K, g))
+
+
+@pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256),   # largest K of the one-launch form
+                                     (1, 16, 384, 128), (385, 520, 1024, 256), (64, 256, 256, 256)])
+def test_linear_one_launch_matches_oracle(cr, M, N, K, g):
+    _linear_case(cr, _random_layer(M, N, K, g), one_launch=True)
+
+
+def test_linear_one_launch_on_the_bench_layer(cr):
+    d = synth.make_workload("dit_qkv_1024")
+    _linear_case(cr, d, rows=_rows_sample(d["x"].shape[0]), one_launch=True)
+
+
+def test_linear_one_launch_rejects_k_beyond_its_workers(cr):
+    import torch
+
+    M, N, K = 64, 256, 20608
+    X = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    Wq = torch.zeros((N, K), dtype=torch.int8, device="cuda")
+    sw = torch.ones((1,), dtype=torch.float32, device="cuda")
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.convrot_linear_one_launch(X, Wq, sw, 128)
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("one_launch", [False, True])
+def test_linear_back_to_back_calls_on_one_workspace(cr, one_launch):
     """Consecutive calls reuse the workspace: later calls must not see earlier readiness counters."""
     import torch
 
@@ -310,11 +337,15 @@ def test_linear_back_to_back_calls_on_one_workspace(cr):
     ref_a = cr.convrot_linear(Xa, Wa, sa, 256, to_torch_bf16(a["bias"]))
     ref_b = cr.convrot_linear(Xb, Wb, sb, 256)
     outs = []
+    layer = cr.convrot_linear_one_launch if one_launch else cr.convrot_linear
+    if one_launch:  # the same form on both sides of the comparison
+        ref_a = layer(Xa, Wa, sa, 256, to_torch_bf16(a["bias"]))
+        ref_b = layer(Xb, Wb, sb, 256)
     for i in range(6):  # alternate layers on the same workspace, no synchronisation in between
         if i % 2 == 0:
-            outs.append(("a", cr.convrot_linear(Xa, Wa, sa, 256, to_torch_bf16(a["bias"]), ws=ws)))
+            outs.append(("a", layer(Xa, Wa, sa, 256, to_torch_bf16(a["bias"]), ws=ws)))
         else:
-            outs.append(("b", cr.convrot_linear(Xb, Wb, sb, 256, ws=ws)))
+            outs.append(("b", layer(Xb, Wb, sb, 256, ws=ws)))
     torch.cuda.synchronize()
     assert cr.convrot_read_device_status(ws) == 0
     for tag, y in outs:

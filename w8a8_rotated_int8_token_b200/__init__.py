@@ -23,6 +23,7 @@ __all__ = [
     "convrot_quant_act",
     "convrot_linear_workspace_bytes",
     "convrot_linear",
+    "convrot_linear_one_launch",
     "convrot_prepare_weight_ex",
     "convrot_quant_act_ex",
     "convrot_linear_ex",
@@ -162,6 +163,30 @@ def convrot_linear(X, Wq, w_scale, g: int = 256, bias=None, Y=None, ws=None, str
         ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=X.device)
     _check(lib().convrot_linear(_ptr(X), M, K, g, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y), _ptr(ws),
                                 ws.numel(), _stream_ptr(stream)), "convrot_linear")
+    return Y
+
+
+def convrot_linear_one_launch(X, Wq, w_scale, g: int = 256, bias=None, Y=None, ws=None, stream=None):
+    """convrot_linear as one kernel launch (rotate+quantise workers inside the GEMM kernel; K <= 20480)."""
+    import torch
+
+    _require(X, torch.bfloat16, None, "X")
+    M, K = X.shape
+    _require(Wq, torch.int8, None, "Wq")
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("Wq must be [N, K] with the K of X")
+    _require(w_scale, torch.float32, (1,), "w_scale")
+    if bias is not None:
+        _require(bias, torch.bfloat16, (N,), "bias")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _require(Y, torch.bfloat16, (M, N), "Y")
+    need = convrot_linear_workspace_bytes(M, N, K, g)
+    if ws is None:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=X.device)
+    _check(lib().convrot_linear_one_launch(_ptr(X), M, K, g, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
+                                           _ptr(ws), ws.numel(), _stream_ptr(stream)), "convrot_linear_one_launch")
     return Y
 
 

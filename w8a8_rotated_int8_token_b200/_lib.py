@@ -30,6 +30,8 @@ SIGNATURES = {
     "convrot_linear_timed": (_int, [_c_void_p, _i64, _i64, _int, _c_void_p, _c_void_p, _i64, _c_void_p,
                                     _c_void_p, _c_void_p, _size, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "convrot_linear_launch_count": (_int, [_i64, _i64, _i64, _int]),
+    "convrot_linear_one_launch": (_int, [_c_void_p, _i64, _i64, _int, _c_void_p, _c_void_p, _i64, _c_void_p,
+                                         _c_void_p, _c_void_p, _size, _c_void_p]),
     "convrot_prepare_weight_ex": (_int, [_c_void_p, _int, _i64, _i64, _int, _int, _c_void_p, _c_void_p, _c_void_p,
                                          _size, _c_void_p]),
     "convrot_quant_act_ex": (_int, [_c_void_p, _int, _i64, _i64, _i64, _int, _c_void_p, _c_void_p, _c_void_p]),

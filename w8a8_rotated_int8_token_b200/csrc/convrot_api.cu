@@ -14,13 +14,13 @@
 
 namespace {
 
-constexpr int kAbiVersion = 4;
+constexpr int kAbiVersion = 5;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
-// The one-launch form (rotate+quantise worker warps inside the GEMM kernel) is
-// correct but, measured on the DiT QKV layer, its workers fall behind the
-// tensor cores (137 us vs 94 + 16 us for the two kernels), so the layer runs
-// as two kernels chained with programmatic dependent launch.
-constexpr bool kFusedLinear = false;
+// convrot_linear runs two kernels chained with programmatic dependent launch.
+// The one-launch form (rotate+quantise worker warps inside the GEMM kernel,
+// convrot_linear_one_launch) is correct but, measured on the DiT QKV layer,
+// its workers fall behind the tensor cores (137 us against 94 + 16 us for the
+// two kernels at the time), so it is offered only as its own entry point.
 
 // Workspace of convrot_linear:
 // [status word | 256 B][M-block ready counters, 8 B each][token scales][int8 codes].
@@ -211,12 +211,14 @@ size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
 
 namespace {
 
-// convrot_linear: one fused launch when the worker layout fits (K <= 20480),
-// else the rotate+quantise kernel followed by the GEMM. Events (may be null)
-// are recorded before and after the launches.
+// The layer: the rotate+quantise kernel followed by the GEMM, or (one_launch)
+// the single kernel whose worker warps rotate and quantise while its tensor
+// cores multiply the finished M-blocks (K <= 20480, default options only).
+// Events (may be null) are recorded before, between and after the launches.
 convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq, const float* w_scale,
                            int64_t N, const void* bias, void* Y, void* ws, size_t ws_bytes, cudaEvent_t ev0,
-                           cudaEvent_t ev1, cudaEvent_t ev2, cudaStream_t s, EpiOptions opt = EpiOptions()) {
+                           cudaEvent_t ev1, cudaEvent_t ev2, cudaStream_t s, EpiOptions opt = EpiOptions(),
+                           bool one_launch = false) {
   convrot_status sh = check_rotation_shape(M, K, g);
   if (sh != CONVROT_OK) return sh;
   sh = check_gemm_shape(M, N, K, 8);
@@ -235,8 +237,10 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   float* x_scale = reinterpret_cast<float*>(wsb + lay.scale_off);
   int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
 
-  int tpr = 0, rpp = 0, cta_threads = 0;
-  if (kFusedLinear && !opt.general() && opt.ldx == 0 && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) {
+  if (one_launch) {
+    int tpr = 0, rpp = 0, cta_threads = 0;
+    if (opt.general() || opt.ldx != 0 || !convrot::fused_shape(K, &tpr, &rpp, &cta_threads))
+      return CONVROT_ERR_UNSUPPORTED;
     // one launch: worker warps rotate + quantise while the GEMM consumes finished M-blocks
     convrot::GemmParams gp{};
     gp.M = static_cast<int>(M);
@@ -324,8 +328,14 @@ convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K,
 
 int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g) {
   if (check_rotation_shape(M, K, g) != CONVROT_OK || check_gemm_shape(M, N, K, 8) != CONVROT_OK) return 0;
-  int tpr = 0, rpp = 0, cta_threads = 0;
-  return (kFusedLinear && convrot::fused_shape(K, &tpr, &rpp, &cta_threads)) ? 1 : 2;
+  return 2;
+}
+
+convrot_status convrot_linear_one_launch(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq,
+                                         const float* w_scale, int64_t N, const void* bias, void* Y, void* ws,
+                                         size_t ws_bytes, convrot_stream_t stream) {
+  return linear_impl(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, nullptr, nullptr, nullptr,
+                     reinterpret_cast<cudaStream_t>(stream), EpiOptions(), true);
 }
 
 size_t convrot_gemm_workspace_bytes(void) { return kStatusBytes; }

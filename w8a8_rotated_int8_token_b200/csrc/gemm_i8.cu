@@ -10,7 +10,8 @@
 //
 // Three forms share the roles below: the CTA-pair kernel (256x256 tiles on two
 // SMs, the layer's GEMM for M > 64), the weight-streaming kernel (M <= 64) and
-// the single-SM kernel described here (also the one-launch fused form).
+// the single-SM kernel described here, which carries the rotate+quantise
+// workers of the one-launch form of the layer.
 //
 // Structure of the single-SM form: a persistent kernel, one CTA per SM.
 //   warp 0, one lane : TMA producer. 128x128 (A) and 256x128 (B) int8 tiles,
@@ -1389,24 +1390,17 @@ cudaError_t launch_smallm(const int8_t* A, const int8_t* B, void* out, GemmParam
 
 cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out, GemmParams p,
                            cudaStream_t stream) {
-  if (p.M <= kSmallM && p.single_sm == 0) {
+  if (p.M <= kSmallM) {
     if (epi == kEpiDequantBf16) return launch_smallm<kEpiDequantBf16>(A, B, out, p, stream);
     if (epi == kEpiDequantGen) return launch_smallm<kEpiDequantGen>(A, B, out, p, stream);
     if (epi == kEpiDequantGenGelu) return launch_smallm<kEpiDequantGenGelu>(A, B, out, p, stream);
     if (epi == kEpiRawS32) return launch_smallm<kEpiRawS32>(A, B, out, p, stream);
     return cudaErrorInvalidValue;
   }
-  if (p.single_sm == 0) {
-    if (epi == kEpiDequantBf16) return launch_pair<kEpiDequantBf16>(A, B, out, p, stream);
-    if (epi == kEpiDequantGen) return launch_pair<kEpiDequantGen>(A, B, out, p, stream);
-    if (epi == kEpiDequantGenGelu) return launch_pair<kEpiDequantGenGelu>(A, B, out, p, stream);
-    if (epi == kEpiRawS32) return launch_pair<kEpiRawS32>(A, B, out, p, stream);
-    return cudaErrorInvalidValue;
-  }
-  if (epi == kEpiDequantBf16) return launch_impl<kEpiDequantBf16, 0>(A, B, out, p, stream);
-  if (epi == kEpiDequantGen) return launch_impl<kEpiDequantGen, 0>(A, B, out, p, stream);
-  if (epi == kEpiDequantGenGelu) return launch_impl<kEpiDequantGenGelu, 0>(A, B, out, p, stream);
-  if (epi == kEpiRawS32) return launch_impl<kEpiRawS32, 0>(A, B, out, p, stream);
+  if (epi == kEpiDequantBf16) return launch_pair<kEpiDequantBf16>(A, B, out, p, stream);
+  if (epi == kEpiDequantGen) return launch_pair<kEpiDequantGen>(A, B, out, p, stream);
+  if (epi == kEpiDequantGenGelu) return launch_pair<kEpiDequantGenGelu>(A, B, out, p, stream);
+  if (epi == kEpiRawS32) return launch_pair<kEpiRawS32>(A, B, out, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -32,7 +32,6 @@ struct GemmParams {
   int* status;            // status word: a timed-out wait ORs 5 into it
   uint64_t timeout_ns;    // bound of every device-side wait
   int group_m;            // M-blocks per raster group (0 = default)
-  int single_sm;          // 1: one-CTA tiles (128x256); 0: CTA-pair tiles (256x256, cta_group::2)
   int num_m_blocks, num_n_blocks, num_k_blocks;  // filled by the launcher
   // fused form (launch_linear_fused): the kernel also rotates and quantises X
   const uint16_t* X;              // [M,K] bf16 bits
