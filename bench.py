@@ -43,8 +43,8 @@ INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B2
 # otherwise the bench reports null.
 GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh"]
 GEMM_TRAFFIC = {
-    "dit_qkv_1024": {"bytes": 60552192 + 48752640,
-                     "sources_sha256": "db12ebca48b98470125439c244b8752a705b51805c9ee1deac0ac4520bf7ccfc"},
+    "dit_qkv_1024": {"bytes": 59904768 + 48083456,
+                     "sources_sha256": "a070901777178b94bffd44bd6441f83d97c2752a4107e86a9b74e32cf4b4c482"},
 }
 
 
