@@ -56,7 +56,7 @@ def check_codes(q_gpu: np.ndarray, s_gpu: np.ndarray, x_rot: np.ndarray, q_ref: 
         quot = x_rot[bad] / s_b
         tie_dist = np.abs(np.abs(quot - np.floor(quot)) - 0.5)
         assert tie_dist.max() <= CODE_TIE_WINDOW, f"a differing code is not at a near-tie ({tie_dist.max()})"
-    assert q_gpu.min(initial=0) >= -127 and q_gpu.max(initial=0) <= 127
+    assert q_gpu.min(initial=0) >= -127 and q_gpu.max(initial=0) <= 127, "a code outside the range [-127, 127]"
     return {"mismatch_frac": frac, "scale_rel_max": float(rel.max(initial=0.0))}
 
 
