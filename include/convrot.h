@@ -23,7 +23,8 @@
  *
  * Conventions for every entry point:
  *   - Matrices are row-major with K contiguous: X [M,K], W/Wq [N,K], Y [M,N].
- *     X, W, bias and Y are bf16 (IEEE bfloat16 bit patterns, 2 bytes each).
+ *     X, W, bias and Y are bf16 (IEEE bfloat16 bit patterns, 2 bytes each),
+ *     except in the *_ex entry points, which also take fp16 and row strides.
  *   - Every data pointer is a DEVICE pointer owned by the caller, 16-byte
  *     aligned (workspaces: 256-byte aligned). The library never allocates,
  *     never frees and never synchronises, except where an entry point says so.
@@ -32,11 +33,13 @@
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns an error code and enqueues nothing.
  *   - A launch failure returns CONVROT_ERR_CUDA.
- *   - Waits inside the GEMM kernel are bounded (about 2 s). If one runs out,
- *     the kernel records CONVROT_ERR_DEVICE_TIMEOUT in the workspace status
- *     word and returns without faulting; convrot_read_device_status reports it.
- *   - Entry points hold no state between calls and are safe to call from
- *     several host threads on different streams with separate workspaces.
+ *   - Every wait inside a kernel is bounded (about 2 s). If one runs out, the
+ *     kernel records CONVROT_ERR_DEVICE_TIMEOUT in the workspace status word
+ *     (where the entry point has one) and returns without faulting;
+ *     convrot_read_device_status reports it.
+ *   - Entry points hold no state between calls (convrot_linear_noalloc's
+ *     built-in scratch aside) and are safe to call from several host threads
+ *     on different streams with separate workspaces.
  */
 #ifndef CONVROT_H
 #define CONVROT_H
