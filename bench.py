@@ -35,6 +35,7 @@ UNIT = "TOPS"
 N_SETS = 4  # rotating input/output sets per rank so that no step finds its data in L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200
+SMALL_M = 64  # up to this many tokens the layer's GEMM is the weight-streaming form
 
 # DRAM bytes per launch of the dominant kernel (the pair GEMM) on a workload,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum). A
@@ -481,7 +482,7 @@ def main():
     if rank != 0:
         return 0
     # the dominant kernel: the GEMM (second launch), or the whole layer in the one-launch form
-    t_dom = t_second if launches == 2 else t_layer
+    t_dom = t_second
     dom_tops = ops / (t_dom * 1e-3) / 1e12
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -489,10 +490,9 @@ def main():
         "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(w),
         "pct_int8_peak": 100.0 * value / world / int8_peak,
         "roofline": {"bound": "tensor",
-                     "kernel": ("gemm_i8_pair_kernel (tcgen05.mma.cta_group::2 kind::i8, dequant/bias epilogue)"
-                                if launches == 2 else "gemm_i8_kernel with fused rotate+quantise workers"),
+                     "kernel": "gemm_i8_pair_kernel (tcgen05.mma.cta_group::2 kind::i8, dequant/bias epilogue)",
                      "achieved": dom_tops, "peak": int8_peak, "unit": "TOPS", "frac": dom_tops / int8_peak,
-                     "traffic": gemm_traffic(args.config) if launches == 2 and not variant else None,
+                     "traffic": gemm_traffic(args.config) if not variant else None,
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "us_per_launch": t_dom * 1e3,
                      "us_source": ("layer time minus the standalone rotate+quantise kernel" if variant
@@ -513,6 +513,16 @@ def main():
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
     }
+    if M <= SMALL_M:
+        # the weight-streaming GEMM (tokens as the MMA's N side): bound by HBM on the
+        # weight bytes; algorithmic bytes M*K + N*K + 2*M*N (+ 2*N bias) per launch
+        gbytes = float(M * K + N * K + 2 * M * N + (2 * N if bias is not None else 0))
+        gbs = gbytes / (t_dom * 1e-3) / 1e9
+        out["roofline"].update({
+            "bound": "hbm", "kernel": "gemm_i8_smallm_kernel (swap-AB tcgen05 kind::i8, weight streaming)",
+            "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "algorithmic_bytes": gbytes, "traffic": None,
+            "peak_source": f"{peak_src} HBM copy bandwidth {peaks['hbm_gbs']} GB/s"})
     if variant:  # no per-launch events in a variant run: only the standalone timing is real
         del out["kernels"]["rotate_quant_kernel (first launch of the step, events)"]
     if t_g is not None:
