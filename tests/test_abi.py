@@ -116,6 +116,8 @@ def test_other_entry_points_reject_bad_arguments_on_host(L):
     assert L.convrot_prepare_weight(FAKE, 8, 256, 256, FAKE, FAKE, FAKE, 2, None) == 3
     assert L.convrot_gemm_s32(FAKE, FAKE, 8, 6, 256, FAKE, FAKE, 256, None) == 1    # N % 4
     assert L.convrot_gemm_s32(FAKE, FAKE, 8, 8, 24, FAKE, FAKE, 256, None) == 1     # K % 16
+    # more output tiles than an int counts (no such output fits in memory, but it must not wrap)
+    assert L.convrot_gemm_s32(FAKE, FAKE, 2**31 - 1, 2**31 - 8, 256, FAKE, FAKE, 256, None) == 2
     assert L.convrot_gemm_s32(FAKE, FAKE, 8, 8, 256, FAKE, FAKE, 16, None) == 3     # workspace
     assert L.convrot_gemm_dequant(FAKE, None, FAKE, FAKE, 8, 8, 256, None, FAKE, FAKE, 256, None) == 1
     assert L.convrot_read_device_status(None, None) == 3

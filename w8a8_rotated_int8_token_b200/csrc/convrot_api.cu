@@ -73,6 +73,8 @@ convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int n_multiple)
   if (K % 16 != 0 || N % n_multiple != 0) return CONVROT_ERR_INVALID_ARG;
   const int64_t lim = (int64_t(1) << 31) - 1;
   if (M > lim || N > lim || K > lim) return CONVROT_ERR_UNSUPPORTED;
+  // the GEMM kernels count output tiles (128 x 128 at the finest) in int
+  if (((M + 127) / 128) * ((N + 127) / 128) > lim) return CONVROT_ERR_UNSUPPORTED;
   return CONVROT_OK;
 }
 
