@@ -32,6 +32,12 @@
  *     stream) on the calling thread's current device.
  *   - Arguments are checked on the host before anything is launched; a bad
  *     argument returns an error code and enqueues nothing.
+ *   - M = 0 (no tokens: an empty batch, an expert no token was routed to) is
+ *     valid wherever M appears. The call checks its other arguments, returns
+ *     CONVROT_OK and enqueues nothing; the M-sized pointers may then be NULL
+ *     and the workspace is not touched (its status word keeps its value).
+ *     convrot_linear_timed still records the caller's events, and
+ *     convrot_linear_noalloc writes 0 to its device_status.
  *   - A launch failure returns CONVROT_ERR_CUDA.
  *   - Every wait inside a kernel is bounded (about 2 s). If one runs out, the
  *     kernel records CONVROT_ERR_DEVICE_TIMEOUT in the workspace status word
@@ -101,7 +107,7 @@ CONVROT_API convrot_status convrot_prepare_weight(const void* W, int64_t N, int6
  * length-g group (fast Walsh-Hadamard transform in float32, never stored),
  * take the token's absmax, and write int8 codes and the float32 scale
  * (InvokeAI "int8 Compute", second paragraph: rotate, then quantise per token).
- *   X        [M,K] bf16, device.            M >= 1; K % g == 0; K <= CONVROT_MAX_K.
+ *   X        [M,K] bf16, device.            M >= 0; K % g == 0; K <= CONVROT_MAX_K.
  *   Xq       [M,K] int8 out, device.
  *   x_scale  [M] float out, device.
  * One kernel launch.
@@ -117,7 +123,7 @@ CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K
  * bias are fused into the GEMM epilogue. Two kernels (rotate+quantise, then
  * the GEMM, chained with programmatic dependent launch);
  * convrot_linear_launch_count reports the number for a shape.
- *   X        [M,K] bf16, device.   M >= 1, N >= 1, K % g == 0, K <= CONVROT_MAX_K,
+ *   X        [M,K] bf16, device.   M >= 0, N >= 1, K % g == 0, K <= CONVROT_MAX_K,
  *                                   N % 8 == 0.
  *   Wq       [N,K] int8, device (from convrot_prepare_weight with the same g).
  *   w_scale  1 float, device.
@@ -231,7 +237,7 @@ CONVROT_API convrot_status convrot_linear_timed(const void* X, int64_t M, int64_
                                                 void* ev_start, void* ev_mid, void* ev_end,
                                                 convrot_stream_t stream);
 
-/* Kernel launches one convrot_linear call of this shape enqueues (1 or 2), 0 if invalid. */
+/* Kernel launches one convrot_linear call of this shape enqueues: 2, or 0 for M = 0 or an invalid shape. */
 CONVROT_API int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g);
 
 /*
@@ -290,7 +296,7 @@ CONVROT_API convrot_status convrot_linear_noalloc(const void* X, int64_t M, int6
  * convrot_linear / convrot_gemm_* back to the host and return it
  * (CONVROT_OK, or CONVROT_ERR_DEVICE_TIMEOUT if a bounded wait ran out).
  * SYNCHRONISES `stream`. The word is reset at the start of every call that
- * uses the workspace.
+ * uses the workspace (except a call with M = 0, which enqueues nothing).
  */
 CONVROT_API convrot_status convrot_read_device_status(const void* ws, convrot_stream_t stream);
 

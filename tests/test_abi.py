@@ -62,7 +62,7 @@ def linear_ws_layout(M, K):
 
 
 def test_status_strings_and_version(L):
-    assert L.convrot_abi_version() == 5
+    assert L.convrot_abi_version() == 6
     for code in range(6):
         s = L.convrot_status_string(code)
         assert s and s != b"unknown status"
@@ -78,7 +78,8 @@ def test_workspace_sizes(L):
     assert L.convrot_linear_workspace_bytes(M, N, K, 64) == 0       # unsupported g
     assert L.convrot_linear_workspace_bytes(M, N, 3000, 256) == 0   # K % g != 0
     assert L.convrot_linear_workspace_bytes(M, 9212, K, 256) == 0   # N % 8 != 0
-    assert L.convrot_linear_workspace_bytes(0, N, K, 256) == 0
+    assert L.convrot_linear_workspace_bytes(0, N, K, 256) == linear_ws_layout(0, K)["total"]  # M = 0 is valid
+    assert L.convrot_linear_workspace_bytes(-1, N, K, 256) == 0
     assert L.convrot_gemm_workspace_bytes() == 256
     assert L.convrot_prepare_weight_workspace_bytes() >= 4
 
@@ -91,7 +92,6 @@ FAKE = 0x10000  # 16-byte aligned non-null value; never dereferenced: every call
     ((FAKE, 64, 256, 64, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 2),      # g unsupported
     ((FAKE, 64, 300, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),     # K % g
     ((FAKE, 64, 65536, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 40), 2),   # K above limit
-    ((FAKE, 0, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),      # M = 0
     ((FAKE, 64, 256, 256, FAKE, FAKE, 0, None, FAKE, FAKE, 1 << 30), 1),       # N = 0
     ((FAKE, 64, 256, 256, FAKE, FAKE, 260, None, FAKE, FAKE, 1 << 30), 1),     # N % 8
     ((None, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30), 1),     # null X
@@ -167,6 +167,44 @@ def test_variant_entry_points_reject_bad_arguments_on_host(L):
     assert L.convrot_quant_act_ex(FAKE, 9, 8, 256, 0, 256, FAKE, FAKE, None) == 2
     assert L.convrot_quant_act_ex(FAKE, 1, 8, 300, 0, 256, FAKE, FAKE, None) == 1
     assert L.convrot_quant_act_ex(FAKE, 1, 8, 256, 100, 256, FAKE, FAKE, None) == 1
+
+
+def test_empty_batch_is_a_checked_no_op_on_host(L):
+    """M = 0 (no tokens) returns OK and enqueues nothing; the other arguments are still checked.
+
+    There is no GPU here, so any CUDA call the library made would fail and return
+    CONVROT_ERR_CUDA (4): an OK with null data pointers and a null workspace shows
+    that nothing was launched or copied.
+    """
+    # convrot_linear(X, M, K, g, Wq, w_scale, N, bias, Y, ws, ws_bytes, stream)
+    assert L.convrot_linear(None, 0, 3072, 256, FAKE, FAKE, 9216, None, None, None, 0, None) == 0
+    assert L.convrot_linear(None, 0, 3072, 64, FAKE, FAKE, 9216, None, None, None, 0, None) == 2     # g
+    assert L.convrot_linear(None, 0, 3000, 256, FAKE, FAKE, 9216, None, None, None, 0, None) == 1    # K % g
+    assert L.convrot_linear(None, 0, 3072, 256, FAKE, FAKE, 0, None, None, None, 0, None) == 1       # N = 0
+    assert L.convrot_linear(None, 0, 3072, 256, FAKE, FAKE, 9212, None, None, None, 0, None) == 1    # N % 8
+    assert L.convrot_linear(None, -1, 3072, 256, FAKE, FAKE, 9216, None, None, None, 0, None) == 1   # M < 0
+    assert L.convrot_linear_one_launch(None, 0, 3072, 256, FAKE, FAKE, 9216, None, None, None, 0, None) == 0
+    assert L.convrot_linear_one_launch(None, 0, 20608, 128, FAKE, FAKE, 256, None, None, None, 0, None) == 2
+    assert L.convrot_linear_noalloc(None, 0, 3072, 256, FAKE, FAKE, 9216, None, None, None, None) == 0
+    assert L.convrot_linear_noalloc(None, 0, 3000, 256, FAKE, FAKE, 9216, None, None, None, None) == 1
+    assert L.convrot_linear_launch_count(0, 9216, 3072, 256) == 0
+    # convrot_linear_ex(X, dtype, M, K, ldx, g, Wq, w_scale, mode, N, bias, addend, act, Y, ldy, ws, ws_bytes, s)
+    assert L.convrot_linear_ex(None, 1, 0, 256, 0, 256, FAKE, FAKE, 1, 256, None, None, 1, None, 0, None, 0,
+                               None) == 0
+    assert L.convrot_linear_ex(None, 1, 0, 256, 260, 256, FAKE, FAKE, 1, 256, None, None, 1, None, 0, None, 0,
+                               None) == 1                                                          # ldx % 8
+    assert L.convrot_linear_ex(None, 2, 0, 256, 0, 256, FAKE, FAKE, 0, 256, None, None, 0, None, 0, None, 0,
+                               None) == 2                                                          # dtype
+    assert L.convrot_quant_act(None, 0, 256, 256, None, None, None) == 0
+    assert L.convrot_quant_act(None, 0, 256, 512, None, None, None) == 2
+    assert L.convrot_quant_act_ex(None, 1, 0, 256, 264, 256, None, None, None) == 0
+    assert L.convrot_quant_act_ex(None, 1, 0, 256, 100, 256, None, None, None) == 1
+    assert L.convrot_gemm_dequant(None, None, FAKE, FAKE, 0, 8, 256, None, None, None, 0, None) == 0
+    assert L.convrot_gemm_dequant(None, None, FAKE, FAKE, 0, 8, 24, None, None, None, 0, None) == 1  # K % 16
+    assert L.convrot_gemm_s32(None, FAKE, 0, 8, 256, None, None, 0, None) == 0
+    # a weight still has at least one output channel
+    assert L.convrot_prepare_weight(FAKE, 0, 256, 256, FAKE, FAKE, FAKE, 256, None) == 1
+    assert L.convrot_prepare_weight_ex(FAKE, 0, 0, 256, 256, 1, FAKE, FAKE, None, 0, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

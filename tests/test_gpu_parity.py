@@ -282,6 +282,43 @@ def test_zero_input_gives_zero_output_and_bias(cr):
     assert torch.equal(Yb.view(torch.int16), b.view(torch.int16).expand(130, -1))
 
 
+def test_empty_batch_gives_empty_output(cr):
+    """M = 0 (no tokens) through every public entry point: empty results, no launch, no error,
+    and the next call on the same workspace still matches the oracle."""
+    import torch
+
+    M, N, K, g = 0, 264, 1024, 256
+    d = _random_layer(130, N, K, g)
+    Wq, sw = cr.convrot_prepare_weight(to_torch_bf16(d["w"]), g)
+    X0 = torch.empty((0, K), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(cr.convrot_linear_workspace_bytes(130, N, K, g), dtype=torch.uint8, device="cuda")
+    ws.view(torch.int32)[0] = 5  # a status word left by an earlier call (the timeout code)
+    assert cr.convrot_linear(X0, Wq, sw, g, ws=ws).shape == (0, N)
+    assert cr.convrot_linear_one_launch(X0, Wq, sw, g, ws=ws).shape == (0, N)
+    Xq0, s0 = cr.convrot_quant_act(X0, g)
+    assert Xq0.shape == (0, K) and s0.shape == (0,)
+    Wc, swc = cr.convrot_prepare_weight_ex(to_torch_bf16(d["w"]).half(), g, cr.WSCALE_CHANNEL)
+    assert cr.convrot_linear_ex(X0.half(), Wc, swc, g, activation=cr.ACT_GELU_ERF).shape == (0, N)
+    assert cr.convrot_gemm_dequant(Xq0, s0, Wq, sw).shape == (0, N)
+    assert cr.convrot_gemm_s32(Xq0, Wq).shape == (0, N)
+    layer = cr.ConvRotLinear(to_torch_bf16(d["w"]), None, g)
+    assert layer(X0).shape == (0, N)
+    # the allocation-free entry reports this call's status (0), not a leftover value
+    L = cr.lib()
+    dev_status = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    assert L.convrot_linear_noalloc(None, 0, K, g, Wq.data_ptr(), sw.data_ptr(), N, None, None,
+                                    dev_status.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert int(dev_status.item()) == 0
+    assert cr.convrot_read_device_status(ws) == 5  # the empty calls left the workspace as it was
+    # a full call on the same workspace: its first kernel resets the status word
+    Y = cr.convrot_linear(to_torch_bf16(d["x"]), Wq, sw, g, ws=ws)
+    assert cr.convrot_read_device_status(ws) == 0
+    wq_ref, sw_ref = oracle.prepare_weight(oracle.bf16_to_f64(d["w"]), g)
+    ref = oracle.linear(oracle.bf16_to_f64(d["x"]), wq_ref, sw_ref, g, None)
+    assert nrmse(bf16_tensor_to_f64(Y), ref) <= NRMSE_TOL
+
+
 def _random_layer(M, N, K, g):
     rng = np.random.default_rng(M + N + K)
     x = rng.standard_normal((M, K)).astype(np.float32)

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 5;
+constexpr int kAbiVersion = 6;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
 // convrot_linear runs two kernels chained with programmatic dependent launch.
 // The one-launch form (rotate+quantise worker warps inside the GEMM kernel,
@@ -58,8 +58,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 convrot_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA; }
 
 // Checks shared by every entry point that rotates rows of length K in groups of g.
+// rows = 0 passes: the callers return before touching a buffer (an empty batch).
 convrot_status check_rotation_shape(int64_t rows, int64_t K, int g) {
-  if (rows < 1 || K < 1) return CONVROT_ERR_INVALID_ARG;
+  if (rows < 0 || K < 1) return CONVROT_ERR_INVALID_ARG;
   if (g != 128 && g != 256) return CONVROT_ERR_UNSUPPORTED;
   if (K % g != 0) return CONVROT_ERR_INVALID_ARG;
   if (K > CONVROT_MAX_K) return CONVROT_ERR_UNSUPPORTED;
@@ -68,8 +69,9 @@ convrot_status check_rotation_shape(int64_t rows, int64_t K, int g) {
 }
 
 // Checks of the GEMM shape: TMA needs 16-byte row strides; coordinates are int32.
+// M = 0 passes, as above.
 convrot_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int n_multiple) {
-  if (M < 1 || N < 1 || K < 1) return CONVROT_ERR_INVALID_ARG;
+  if (M < 0 || N < 1 || K < 1) return CONVROT_ERR_INVALID_ARG;
   if (K % 16 != 0 || N % n_multiple != 0) return CONVROT_ERR_INVALID_ARG;
   const int64_t lim = (int64_t(1) << 31) - 1;
   if (M > lim || N > lim || K > lim) return CONVROT_ERR_UNSUPPORTED;
@@ -135,6 +137,7 @@ size_t convrot_prepare_weight_workspace_bytes(void) { return 256; }
 convrot_status convrot_prepare_weight_ex(const void* W, int dtype, int64_t N, int64_t K, int g, int wscale_mode,
                                          int8_t* Wq, float* w_scale, void* ws, size_t ws_bytes,
                                          convrot_stream_t stream) {
+  if (N < 1) return CONVROT_ERR_INVALID_ARG;  // a weight has at least one output channel
   const convrot_status sh = check_rotation_shape(N, K, g);
   if (sh != CONVROT_OK) return sh;
   if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
@@ -180,9 +183,10 @@ convrot_status convrot_quant_act_ex(const void* X, int dtype, int64_t M, int64_t
   const convrot_status sh = check_rotation_shape(M, K, g);
   if (sh != CONVROT_OK) return sh;
   if (dtype != CONVROT_DTYPE_BF16 && dtype != CONVROT_DTYPE_F16) return CONVROT_ERR_UNSUPPORTED;
+  if (ldx != 0 && (ldx < K || ldx % 8 != 0)) return CONVROT_ERR_INVALID_ARG;
+  if (M == 0) return CONVROT_OK;  // no tokens: nothing to write, nothing launched
   if (X == nullptr || Xq == nullptr || x_scale == nullptr) return CONVROT_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(x_scale, 4)) return CONVROT_ERR_INVALID_ARG;
-  if (ldx != 0 && (ldx < K || ldx % 8 != 0)) return CONVROT_ERR_INVALID_ARG;
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(X);
   p.in_f16 = dtype == CONVROT_DTYPE_F16 ? 1 : 0;
@@ -225,12 +229,22 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   if (sh != CONVROT_OK) return sh;
   sh = check_gemm_shape(M, N, K, 8);
   if (sh != CONVROT_OK) return sh;
+  if ((opt.ldx != 0 && (opt.ldx < K || opt.ldx % 8 != 0)) || (opt.ldy != 0 && (opt.ldy < N || opt.ldy % 8 != 0)))
+    return CONVROT_ERR_INVALID_ARG;
+  int tpr = 0, rpp = 0, cta_threads = 0;
+  if (one_launch && (opt.general() || opt.ldx != 0 || !convrot::fused_shape(K, &tpr, &rpp, &cta_threads)))
+    return CONVROT_ERR_UNSUPPORTED;
+  if (M == 0) {
+    // no tokens: Y is empty; nothing is launched and no buffer is touched (the
+    // caller's events, if any, are still recorded so that they complete)
+    for (cudaEvent_t ev : {ev0, ev1, ev2})
+      if (ev != nullptr && cudaEventRecord(ev, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    return CONVROT_OK;
+  }
   if (X == nullptr || Wq == nullptr || w_scale == nullptr || Y == nullptr) return CONVROT_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Wq, 16) || !aligned(w_scale, opt.wscale_per_channel ? 16 : 4) ||
       !aligned(Y, 16) || (bias != nullptr && !aligned(bias, 16)) ||
       (opt.addend != nullptr && !aligned(opt.addend, 16)))
-    return CONVROT_ERR_INVALID_ARG;
-  if ((opt.ldx != 0 && (opt.ldx < K || opt.ldx % 8 != 0)) || (opt.ldy != 0 && (opt.ldy < N || opt.ldy % 8 != 0)))
     return CONVROT_ERR_INVALID_ARG;
   const LinearWs lay = linear_ws_layout(M, K);
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE;
@@ -240,9 +254,6 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
 
   if (one_launch) {
-    int tpr = 0, rpp = 0, cta_threads = 0;
-    if (opt.general() || opt.ldx != 0 || !convrot::fused_shape(K, &tpr, &rpp, &cta_threads))
-      return CONVROT_ERR_UNSUPPORTED;
     // one launch: worker warps rotate + quantise while the GEMM consumes finished M-blocks
     convrot::GemmParams gp{};
     gp.M = static_cast<int>(M);
@@ -330,7 +341,7 @@ convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K,
 
 int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g) {
   if (check_rotation_shape(M, K, g) != CONVROT_OK || check_gemm_shape(M, N, K, 8) != CONVROT_OK) return 0;
-  return 2;
+  return M == 0 ? 0 : 2;
 }
 
 convrot_status convrot_linear_one_launch(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq,
@@ -347,6 +358,7 @@ convrot_status convrot_gemm_dequant(const int8_t* Xq, const float* x_scale, cons
                                     size_t ws_bytes, convrot_stream_t stream) {
   const convrot_status sh = check_gemm_shape(M, N, K, 8);
   if (sh != CONVROT_OK) return sh;
+  if (M == 0) return CONVROT_OK;  // no tokens: nothing launched
   if (Xq == nullptr || x_scale == nullptr || Wq == nullptr || w_scale == nullptr || Y == nullptr)
     return CONVROT_ERR_INVALID_ARG;
   if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(x_scale, 4) || !aligned(w_scale, 4) ||
@@ -363,6 +375,7 @@ convrot_status convrot_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, i
                                 void* ws, size_t ws_bytes, convrot_stream_t stream) {
   const convrot_status sh = check_gemm_shape(M, N, K, 4);
   if (sh != CONVROT_OK) return sh;
+  if (M == 0) return CONVROT_OK;  // no tokens: nothing launched
   if (Xq == nullptr || Wq == nullptr || acc == nullptr) return CONVROT_ERR_INVALID_ARG;
   if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(acc, 16)) return CONVROT_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < kStatusBytes) return CONVROT_ERR_WORKSPACE;

@@ -51,14 +51,20 @@ void* scratch_address() {
 extern "C" convrot_status convrot_linear_noalloc(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq,
                                                  const float* w_scale, int64_t N, const void* bias, void* Y,
                                                  int* device_status, convrot_stream_t stream) {
-  const size_t need = convrot_linear_workspace_bytes(M, N, K, g);
-  if (need == 0) {
-    // invalid shape: let convrot_linear report which check failed, before any setup
-    return convrot_linear(X, M, K, g, Wq, w_scale, N, bias, Y, nullptr, 0, stream);
-  }
-  if (need > static_cast<size_t>(CONVROT_NOALLOC_SCRATCH_BYTES)) return CONVROT_ERR_WORKSPACE;
   if (device_status != nullptr && (reinterpret_cast<uintptr_t>(device_status) % 4) != 0)
     return CONVROT_ERR_INVALID_ARG;
+  const size_t need = convrot_linear_workspace_bytes(M, N, K, g);
+  if (need == 0 || M == 0) {
+    // an invalid shape (convrot_linear reports which check failed, before any
+    // setup) or no tokens (it returns without launching; the scratch is not
+    // used, and this call's status, 0, is what device_status receives)
+    const convrot_status st = convrot_linear(X, M, K, g, Wq, w_scale, N, bias, Y, nullptr, 0, stream);
+    if (st != CONVROT_OK || device_status == nullptr) return st;
+    return cudaMemsetAsync(device_status, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? CONVROT_OK
+               : CONVROT_ERR_CUDA;
+  }
+  if (need > static_cast<size_t>(CONVROT_NOALLOC_SCRATCH_BYTES)) return CONVROT_ERR_WORKSPACE;
   void* ws = scratch_address();
   if (ws == nullptr) return CONVROT_ERR_CUDA;
   const convrot_status st =
