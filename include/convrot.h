@@ -46,6 +46,11 @@
  *   - Entry points hold no state between calls (convrot_linear_noalloc's
  *     built-in scratch aside) and are safe to call from several host threads
  *     on different streams with separate workspaces.
+ *   - A call may be captured into a CUDA graph (stream capture); each replay
+ *     recomputes everything from the current contents of the captured
+ *     buffers. The exception is convrot_linear_one_launch, which refuses a
+ *     capturing stream. convrot_linear_noalloc needs one call on the device
+ *     before any capture begins.
  */
 #ifndef CONVROT_H
 #define CONVROT_H
@@ -152,7 +157,10 @@ CONVROT_API convrot_status convrot_linear(const void* X, int64_t M, int64_t K, i
  * measured slower than the two-kernel convrot_linear (137 against 110 us).
  * Same arguments, workspace and errors as convrot_linear, plus
  * CONVROT_ERR_UNSUPPORTED when K > 20480 (the worker warps of one CTA hold a
- * token) or K % 128 != 0.
+ * token) or K % 128 != 0. Not for CUDA graphs: the counters' per-call tag is
+ * drawn on the host at each call, so a replayed graph would reuse it. A call
+ * on a stream that is capturing returns CONVROT_ERR_UNSUPPORTED and enqueues
+ * nothing.
  */
 CONVROT_API convrot_status convrot_linear_one_launch(const void* X, int64_t M, int64_t K, int g,
                                                      const int8_t* Wq, const float* w_scale, int64_t N,

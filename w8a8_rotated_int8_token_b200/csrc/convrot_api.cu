@@ -254,6 +254,12 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   int8_t* Xq = reinterpret_cast<int8_t*>(wsb + lay.codes_off);
 
   if (one_launch) {
+    // The call's epoch is drawn here on the host: a CUDA graph would replay
+    // the captured value, and from the second replay on the readiness
+    // counters would already hold it. So a capturing stream is refused.
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (capture != cudaStreamCaptureStatusNone) return CONVROT_ERR_UNSUPPORTED;
     // one launch: worker warps rotate + quantise while the GEMM consumes finished M-blocks
     convrot::GemmParams gp{};
     gp.M = static_cast<int>(M);
