@@ -262,3 +262,34 @@ def test_strided_quant_act_is_the_dense_one(cr):
     q1, s1 = cr.convrot_quant_act_ex(Xbig[:, :K], g)
     torch.cuda.synchronize()
     assert torch.equal(q0, q1) and torch.equal(s0, s1)
+
+
+@pytest.mark.parametrize("M", [200, 16])
+def test_layer_wrapper_runs_the_variant_entry_points(cr, M):
+    """ConvRotLinear with fp16, per-channel scales, GELU and an addend gives, bit for bit, what the
+    direct calls it stands for give, and the default wrapper what convrot_linear gives."""
+    import torch
+
+    N, K, g = 264, 1024, 256
+    rng = np.random.default_rng(M)
+    x = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    w = synth.f32_to_bf16_bits((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+    b = synth.f32_to_bf16_bits((rng.standard_normal(N) * 0.01).astype(np.float32))
+    z = synth.f32_to_bf16_bits((rng.standard_normal((M, N)) * 0.05).astype(np.float32))
+    X, W, B, Z = (_to_torch(_as_dtype_bits(t, F16), F16) for t in (x, w, b, z))
+
+    layer = cr.ConvRotLinear(W, B, g, wscale_mode=cr.WSCALE_CHANNEL, activation=cr.ACT_GELU_ERF)
+    assert layer.w_scale.shape == (N,)
+    Y = layer(X, addend=Z)
+    Wq, sw = cr.convrot_prepare_weight_ex(W, g, cr.WSCALE_CHANNEL)
+    Y_direct = cr.convrot_linear_ex(X, Wq, sw, g, B, cr.ACT_GELU_ERF, addend=Z)
+    torch.cuda.synchronize()
+    assert torch.equal(layer.Wq, Wq) and torch.equal(layer.w_scale, sw)
+    assert Y.dtype == torch.float16 and torch.equal(Y.view(torch.int16), Y_direct.view(torch.int16))
+
+    Xb, Wb, Bb = (_to_torch(t, BF16) for t in (x, w, b))
+    plain = cr.ConvRotLinear(Wb, Bb, g)
+    Wq_b, sw_b = cr.convrot_prepare_weight(Wb, g)
+    Y_plain = plain(Xb)
+    torch.cuda.synchronize()
+    assert torch.equal(Y_plain.view(torch.int16), cr.convrot_linear(Xb, Wq_b, sw_b, g, Bb).view(torch.int16))

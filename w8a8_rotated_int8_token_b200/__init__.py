@@ -347,13 +347,23 @@ class ConvRotLinear:
     """A ConvRot linear layer: prepared int8 weight + optional bias, reusable workspace.
 
     ``layer = ConvRotLinear(W, bias, g=256)`` rotates and quantises W once;
-    ``layer(X)`` runs convrot_linear on the current stream.
+    ``layer(X)`` runs convrot_linear on the current stream. With a float16 W,
+    ``wscale_mode=WSCALE_CHANNEL`` or ``activation=ACT_GELU_ERF`` the layer
+    runs convrot_linear_ex instead (X, bias and Y then share W's dtype), and
+    ``layer(X, addend=Z)`` adds Z [M,N] before the activation.
     """
 
-    def __init__(self, W, bias=None, g: int = 256):
+    def __init__(self, W, bias=None, g: int = 256, wscale_mode: int = WSCALE_TENSOR, activation: int = ACT_NONE):
+        import torch
+
         self.g = g
         self.N, self.K = W.shape
-        self.Wq, self.w_scale = convrot_prepare_weight(W, g)
+        self.activation = int(activation)
+        self.general = W.dtype != torch.bfloat16 or wscale_mode != WSCALE_TENSOR or self.activation != ACT_NONE
+        if self.general:
+            self.Wq, self.w_scale = convrot_prepare_weight_ex(W, g, wscale_mode)
+        else:
+            self.Wq, self.w_scale = convrot_prepare_weight(W, g)
         self.bias = bias
         self._ws = None
 
@@ -365,5 +375,9 @@ class ConvRotLinear:
             self._ws = torch.empty((need,), dtype=torch.uint8, device=self.Wq.device)
         return self._ws
 
-    def __call__(self, X, Y=None, stream=None):
-        return convrot_linear(X, self.Wq, self.w_scale, self.g, self.bias, Y, self.workspace(X.shape[0]), stream)
+    def __call__(self, X, Y=None, stream=None, addend=None):
+        ws = self.workspace(X.shape[0])
+        if self.general or addend is not None:
+            return convrot_linear_ex(X, self.Wq, self.w_scale, self.g, self.bias, self.activation, Y, ws, stream,
+                                     addend)
+        return convrot_linear(X, self.Wq, self.w_scale, self.g, self.bias, Y, ws, stream)
