@@ -149,7 +149,8 @@ def _gemm_exact(cr, xq: np.ndarray, wq: np.ndarray, rows=None):
 
 
 @pytest.mark.parametrize("M,N,K", [(64, 256, 256), (1, 8, 16), (1, 256, 128), (130, 264, 272), (257, 520, 4096),
-                                   (128, 1024, 12288), (513, 12288, 128)])
+                                   (128, 1024, 12288), (513, 12288, 128),
+                                   (8, 20480, 256)])  # weight-streaming form, 160 tiles: two per CTA on some SMs
 def test_gemm_s32_bit_exact(cr, M, N, K):
     rng = np.random.default_rng(M + N + K)
     xq = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
@@ -331,7 +332,8 @@ def _random_layer(M, N, K, g):
 
 @pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256), (129, 136, 20608, 128),
                                      (67, 264, 32768, 256),    # largest K
-                                     (1, 16, 384, 128), (385, 520, 1024, 256)])
+                                     (1, 16, 384, 128), (385, 520, 1024, 256),
+                                     (33, 19712, 512, 256)])  # 154 weight tiles at M <= 64 (vocabulary-sized N)
 def test_linear_ragged_and_large_k(cr, M, N, K, g):
     _linear_case(cr, _random_layer(M, N, K, g))
 
