@@ -46,11 +46,12 @@
  *   - Entry points hold no state between calls (convrot_linear_noalloc's
  *     built-in scratch aside) and are safe to call from several host threads
  *     on different streams with separate workspaces.
- *   - A call may be captured into a CUDA graph (stream capture); each replay
- *     recomputes everything from the current contents of the captured
- *     buffers. The exception is convrot_linear_one_launch, which refuses a
- *     capturing stream. convrot_linear_noalloc needs one call on the device
- *     before any capture begins.
+ *   - Calls that only enqueue work may be captured into a CUDA graph (stream
+ *     capture); each replay recomputes everything from the current contents
+ *     of the captured buffers. The exceptions: convrot_linear_one_launch
+ *     refuses a capturing stream, convrot_read_device_status synchronises and
+ *     so cannot be captured, and convrot_linear_noalloc needs one call on the
+ *     device before any capture begins.
  */
 #ifndef CONVROT_H
 #define CONVROT_H
