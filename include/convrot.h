@@ -287,9 +287,12 @@ CONVROT_API convrot_status convrot_gemm_s32(const int8_t* Xq, const int8_t* Wq,
  *   roughly M*K > 64 MiB) returns CONVROT_ERR_WORKSPACE and enqueues nothing.
  *   device_status: NULL, or a device int that receives the call's status word
  *   (0, or CONVROT_ERR_DEVICE_TIMEOUT) once the call has run on `stream`.
- * Allocates nothing. The first call on each device looks up the array's device
- * address (cudaGetSymbolAddress, with that device current) and keeps it; make
- * that first call before any stream capture begins. All calls share the array:
+ * Allocates nothing. The first call in each CUDA context looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current) and keeps it
+ * with the context's id; make that first call before any stream capture
+ * begins. cudaDeviceReset between calls is supported: the next call is the
+ * first one in the new context and looks the address up again (before any
+ * capture, as above). All calls share the array:
  * calls that may overlap on the GPU (unordered streams, several host threads)
  * race on it and must not be issued. Each call clears the status word and
  * rewrites the codes and scales, so no result depends on an earlier call.

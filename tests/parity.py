@@ -7,7 +7,11 @@ Tolerances (stated once, used everywhere):
     boundary (k + 0.5): the kernel rotates in float32 with a different
     summation order, so only near-ties may round the other way.
   * token / tensor scales: relative difference <= 1e-6.
-  * bf16 output: NRMSE <= 2e-3 against the oracle's float64 result.
+  * bf16 output: NRMSE <= 2e-3 against the oracle's float64 result, and
+    every element within the rounding bound of the oracle's arithmetic applied
+    to the kernel's own codes and scales (``check_output_elementwise``): the
+    one output rounding (half an ulp of bf16 or fp16) plus the float32
+    dequantisation roundings, so that a single wrong element fails.
 """
 
 from __future__ import annotations
@@ -58,6 +62,63 @@ def check_codes(q_gpu: np.ndarray, s_gpu: np.ndarray, x_rot: np.ndarray, q_ref: 
         assert tie_dist.max() <= CODE_TIE_WINDOW, f"a differing code is not at a near-tie ({tie_dist.max()})"
     assert q_gpu.min(initial=0) >= -127 and q_gpu.max(initial=0) <= 127, "a code outside the range [-127, 127]"
     return {"mismatch_frac": frac, "scale_rel_max": float(rel.max(initial=0.0))}
+
+
+OUT_REL = {"bf16": 2.0**-8, "f16": 2.0**-11}  # half an ulp, relative: 8 and 11 significant bits
+OUT_ABS = {"bf16": 2.0**-134, "f16": 2.0**-25}  # half the smallest subnormal
+F32_REL = 2.0**-21                           # a few float32 roundings in the epilogue (2^-24 each)
+GELU_REL = 4e-7                              # erf approximation (<= 1.5e-7) and exp rounding, relative to |z|
+
+
+def check_output_elementwise(y: np.ndarray, acc: np.ndarray, s_x: np.ndarray, s_w, bias=None, addend=None,
+                             gelu: bool = False, out: str = "bf16") -> float:
+    """Bound every output element against z = acc * (s_x[m] * s_w) + bias[n] (+ addend), then GELU.
+
+    ``acc``, ``s_x`` and ``s_w`` are the kernel's own int32 accumulators (from
+    the oracle's exact GEMM of the kernel's codes) and scales, which the
+    caller has already checked against the oracle with ``check_codes``. What
+    is left between the kernel and this float64 value is the epilogue's
+    float32 arithmetic and the single rounding to the output dtype:
+
+        |y - ref| <= OUT_REL * |ref| + (1 + OUT_REL) * err + OUT_ABS,
+        err = F32_REL * (|acc * s_x * s_w| + |bias| + |addend|)  (times 1.13, GELU's largest slope,
+              plus GELU_REL * |z| with GELU).
+
+    Returns the largest |y - ref| / bound (<= 1 passes); raises on a violation.
+    """
+    y = np.asarray(y, np.float64)
+    acc = np.asarray(acc, np.float64)
+    sx = np.asarray(s_x, np.float64)[:, None]
+    sw = np.asarray(s_w, np.float64)
+    sw = sw[None, :] if sw.ndim == 1 and sw.size > 1 else sw.reshape(())
+    prod = acc * (sx * sw)
+    z = prod.copy()
+    mag = np.abs(prod)
+    if bias is not None:
+        b = np.asarray(bias, np.float64)[None, :]
+        z = z + b
+        mag = mag + np.abs(b)
+    if addend is not None:
+        a = np.asarray(addend, np.float64)
+        z = z + a
+        mag = mag + np.abs(a)
+    err = F32_REL * mag
+    if gelu:
+        from scipy.special import erf
+
+        ref = 0.5 * z * (1.0 + erf(z / np.sqrt(2.0)))
+        err = 1.13 * err + GELU_REL * np.abs(z)
+    else:
+        ref = z
+    bound = OUT_REL[out] * np.abs(ref) + (1.0 + OUT_REL[out]) * err + OUT_ABS[out] + 1e-300
+    assert np.all(np.isfinite(y)), "a non-finite output element"
+    ratio = np.abs(y - ref) / bound
+    worst = float(ratio.max(initial=0.0))
+    if worst > 1.0:
+        i = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+        raise AssertionError(f"output element {tuple(int(v) for v in i)} = {y[i]!r}, expected {ref[i]!r} "
+                             f"within {bound[i]:.3e} ({worst:.2f} x the bound)")
+    return worst
 
 
 def nrmse(y: np.ndarray, ref: np.ndarray) -> float:

@@ -13,7 +13,8 @@ import pytest
 
 import oracle
 import synth
-from parity import (NRMSE_TOL, bf16_tensor_to_f64, check_codes, nrmse, to_torch_bf16)
+from parity import (NRMSE_TOL, bf16_tensor_to_f64, check_codes, check_output_elementwise, nrmse,
+                    to_torch_bf16)
 from test_abi import linear_ws_layout
 
 pytestmark = pytest.mark.gpu
@@ -234,6 +235,13 @@ def _linear_case(cr, d, rows=None, one_launch=False):
     xr = oracle.rotate(xs, g)
     q_ref, s_ref = oracle.quantize_per_token(xr)
     check_codes(xq_gpu, sx_gpu, xr, q_ref, s_ref)
+    # the weight codes and scale the kernel prepared, then every output element
+    # against the oracle's arithmetic on the kernel's own codes and scales
+    wq_gpu = Wq.cpu().numpy()
+    sw_gpu = sw.cpu().numpy().reshape(1)
+    check_codes(wq_gpu, sw_gpu, oracle.rotate(oracle.bf16_to_f64(d["w"]), g), wq_ref, np.array([sw_ref]),
+                per_token=False)
+    check_output_elementwise(y, oracle.gemm_s32(xq_gpu, wq_gpu), sx_gpu, float(sw_gpu[0]), b)
     return Y, err
 
 

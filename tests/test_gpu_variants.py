@@ -15,7 +15,8 @@ import pytest
 
 import oracle
 import synth
-from parity import NRMSE_TOL, check_codes, nrmse
+from parity import NRMSE_TOL, check_codes, check_output_elementwise, nrmse
+from test_abi import linear_ws_layout
 
 pytestmark = pytest.mark.gpu
 
@@ -70,6 +71,37 @@ def _from_torch(t, dtype: int) -> np.ndarray:
     return _to_f64(u16, dtype)
 
 
+def _kernel_codes(ws, M: int, K: int, rows: np.ndarray):
+    """The token scales and activation codes a layer call left in its workspace (sampled rows)."""
+    wsn = ws.cpu().numpy()
+    lay = linear_ws_layout(M, K)
+    sx = wsn[lay["scale"]:lay["scale"] + 4 * M].view(np.float32)[rows]
+    xq = wsn[lay["codes"]:lay["codes"] + M * K].view(np.int8).reshape(M, K)[rows]
+    return xq, sx
+
+
+def _check_elementwise(ws, M, K, rows, x_rows64, w64, g, mode, Wq, sw, y, bias64, addend64, act, dtype):
+    """The call's codes and scales against the oracle's (near-ties only), then every output
+    element against the oracle's arithmetic on the kernel's own codes and scales."""
+    xq_gpu, sx_gpu = _kernel_codes(ws, M, K, rows)
+    xr = oracle.rotate(x_rows64, g)
+    q_ref, s_ref = oracle.quantize_per_token(xr)
+    check_codes(xq_gpu, sx_gpu, xr, q_ref, s_ref)
+    wq_gpu = Wq.cpu().numpy()
+    sw_gpu = sw.cpu().numpy().reshape(-1)
+    wr = oracle.rotate(w64, g)
+    if mode == CHANNEL:
+        wq_ref, sw_ref = oracle.quantize_per_token(wr)
+        check_codes(wq_gpu, sw_gpu, wr, wq_ref, sw_ref)
+        sw_use = sw_gpu
+    else:
+        wq_ref, sw_ref = oracle.quantize_tensorwise(wr)
+        check_codes(wq_gpu, sw_gpu, wr, wq_ref, np.array([sw_ref]), per_token=False)
+        sw_use = float(sw_gpu[0])
+    return check_output_elementwise(y, oracle.gemm_s32(xq_gpu, wq_gpu), sx_gpu, sw_use, bias64, addend64,
+                                    gelu=(act == GELU), out="bf16" if dtype == BF16 else "f16")
+
+
 def _oracle_layer(x, w, g, mode, bias, act):
     if mode == CHANNEL:
         wq, sw = oracle.prepare_weight_per_channel(w, g)
@@ -121,6 +153,8 @@ def test_linear_ex_matches_oracle(cr, name, dtype, mode, act):
     assert np.all(np.isfinite(y))
     err = nrmse(y, ref)
     assert err <= NRMSE_TOL, f"{name} dtype={dtype} mode={mode} act={act}: NRMSE {err}"
+    _check_elementwise(ws, M, K, rows, _to_f64(xb[rows], dtype), _to_f64(wb, dtype), g, mode, Wq, sw, y,
+                       None if bb is None else _to_f64(bb, dtype), None, act, dtype)
 
 
 @pytest.mark.parametrize("name,dtype", [("tiny", BF16), ("tiny", F16), ("dit_qkv_1024", BF16), ("textenc_m16", F16)])
@@ -247,6 +281,8 @@ def test_strided_rows_and_addend_match_oracle(cr, name, dtype, act):
     y = _from_torch(Y.contiguous(), dtype)[rows]
     err = nrmse(y, ref)
     assert err <= NRMSE_TOL, f"{name}: NRMSE {err}"
+    _check_elementwise(ws, M, K, rows, _to_f64(xb[rows], dtype), _to_f64(wb, dtype), g, TENSOR, Wq, sw, y,
+                       None if bb is None else _to_f64(bb, dtype), _to_f64(zb[rows], dtype), act, dtype)
 
 
 def test_strided_quant_act_is_the_dense_one(cr):

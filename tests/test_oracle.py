@@ -353,6 +353,38 @@ def test_nrmse_definition():
 # FP16 compute dtype, per-output-channel weight scale, exact-erf GELU.
 
 
+def _bf16_from_definition(bits: int) -> float:
+    """bfloat16 decoded by hand: sign, 8-bit exponent (bias 127), 7-bit fraction (the upper
+    half of an IEEE binary32 word)."""
+    s = -1.0 if bits & 0x8000 else 1.0
+    e = (bits >> 7) & 0xFF
+    f = bits & 0x7F
+    if e == 0:
+        return s * f * 2.0**-133
+    if e == 255:
+        return s * float("inf") if f == 0 else float("nan")
+    return s * (1.0 + f / 128.0) * 2.0 ** (e - 127)
+
+
+@pytest.mark.parametrize("bits,value", [(0x3F80, 1.0), (0xC000, -2.0), (0x3FFF, 1.9921875),
+                                        (0x7F7F, (2.0 - 2.0**-7) * 2.0**127), (0x0001, 2.0**-133),
+                                        (0x007F, 127 * 2.0**-133), (0x0080, 2.0**-126), (0x4049, 3.140625),
+                                        (0xBE4D, -0.2001953125), (0x8000, -0.0), (0x7F80, float("inf"))])
+def test_bf16_widening_follows_the_format(bits, value):
+    got = float(oracle.bf16_to_f64(np.array([bits], np.uint16))[0])
+    assert got == value == _bf16_from_definition(bits)
+    assert np.signbit(got) == bool(bits & 0x8000)
+
+
+def test_bf16_widening_of_every_finite_pattern():
+    bits = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16)
+    finite = ((bits >> 7) & 0xFF) != 0xFF
+    got = oracle.bf16_to_f64(bits[finite])
+    want = np.array([_bf16_from_definition(int(b)) for b in bits[finite]])
+    assert np.array_equal(got, want)
+    assert np.array_equal(np.signbit(got), (bits[finite] & 0x8000) != 0)
+
+
 def _f16_from_definition(bits: int) -> float:
     """IEEE binary16 decoded by hand: sign, 5-bit exponent (bias 15), 10-bit fraction."""
     s = -1.0 if bits & 0x8000 else 1.0

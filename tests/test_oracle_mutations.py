@@ -35,6 +35,8 @@ MUTATIONS = {
     "per_channel_scale_tensorwise": ("    return quantize_per_token(rotate(w, g))\n",
                                      "    q, s = quantize_tensorwise(rotate(w, g))\n    return q, np.full(q.shape[0], s)\n"),
     "addend_dropped": ("        y = y + np.asarray(addend, np.float64)\n", "        y = y\n"),
+    "bf16_low_mantissa_dropped": ("(np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16)",
+                                  "((np.asarray(bits, dtype=np.uint16).astype(np.uint32) & 0xFFF0) << 16)"),
     "per_channel_scale_on_tokens_axis": ("np.asarray(s_w, np.float64)[None, :])", "np.asarray(s_w, np.float64)[:, None])"),
 }
 

@@ -9,9 +9,13 @@
 // int8 activation codes) lives here in one file-scope device array of fixed
 // size, allocated when the library's device code is loaded on a GPU and held
 // until the process exits. Host code cannot use the array's name as a device
-// address (it is a host-side stand-in), so the first call on each device asks
-// the runtime for the array's device address with cudaGetSymbolAddress, with
-// that device current, and keeps it for later calls.
+// address (it is a host-side stand-in), so the first call in each CUDA
+// context asks the runtime for the array's device address with
+// cudaGetSymbolAddress, with that device current, and keeps it together with
+// the context's unique id. A later call in another context of the same device
+// (after cudaDeviceReset, or once the primary context was released and made
+// anew, which loads the module again and may move the array) looks it up
+// again.
 //
 // Every call shares the one array and leaves its contents behind. The status
 // word is cleared by the first kernel of every call, and the codes and scales
@@ -19,10 +23,11 @@
 // Calls that may overlap on the GPU (different streams without ordering, or
 // several host threads) race on the array and must not be issued.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "convrot.h"
 
@@ -32,17 +37,68 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[CONVROT_NOALLOC
 namespace {
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
 
-// Device address of g_noalloc_scratch on the current device (set up once per device).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The driver's context queries, found once through the runtime (the library
+// does not link libcuda directly).
+bool context_queries(CtxGetCurrentFn* get_current, CtxGetIdFn* get_id) {
+  static CtxGetCurrentFn cur = nullptr;
+  static CtxGetIdFn id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      cur = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  *get_current = cur;
+  *get_id = id;
+  return cur != nullptr && id != nullptr;
+}
+
+// Unique id of the calling thread's current context (0 if there is none).
+unsigned long long current_context_id(CtxGetCurrentFn get_current, CtxGetIdFn get_id) {
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+struct ScratchSlot {
+  unsigned long long ctx_id = 0;  // context the address belongs to (0: none yet)
+  void* addr = nullptr;
+};
+
+std::mutex g_scratch_mutex;
+ScratchSlot g_scratch_slot[kMaxDevices];
+
+// Device address of g_noalloc_scratch in the current device's current context.
 void* scratch_address() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p != nullptr) return p;
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+  if (!context_queries(&get_current, &get_id)) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  ScratchSlot& slot = g_scratch_slot[dev];
+  unsigned long long id = current_context_id(get_current, get_id);
+  if (id != 0 && id == slot.ctx_id) return slot.addr;
+  // first call in this context (the lookup also makes the device's primary
+  // context current if no context was yet)
   void* addr = nullptr;
   if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) return nullptr;
-  g_scratch_addr[dev].store(addr, std::memory_order_release);
+  id = current_context_id(get_current, get_id);
+  if (id == 0) return nullptr;
+  slot.ctx_id = id;
+  slot.addr = addr;
   return addr;
 }
 
