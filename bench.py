@@ -10,6 +10,22 @@ g=256, with bias.
     python bench.py --impl reference ...   # the CPU oracle as the reference arm
     python bench.py --dtype f16 --wscale channel --act gelu   # a layer variant (convrot_linear_ex)
 
+Besides the headline the line carries:
+  * ``int8_peak``: the int8 tensor pipe's rate measured on this GPU by a probe
+    that issues the GEMM's own instruction (tcgen05.mma.cta_group::2.kind::i8,
+    256x256x32) from shared memory with no global traffic, in bursts (the
+    denominator of the GEMM's roofline) and in a longer loop under the power
+    limit (sustained);
+  * ``configs``: every layer shape of the workload table timed by CUDA events
+    (median and min over the repetitions, inputs rotated over enough buffer
+    sets to exceed L2): the layer's time per call, TOPS, the GEMM's TOPS and
+    fraction of the int8 peak, the rotate+quantise pass's GB/s and fraction of
+    HBM, and for the weight-streaming shapes (M <= 128) the fraction of HBM on
+    the layer's algorithmic bytes;
+  * ``e2e``: the same metric through the public Python API with host buffers,
+    the host-to-device copies, the layers and the device-to-host copies on
+    three streams ordered by events over the rotating buffer sets.
+
 Under torchrun (N > 1) every rank runs an independent replica of the same
 workload on its own GPU (the layer has no cross-GPU step); the value is the
 work of all ranks over the slowest rank's device time.
@@ -19,6 +35,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -33,9 +50,12 @@ sys.path.insert(0, ROOT)
 METRIC = "ConvRot linear TOPS (rotate+quant+i8 GEMM+dequant) and % of B200 INT8 peak"
 UNIT = "TOPS"
 N_SETS = 4  # rotating input/output sets per rank so that no step finds its data in L2
+L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200
+INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200 (context only)
+NOMINAL_INT8_TOPS = 4500.0  # datasheet dense int8 (context only)
 SMALL_M = 64  # up to this many tokens the layer's GEMM is the weight-streaming form
+PROBE_OPS_PER_ITER_PER_PAIR = 2.0 * 256 * 256 * 128  # four 256x256x32 MMAs
 
 # DRAM bytes per launch of the dominant kernel (the pair GEMM) on a workload,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum). A
@@ -47,6 +67,10 @@ GEMM_TRAFFIC = {
     "dit_qkv_1024": {"bytes": 59904768 + 48083456,
                      "sources_sha256": "a070901777178b94bffd44bd6441f83d97c2752a4107e86a9b74e32cf4b4c482"},
 }
+
+# Every layer shape of the workload table, timed after the headline.
+CONFIG_NAMES = ["tiny", "dit_qkv_1024", "dit_mlp_up_1024", "dit_mlp_down_1024", "dit_mlp_2048",
+                "textenc_m1", "textenc_m16", "textenc_m128", "textenc_m512"]
 
 
 def gemm_traffic(config: str):
@@ -62,7 +86,7 @@ def gemm_traffic(config: str):
     return float(rec["bytes"]) if h.hexdigest() == rec["sources_sha256"] else None
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
@@ -72,11 +96,14 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config table")
+    ap.add_argument("--no-peak", action="store_true", help="skip the int8 peak probe")
+    ap.add_argument("--config-reps", type=int, default=30, help="timed repetitions per config")
     # layer variants (convrot_linear_ex); the defaults are the headline layer
     ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16", help="dtype of X, W, bias and Y")
     ap.add_argument("--wscale", choices=["tensor", "channel"], default="tensor", help="weight-scale granularity")
     ap.add_argument("--act", choices=["none", "gelu"], default="none", help="activation fused into the epilogue")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def reduce_max(v: float, device) -> float:
@@ -114,6 +141,15 @@ def workload_config(w) -> dict:
                   f"{N_SETS - 1} steps earlier (>126 MB L2 in between)"}
 
 
+def sets_for(bytes_per_set: float) -> int:
+    """Rotating buffer sets so that a set is reused only after more than L2's worth of other sets."""
+    return int(min(8, max(N_SETS, math.ceil(2 * L2_BYTES / max(bytes_per_set, 1.0)) + 1)))
+
+
+def med_min(xs):
+    return float(statistics.median(xs)), float(min(xs))
+
+
 # --------------------------------------------------------------- clocks
 
 
@@ -124,7 +160,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.index = index
         self.period = period_s
         self.samples = []
@@ -258,6 +294,251 @@ def run_reference(args):
 # ------------------------------------------------------------------ GPU
 
 
+def bits_to_dev(bits, dev, dtype=None):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    return t if dtype is None or dtype == torch.bfloat16 else t.to(dtype)
+
+
+def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, sustained_s: float = 0.4) -> dict:
+    """The int8 tensor pipe's rate on this GPU (probe of the GEMM's own instruction, no global traffic).
+
+    burst: single launches of about `burst_ms`, timed by events, after two warm-up
+    launches (the GEMM is timed the same way, alone or inside short steps);
+    sustained: launches back to back for about `sustained_s` under the power limit.
+    """
+    import torch
+
+    ws = torch.empty((256,), dtype=torch.uint8, device=dev)
+    ctas = cr.convrot_probe_i8_peak(64, ws=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    pairs = ctas // 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # calibrate the iteration count to about burst_ms per launch
+    iters = 1024
+    e0.record(stream)
+    cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    iters = int(max(256, min(1 << 20, iters * burst_ms / max(e0.elapsed_time(e1), 1e-3))))
+    ops = PROBE_OPS_PER_ITER_PER_PAIR * iters * pairs
+    for _ in range(2):
+        cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    burst = []
+    with ClockSampler(clock_index, 0.001) as clk_b:
+        for _ in range(5):
+            e0.record(stream)
+            cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            burst.append(ops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+    n_sus = int(max(1, sustained_s * 1e3 / burst_ms))
+    with ClockSampler(clock_index, 0.005) as clk_s:
+        e0.record(stream)
+        for _ in range(n_sus):
+            cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    sustained = ops * n_sus / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    if cr.convrot_read_device_status(ws) != 0:
+        raise RuntimeError("int8 peak probe: a device wait timed out")
+    b, s = clk_b.summary(), clk_s.summary()
+    return {"burst_tops": max(burst), "burst_tops_median": statistics.median(burst), "sustained_tops": sustained,
+            "burst_clock_mhz": b["sm_mhz"], "sustained_clock_mhz": s["sm_mhz"],
+            "reasons": sorted(set(b["reasons"]) | set(s["reasons"])),
+            "ops_per_clk_per_sm_burst": (max(burst) * 1e12 / (b["sm_mhz"] * 1e6) / ctas) if b["sm_mhz"] else None,
+            "probe": f"{pairs} CTA pairs x {iters} x 4 tcgen05.mma.cta_group::2.kind::i8 (256x256x32), "
+                     f"operands in shared memory, no global traffic; burst = best of 5 launches of ~{burst_ms:g} ms, "
+                     f"sustained = {n_sus} launches back to back",
+            "context": {"nominal_dense_int8_tops": NOMINAL_INT8_TOPS}}
+
+
+def layer_inputs(cr, name: str, dev, up_cache: dict):
+    """Device tensors of one config: X (bf16 [M,K]), the prepared weight, bias."""
+    import synth
+    import torch
+
+    if name == "dit_mlp_down_1024":
+        # the down projection's input is GELU of the up projection's output: the
+        # up layer itself, with the GELU fused into its epilogue, produces it here
+        if "down_x" not in up_cache:
+            du = synth.make_workload("dit_mlp_up_1024")
+            wq_u, sw_u = cr.convrot_prepare_weight(bits_to_dev(du["w"], dev), du["workload"].g)
+            up_cache["down_x"] = cr.convrot_linear_ex(bits_to_dev(du["x"], dev), wq_u, sw_u, du["workload"].g, None,
+                                                      cr.ACT_GELU_ERF)
+            torch.cuda.synchronize(dev)
+        w = synth.CONFIGS[name]
+        rng = np.random.default_rng(w.seed)
+        wt = rng.standard_normal((w.N, w.K), dtype=np.float32) * np.float32(w.w_std)
+        Wq, sw = cr.convrot_prepare_weight(bits_to_dev(synth.f32_to_bf16_bits(wt), dev), w.g)
+        return w, up_cache["down_x"], Wq, sw, None
+    d = synth.make_workload(name)
+    w = d["workload"]
+    Wq, sw = cr.convrot_prepare_weight(bits_to_dev(d["w"], dev), w.g)
+    bias = None if d["bias"] is None else bits_to_dev(d["bias"], dev)
+    return w, bits_to_dev(d["x"], dev), Wq, sw, bias
+
+
+def bench_config(cr, L, name: str, dev, stream, reps: int, peaks: dict, i8_peak, up_cache: dict) -> dict:
+    """Per-config timing by CUDA events (median and min over `reps`), inputs rotated over buffer sets."""
+    import torch
+
+    w, X0, Wq0, sw, bias = layer_inputs(cr, name, dev, up_cache)
+    M, K, N, g = w.M, w.K, w.N, w.g
+    ws_bytes = cr.convrot_linear_workspace_bytes(M, N, K, g)
+    per_set = 2.0 * M * K + N * K + 2.0 * M * N + ws_bytes
+    ns = sets_for(per_set)
+    sets = [{"X": X0 if i == 0 else X0.clone(), "Wq": Wq0 if i == 0 else Wq0.clone(),
+             "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+             "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=dev),
+             "Xq": torch.empty((M, K), dtype=torch.int8, device=dev),
+             "sx": torch.empty((M,), dtype=torch.float32, device=dev)} for i in range(ns)]
+    sp = stream.cuda_stream
+    b_ptr = None if bias is None else bias.data_ptr()
+
+    def call(i):
+        s = sets[i % ns]
+        st = L.convrot_linear(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw.data_ptr(), N, b_ptr,
+                              s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, sp)
+        if st != 0:
+            raise cr.ConvRotError(st, f"convrot_linear ({name})")
+
+    for i in range(5):
+        call(i)
+    torch.cuda.synchronize(dev)
+    # back to back (the two launches of a call overlap as in a real forward pass)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(reps):
+        call(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_b2b = e0.elapsed_time(e1) / reps
+    # per call and per kernel: events before, between and after the two launches
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for trip in ev:
+        for e in trip:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    for i in range(reps):
+        s = sets[i % ns]
+        st = L.convrot_linear_timed(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw.data_ptr(), N, b_ptr,
+                                    s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, ev[i][0].cuda_event,
+                                    ev[i][1].cuda_event, ev[i][2].cuda_event, sp)
+        if st != 0:
+            raise cr.ConvRotError(st, f"convrot_linear_timed ({name})")
+    torch.cuda.synchronize(dev)
+    t_q_in = [e[0].elapsed_time(e[1]) for e in ev]
+    t_g_in = [e[1].elapsed_time(e[2]) for e in ev]
+    # the rotate+quantise pass alone, each launch between its own events
+    evq = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for i in range(reps):
+        s = sets[i % ns]
+        evq[i][0].record(stream)
+        L.convrot_quant_act(s["X"].data_ptr(), M, K, g, s["Xq"].data_ptr(), s["sx"].data_ptr(), sp)
+        evq[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_q = [e[0].elapsed_time(e[1]) for e in evq]
+    for s in sets:
+        if cr.convrot_read_device_status(s["ws"]) != 0:
+            raise RuntimeError(f"{name}: device status not OK")
+    ops = 2.0 * M * N * K
+    q_bytes = 3.0 * M * K + 4.0 * M
+    gq_med, gq_min = med_min(t_q)
+    qi_med, qi_min = med_min(t_q_in)
+    gg_med, gg_min = med_min(t_g_in)
+    hbm = peaks["hbm_gbs"]
+    out = {
+        "M": M, "K": K, "N": N, "g": g, "sets": ns,
+        "layer_us": t_b2b * 1e3, "layer_tops": ops / (t_b2b * 1e-3) / 1e12,
+        "gemm_us_median": gg_med * 1e3, "gemm_us_min": gg_min * 1e3,
+        "gemm_tops_median": ops / (gg_med * 1e-3) / 1e12,
+        "quant_us_median": gq_med * 1e3, "quant_us_min": gq_min * 1e3,
+        "quant_gbs_median": q_bytes / (gq_med * 1e-3) / 1e9, "quant_gbs_best": q_bytes / (gq_min * 1e-3) / 1e9,
+        "quant_frac_hbm_median": q_bytes / (gq_med * 1e-3) / 1e9 / hbm,
+        "quant_in_step_us_median": qi_med * 1e3,
+        "quant_in_step_frac_hbm": q_bytes / (qi_med * 1e-3) / 1e9 / hbm,
+    }
+    if i8_peak:
+        out["gemm_frac_i8_peak_median"] = out["gemm_tops_median"] / i8_peak
+    if M <= 128:
+        # weight-streaming regime: bound by HBM on the algorithmic bytes of the layer
+        gbytes = float(M * K + N * K + 2 * M * N + (2 * N if bias is not None else 0))
+        out["layer_weight_stream_frac_hbm"] = gbytes / (t_b2b * 1e-3) / 1e9 / hbm
+        out["gemm_weight_stream_frac_hbm"] = gbytes / (gg_med * 1e-3) / 1e9 / hbm
+        out["algorithmic_bytes"] = gbytes
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
+def e2e_overlapped(cr, d, X_sets, Wq_sets, sw, bias, g, Y_sets, ws_sets, dev, io_dtype, steps, warmup, barrier,
+                   max_over_ranks, act=None, world=1):
+    """The metric through the public API with host buffers: per step the input is
+    copied from pinned host memory, the layer runs, and its output is copied back
+    to pinned host memory, on three streams ordered by events over the buffer sets."""
+    import torch
+
+    ns = len(X_sets)
+    M, K = X_sets[0].shape
+    N = Wq_sets[0].shape[0]
+    xh = [bits_to_dev(d["x"], "cpu", io_dtype).pin_memory() for _ in range(2)]
+    yh = [torch.empty((M, N), dtype=io_dtype).pin_memory() for _ in range(2)]
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(ns)]
+    ev_run = [torch.cuda.Event() for _ in range(ns)]
+    ev_out = [torch.cuda.Event() for _ in range(ns)]
+    used = [False] * ns
+
+    def step(i):
+        j = i % ns
+        with torch.cuda.stream(s_in):
+            if used[j]:
+                s_in.wait_event(ev_run[j])  # the layer that last read X_j is done
+            X_sets[j].copy_(xh[i % 2], non_blocking=True)
+            ev_in[j].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_in[j])
+            if used[j]:
+                s_run.wait_event(ev_out[j])  # Y_j has been copied out
+            if act is None:
+                cr.convrot_linear(X_sets[j], Wq_sets[j], sw, g, bias, Y=Y_sets[j], ws=ws_sets[j], stream=s_run)
+            else:
+                cr.convrot_linear_ex(X_sets[j], Wq_sets[j], sw, g, bias, act, Y=Y_sets[j], ws=ws_sets[j],
+                                     stream=s_run)
+            ev_run[j].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_run[j])
+            yh[i % 2].copy_(Y_sets[j], non_blocking=True)
+            ev_out[j].record(s_out)
+        used[j] = True
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    s_run.wait_event(t0)
+    s_out.wait_event(t0)
+    for i in range(steps):
+        step(warmup + i)
+    t1.record(s_out)
+    s_out.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_ms = max_over_ranks(t0.elapsed_time(t1))
+    ops = 2.0 * M * N * K
+    return {"value": job_tops(ops, steps, world, t_ms), "unit": UNIT,
+            "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
+            "d2h_bytes_per_step": int(yh[0].numel() * yh[0].element_size()),
+            "steps": steps, "ms_per_step": t_ms / steps,
+            "schedule": f"host-to-device copy, layer and device-to-host copy on three streams, "
+                        f"ordered by events over {ns} buffer sets"}
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -300,8 +581,7 @@ def main():
     act_code = cr.ACT_NONE if args.act == "none" else cr.ACT_GELU_ERF
 
     def to_dev(bits):
-        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-        return t if io_dtype == torch.bfloat16 else t.to(io_dtype)  # the same values in fp16
+        return bits_to_dev(bits, dev, io_dtype)  # fp16: the same values rounded to fp16
 
     W = to_dev(d["w"])
     if variant:
@@ -363,16 +643,16 @@ def main():
     # ---- the layer kernel timed per launch: events recorded around each call on its stream
     launches = L.convrot_linear_launch_count(M, N, K, g)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for pair in ev:
-        for e in pair:
+    for trip in ev:
+        for e in trip:
             e.record(stream)  # creates the underlying cudaEvent_t
     torch.cuda.synchronize(dev)
 
-    def timed_step(i, pair):
+    def timed_step(i, trip):
         s = sets[i % N_SETS]
         st = L.convrot_linear_timed(s["X"].data_ptr(), M, K, g, s["Wq"].data_ptr(), sw_ptr, N, b_ptr,
-                                    s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, pair[0].cuda_event,
-                                    pair[1].cuda_event, pair[2].cuda_event, sp)
+                                    s["Y"].data_ptr(), s["ws"].data_ptr(), ws_bytes, trip[0].cuda_event,
+                                    trip[1].cuda_event, trip[2].cuda_event, sp)
         if st != 0:
             raise cr.ConvRotError(st, "convrot_linear_timed")
 
@@ -388,6 +668,8 @@ def main():
         t_layer = max_over_ranks(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
         t_first = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
         t_second = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+        t_second_med = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in ev))
+        t_second_min = max_over_ranks(min(e[1].elapsed_time(e[2]) for e in ev))
     # (variants: no per-launch events; the GEMM's time is the layer's minus the
     # standalone rotate+quantise kernel's, below)
 
@@ -432,43 +714,30 @@ def main():
         t_second = t_layer - t_q
 
     peaks, peak_src = load_peaks()
-    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    # ---- the int8 tensor pipe's measured peak (the GEMM's roofline denominator)
+    i8 = None
+    if not args.no_peak:
+        i8 = measure_i8_peak(cr, dev, stream, local)
+        i8["burst_tops"] = max_over_ranks(i8["burst_tops"])  # every rank runs it; the figure is per GPU
+    int8_peak = i8["burst_tops"] if i8 else peaks["bf16_tflops"] * INT8_OVER_BF16
+    int8_peak_src = ("measured int8 probe burst (tcgen05.mma.cta_group::2.kind::i8 from shared memory)" if i8 else
+                     f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
+                     "(nominal int8:bf16 dense ratio)")
     layer_tops = ops / (t_layer * 1e-3) / 1e12
     gemm_tops = None if t_g is None else ops / (t_g * 1e-3) / 1e12
     q_bytes = 3.0 * M * K + 4.0 * M
     q_gbs = q_bytes / (t_q * 1e-3) / 1e9
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers (copies overlapped on streams)
     e2e = None
     if not args.no_e2e:
-        xh = [torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16)).view(torch.bfloat16).to(io_dtype)
-              .pin_memory() for _ in range(2)]
-        yh = [torch.empty((M, N), dtype=io_dtype).pin_memory() for _ in range(2)]
-        e2e_steps = max(1, min(args.steps, 200))
-
-        def e2e_step(i):
-            s = sets[i % N_SETS]
-            s["X"].copy_(xh[i % 2], non_blocking=True)
-            if variant:
-                cr.convrot_linear_ex(s["X"], s["Wq"], sw, g, bias, act_code, Y=s["Y"], ws=s["ws"])
-            else:
-                cr.convrot_linear(s["X"], s["Wq"], sw, g, bias, Y=s["Y"], ws=s["ws"])
-            yh[i % 2].copy_(s["Y"], non_blocking=True)
-
-        for i in range(min(args.warmup, 5)):
-            e2e_step(i)
-        torch.cuda.synchronize(dev)
-        barrier()
-        ev0.record(stream)
-        for i in range(e2e_steps):
-            e2e_step(i)
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        t_e2e = max_over_ranks(ev0.elapsed_time(ev1))
-        e2e = {"value": job_tops(ops, e2e_steps, world, t_e2e), "unit": UNIT,
-               "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(yh[0].numel() * 2),
-               "steps": e2e_steps, "ms_per_step": t_e2e / e2e_steps}
+        e2e_steps = max(1, min(args.steps, 100))
+        e2e = e2e_overlapped(cr, d, [s["X"] for s in sets], [s["Wq"] for s in sets], sw, bias, g,
+                             [s["Y"] for s in sets], [s["ws"] for s in sets], dev, io_dtype, e2e_steps,
+                             min(args.warmup, 5), barrier, max_over_ranks,
+                             act=(act_code if variant else None), world=world)
+        if variant:
+            e2e["note"] = "variant layer through convrot_linear_ex"
 
     cpu = None
     parity = None
@@ -476,14 +745,32 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         y_all = sets[(args.steps - 1) % N_SETS]["Y"].float().cpu().numpy().astype(np.float64)
         cpu, parity = cpu_oracle_leg(d, args.cpu_seconds, y_all)
+    del sets
+    torch.cuda.empty_cache()
+
+    # ---- every config of the workload table (device events; rank 0 prints)
+    configs = None
+    if not args.no_configs and not variant:
+        configs = {}
+        up_cache = {}
+        shift = int(time.time() // 60) % len(CONFIG_NAMES)  # rotate the order from run to run
+        order = CONFIG_NAMES[shift:] + CONFIG_NAMES[:shift]
+        for name in order:
+            configs[name] = bench_config(cr, L, name, dev, stream, args.config_reps, peaks,
+                                         i8["burst_tops"] if i8 else None, up_cache)
+        configs = {"order": order, "reps": args.config_reps,
+                   "timing": "CUDA events on the launching stream; median and min over the repetitions; "
+                             "layer_us from back-to-back calls", **configs}
+        del up_cache
 
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    # the dominant kernel: the GEMM (second launch), or the whole layer in the one-launch form
+    # the dominant kernel: the GEMM (second launch)
     t_dom = t_second
     dom_tops = ops / (t_dom * 1e-3) / 1e12
+    hbm = peaks["hbm_gbs"]
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -496,23 +783,31 @@ def main():
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "us_per_launch": t_dom * 1e3,
                      "us_source": ("layer time minus the standalone rotate+quantise kernel" if variant
-                                   else "CUDA events around the GEMM launch inside each step"),
-                     "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
-                                    "(nominal int8:bf16 dense ratio)"},
+                                   else "CUDA events around the GEMM launch inside each step (mean)"),
+                     "peak_source": int8_peak_src,
+                     "peak_context": {"nominal_dense_int8_tops": NOMINAL_INT8_TOPS,
+                                      "bf16_x2_tops": peaks["bf16_tflops"] * INT8_OVER_BF16,
+                                      "bf16_source": peak_src}},
         "layer_us_per_call_events": t_layer * 1e3,
         "kernels": {
             "rotate_quant_kernel (first launch of the step, events)": {
                 "us": t_first * 1e3, "bound": "hbm", "achieved": q_bytes / (t_first * 1e-3) / 1e9, "unit": "GB/s",
-                "peak": peaks["hbm_gbs"], "frac": q_bytes / (t_first * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                "peak": hbm, "frac": q_bytes / (t_first * 1e-3) / 1e9 / hbm},
             "rotate_quant_kernel (standalone, timed alone)": {
-                "us": t_q * 1e3, "bound": "hbm", "achieved": q_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"],
-                "frac": q_gbs / peaks["hbm_gbs"], "algorithmic_bytes": q_bytes},
+                "us": t_q * 1e3, "bound": "hbm", "achieved": q_gbs, "unit": "GB/s", "peak": hbm,
+                "frac": q_gbs / hbm, "algorithmic_bytes": q_bytes},
         },
+        "hbm_peak_source": f"{peak_src} copy bandwidth {hbm} GB/s",
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
     }
+    if not variant:
+        out["roofline"]["us_per_launch_median"] = t_second_med * 1e3
+        out["roofline"]["us_per_launch_min"] = t_second_min * 1e3
+    if i8:
+        out["int8_peak"] = i8
     if M <= SMALL_M:
         # the weight-streaming GEMM (tokens as the MMA's N side): bound by HBM on the
         # weight bytes; algorithmic bytes M*K + N*K + 2*M*N (+ 2*N bias) per launch
@@ -520,9 +815,9 @@ def main():
         gbs = gbytes / (t_dom * 1e-3) / 1e9
         out["roofline"].update({
             "bound": "hbm", "kernel": "gemm_i8_smallm_kernel (swap-AB tcgen05 kind::i8, weight streaming)",
-            "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
             "algorithmic_bytes": gbytes, "traffic": None,
-            "peak_source": f"{peak_src} HBM copy bandwidth {peaks['hbm_gbs']} GB/s"})
+            "peak_source": f"{peak_src} HBM copy bandwidth {hbm} GB/s"})
     if variant:  # no per-launch events in a variant run: only the standalone timing is real
         del out["kernels"]["rotate_quant_kernel (first launch of the step, events)"]
     if t_g is not None:
@@ -531,6 +826,8 @@ def main():
             "frac": gemm_tops / int8_peak, "ops": ops}
     if variant:
         out["config"]["variant"] = {"io_dtype": args.dtype, "weight_scale": args.wscale, "activation": args.act}
+    if configs is not None:
+        out["configs"] = configs
     if parity is not None:
         out["parity_nrmse_vs_oracle_sample"] = parity
     print(json.dumps(out), flush=True)

@@ -313,6 +313,22 @@ CONVROT_API convrot_status convrot_linear_noalloc(const void* X, int64_t M, int6
 CONVROT_API convrot_status convrot_read_device_status(const void* ws, convrot_stream_t stream);
 
 /*
+ * convrot_probe_i8_peak -- measurement aid for the GEMM's roofline (not part
+ * of the layer): launches one CTA pair per two SMs, each issuing `iters`
+ * times four tcgen05.mma.cta_group::2.kind::i8 instructions (M = 256, N = 256,
+ * K = 32: the instruction the layer's GEMM uses) on zeroed shared-memory
+ * operands, with no global memory traffic. The caller times the launch with
+ * events on `stream`; the work is 2 * 256 * 256 * 128 * iters operations per
+ * pair, convrot_probe_i8_peak_ctas() / 2 pairs. iters in [1, 2^20]. `ws`
+ * (>= 256 bytes, 256-byte aligned) receives the status word
+ * (CONVROT_ERR_DEVICE_TIMEOUT if the final wait ran out).
+ */
+CONVROT_API convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t ws_bytes,
+                                                 convrot_stream_t stream);
+/* CTAs that convrot_probe_i8_peak launches on the current device (0 on error). */
+CONVROT_API int convrot_probe_i8_peak_ctas(void);
+
+/*
  * convrot_test_wait_timeout -- exercises the bounded device wait: launches one
  * CTA that waits on a barrier nothing will complete, for at most timeout_ns
  * nanoseconds (1e3 .. 1e9), then records CONVROT_ERR_DEVICE_TIMEOUT in the

@@ -37,6 +37,7 @@ __all__ = [
     "convrot_gemm_s32",
     "convrot_read_device_status",
     "convrot_test_wait_timeout",
+    "convrot_probe_i8_peak",
     "ConvRotLinear",
     "lib",
 ]
@@ -341,6 +342,19 @@ def convrot_read_device_status(ws, stream=None) -> int:
 def convrot_test_wait_timeout(ws, timeout_ns: int, stream=None) -> None:
     _check(lib().convrot_test_wait_timeout(_ptr(ws), ws.numel(), int(timeout_ns), _stream_ptr(stream)),
            "convrot_test_wait_timeout")
+
+
+def convrot_probe_i8_peak(iters: int, ws=None, stream=None) -> int:
+    """Enqueue the int8 tensor-pipe peak probe (one CTA pair per two SMs, `iters` x 4
+    tcgen05.mma.cta_group::2.kind::i8 of 256x256x32 each, no global traffic); returns
+    the number of CTAs launched. The caller times it with events on `stream`."""
+    import torch
+
+    L = lib()
+    if ws is None:
+        ws = torch.empty((256,), dtype=torch.uint8, device=torch.cuda.current_device())
+    _check(L.convrot_probe_i8_peak(int(iters), _ptr(ws), ws.numel(), _stream_ptr(stream)), "convrot_probe_i8_peak")
+    return int(L.convrot_probe_i8_peak_ctas())
 
 
 class ConvRotLinear:

@@ -46,6 +46,8 @@ SIGNATURES = {
                                       _c_void_p, _c_void_p, _c_void_p]),
     "convrot_read_device_status": (_int, [_c_void_p, _c_void_p]),
     "convrot_test_wait_timeout": (_int, [_c_void_p, _size, _i64, _c_void_p]),
+    "convrot_probe_i8_peak": (_int, [_i64, _c_void_p, _size, _c_void_p]),
+    "convrot_probe_i8_peak_ctas": (_int, []),
 }
 
 _lib = None

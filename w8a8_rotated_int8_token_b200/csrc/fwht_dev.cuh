@@ -31,6 +31,54 @@ __device__ __forceinline__ void fwht_pair_stage(float2 (&p)[4][8]) {
   }
 }
 
+// The stage on the top piece bit taken first, straight from the input words:
+// with a from piece jj and b from piece jj+4 (two elements per 32-bit word),
+// lo = (a0 + b0, a0 - b0) and hi = (a1 + b1, a1 - b1). Only b is widened to
+// float32; a enters the sm_100 mixed-precision add/sub as a 16-bit operand
+// (exact), so each sum or difference is one float32 rounding, as after an
+// explicit widening, at one instruction less per butterfly.
+template <bool F16IN>
+__device__ __forceinline__ void fwht_first_pair(uint32_t wa, float2 b, float2& lo, float2& hi) {
+  if (F16IN) {
+    asm("{\n\t.reg .b16 a0, a1;\n\tmov.b32 {a0, a1}, %4;\n\t"
+        "add.rn.f32.f16 %0, a0, %5;\n\tsub.rn.f32.f16 %1, a0, %5;\n\t"
+        "add.rn.f32.f16 %2, a1, %6;\n\tsub.rn.f32.f16 %3, a1, %6;\n\t}"
+        : "=f"(lo.x), "=f"(lo.y), "=f"(hi.x), "=f"(hi.y)
+        : "r"(wa), "f"(b.x), "f"(b.y));
+  } else {
+    asm("{\n\t.reg .b16 a0, a1;\n\tmov.b32 {a0, a1}, %4;\n\t"
+        "add.rn.f32.bf16 %0, a0, %5;\n\tsub.rn.f32.bf16 %1, a0, %5;\n\t"
+        "add.rn.f32.bf16 %2, a1, %6;\n\tsub.rn.f32.bf16 %3, a1, %6;\n\t}"
+        : "=f"(lo.x), "=f"(lo.y), "=f"(hi.x), "=f"(hi.y)
+        : "r"(wa), "f"(b.x), "f"(b.y));
+  }
+}
+
+// max(a, b, c) in one sm_100 three-input instruction.
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max |value| of a lane's 64 values: |.| folded into 32 two-input maxima,
+// then a tree of three-input maxima (48 instructions, five dependent steps).
+__device__ __forceinline__ float absmax64_v3(const float2 (&w)[4][8]) {
+  float a[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 x = w[i >> 3][i & 7];
+    a[i] = fmaxf(fabsf(x.x), fabsf(x.y));
+  }
+  float b[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) b[i] = fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[10] = fmaxf(a[30], a[31]);
+  const float c0 = fmax3f(b[0], b[1], b[2]), c1 = fmax3f(b[3], b[4], b[5]), c2 = fmax3f(b[6], b[7], b[8]);
+  const float c3 = fmaxf(b[9], b[10]);
+  return fmaxf(fmax3f(c0, c1, c2), c3);
+}
+
 // The five packed stages on the index bits a lane holds apart from the top
 // piece bit: p[jj][e] holds the elements of pieces jj (.x) and jj+4 (.y) at
 // in-piece position e; the stages run on e (1, 2, 4) and jj (1, 2) as f32x2.
@@ -196,6 +244,38 @@ __device__ __forceinline__ QuantScale make_scale(float amax_u) {
     q.ci = cg * (1.0f / (q.s * 0x1p64f));
   }
   return q;
+}
+
+// The stored scale of a row (or tensor): float32(absmax(X R) / 127) =
+// absmax_u / (127 sqrt(g)), one correctly rounded division (for g = 256 the
+// divisor 2032 is exact; for g = 128 it is the nearest float to 127 sqrt(128)).
+template <int G>
+__device__ __forceinline__ float scale_of(float amax_u) {
+  const float div = (G == 256) ? 2032.0f : 1436.8409423828125f;
+  return amax_u / div;
+}
+
+// The factor that maps an unnormalised value u to code units:
+// code = rne(u * ci) with ci = 127 / absmax_u, the same quotient as u / (sqrt(g) s)
+// up to float32 rounding (which can move a code only at a near-tie). The row
+// maximum maps to 127 * (1 +- 2^-22), so no code leaves [-127, 127].
+struct CodeFactor {
+  float ci;   // 0 for an all-zero row
+  float pre;  // 1, or 2^64 for rows whose absmax is below 2^-90
+};
+
+__device__ __forceinline__ CodeFactor code_factor(float amax_u) {
+  CodeFactor c;
+  c.pre = 1.0f;
+  if (amax_u == 0.0f) {
+    c.ci = 0.0f;
+  } else if (amax_u >= 0x1p-90f) {
+    c.ci = 127.0f * __frcp_rn(amax_u);
+  } else {  // tiny row: lift by 2^64 (exact) so that the reciprocal cannot overflow
+    c.pre = 0x1p64f;
+    c.ci = 127.0f * __frcp_rn(amax_u * 0x1p64f);
+  }
+  return c;
 }
 
 // Four codes from four magic-rounded floats: the low byte of (u*ci + 1.5*2^23)

@@ -1,0 +1,103 @@
+// Measured peak of the int8 tensor pipe: the same instruction the layer's GEMM
+// issues (tcgen05.mma.cta_group::2.kind::i8, M = 256, N = 256, K = 32 per
+// instruction, both operands from shared memory) in a loop with no global
+// memory traffic, so that a timed launch gives the rate the tensor cores
+// sustain on this GPU at its current clock. It is a measurement aid for the
+// roofline of the GEMM; it computes nothing of the layer.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "convrot.h"
+#include "ptx_sm100.cuh"
+
+namespace convrot {
+
+namespace {
+
+constexpr int kProbeTile = 128 * 128;  // bytes of this CTA's A (and of its B) operand tile
+constexpr int kProbeThreads = 128;
+constexpr int kTimeoutStatus = 5;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
+    i8_peak_pair_kernel(int64_t iters, int* status, uint64_t timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t done;
+  __shared__ uint32_t tmem_ptr;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool leader = cluster_ctarank() == 0;
+
+  // zero operands (their values do not change the rate); the tensor cores read
+  // them through the async proxy
+  for (int i = threadIdx.x; i < 2 * kProbeTile / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    mbar_init(&done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_ptr, 256);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_ptr;
+
+  if (warp == 1 && lane == 0 && leader) {
+    const uint32_t a_base = smem_addr(smem);
+    const uint32_t b_base = smem_addr(smem + kProbeTile);
+    constexpr uint32_t idesc = idesc_i8(256, 256);
+    for (int64_t i = 0; i < iters; ++i) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_i8_pair(tmem_base, smem_desc_k_sw128(a_base + k * 32), smem_desc_k_sw128(b_base + k * 32), idesc,
+                    (i | k) != 0 ? 1u : 0u);
+    }
+    mma_commit_pair_mc(&done, 0x3);  // both CTAs learn that every MMA has finished
+  }
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&done, 0u, nullptr, timeout_ns)) atomicOr(status, kTimeoutStatus);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 256);
+}
+
+}  // namespace
+
+}  // namespace convrot
+
+extern "C" {
+
+convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  // at most 2^20 x 512 tensor cycles (about 0.3 s at 1.9 GHz): well inside the 2 s bound of the final wait
+  if (iters < 1 || iters > (int64_t(1) << 20)) return CONVROT_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % 256) != 0 || ws_bytes < 256) return CONVROT_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  const int smem = 2 * convrot::kProbeTile + 1024;
+  if (cudaFuncSetAttribute(convrot::i8_peak_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
+  // one CTA pair per two SMs, every SM busy
+  convrot::i8_peak_pair_kernel<<<(sms / 2) * 2, convrot::kProbeThreads, smem, s>>>(iters, status,
+                                                                                    2000000000ull);
+  return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+int convrot_probe_i8_peak_ctas(void) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return (sms / 2) * 2;
+}
+
+}  // extern "C"

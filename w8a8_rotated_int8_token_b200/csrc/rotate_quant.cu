@@ -55,19 +55,30 @@ __device__ __forceinline__ float2 widen2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+#ifndef CONVROT_RQ_MAXNREG
+#define CONVROT_RQ_MAXNREG 112
+#endif
+
+// register cap: g = 128 keeps its lane-pair shuffles' operands live longer
+template <int G>
+constexpr int rq_maxnreg() { return G == 256 ? CONVROT_RQ_MAXNREG : 128; }
+
 template <int G, int MODE, bool F16IN>
-__global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
+__global__ void __maxnreg__(rq_maxnreg<G>()) rotate_quant_kernel(RotQuantParams p) {
   constexpr int LG = G / 64;
   constexpr int PIECE = G / 8;  // elements between consecutive pieces of a lane
-  // kRqStages input slots of rows_per_cta x K bf16, each rounded up to whole
-  // 4 KB warp regions (g = 256 reuses a warp's region for its exchange)
+  constexpr int S = kRqStages;
+  // S input slots of rows_per_cta x K bf16, each rounded up to whole 4 KB
+  // warp regions (g = 256 reuses a warp's region for its exchange)
   extern __shared__ __align__(128) uint8_t stage_mem[];
-  __shared__ uint64_t full[kRqStages];
+  __shared__ uint64_t full[S];
   __shared__ unsigned row_max[3][kMaxRowsPerCta];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
   const int rpc = p.rows_per_cta;
+  const int K = static_cast<int>(p.K);
+  const int rows = static_cast<int>(p.rows);
   const int row_in_cta = tid / p.threads_per_row;  // >= rpc for the padding threads of the last warp
   const int t = tid - row_in_cta * p.threads_per_row;
   const int grp = t / LG;
@@ -76,14 +87,15 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   // Group k reads its pieces in the order j ^ (k mod F), F = 2 (g=256) or 4
   // (g=128), so that the F groups sharing a 128-byte bank window hit
   // different banks. The transform then comes out with piece r multiplied by
-  // (-1)^popcount(r & flip), which the quantisation multiplier undoes.
+  // (-1)^popcount(r & flip), which the quantisation multiplier undoes. The
+  // flip never changes the top piece bit, so pieces jj and jj+4 still pair.
   constexpr int F = (G == 256) ? 2 : 4;
   const int flip = grp & (F - 1);
-  const int64_t nblocks = (p.rows + rpc - 1) / rpc;
+  const int nblocks = (rows + rpc - 1) / rpc;
   const uint32_t stage_bytes = rotquant_slot_bytes(rpc, p.K);
 
   if (tid == 0) {
-    for (int s = 0; s < kRqStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -92,47 +104,49 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   // The input may be the previous kernel's output: wait for it (launches are
   // programmatic), then let the next kernel start its prologue early.
   griddep_wait();
-  griddep_launch_dependents();
   if (MODE == kRqActivation && p.status_reset != nullptr && blockIdx.x == 0 && tid == 0) *p.status_reset = 0;
+  griddep_launch_dependents();
 
-  // The producer (thread 0) loads row block it+1 as soon as block it has
-  // landed, so one block per CTA is in flight while the CTA computes: with a
-  // few CTAs per SM that covers the memory latency, and the first block of
-  // every CTA is not held up behind the later ones.
-  int64_t issued = 0;
-  auto issue = [&](int64_t it) {
-    const int64_t blk = blockIdx.x + it * gridDim.x;
+  // The producer (thread 0) keeps S-1 row blocks of this CTA in flight: block
+  // it+S-1 goes out as soon as block it has landed, into the slot that block
+  // it-1 released at its barrier.
+  int issued = 0;
+  auto issue = [&](int it) {
+    const int blk = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
     if (blk >= nblocks) return;
-    const int64_t r0 = blk * rpc;
-    const int64_t nrows = (p.rows - r0) < rpc ? (p.rows - r0) : rpc;
-    const uint32_t row_bytes = static_cast<uint32_t>(p.K) * 2u;
+    const int r0 = blk * rpc;
+    const int nrows = (rows - r0) < rpc ? (rows - r0) : rpc;
+    const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
     const uint32_t bytes = static_cast<uint32_t>(nrows) * row_bytes;
-    const int slot = static_cast<int>(it % kRqStages);
+    const int slot = it % S;
     uint8_t* const dst = stage_mem + static_cast<size_t>(slot) * stage_bytes;
     mbar_arrive_expect_tx(&full[slot], bytes);
     if (p.ldx == 0 || p.ldx == p.K) {  // dense rows: one copy for the block
-      bulk_load(dst, p.src + r0 * p.K, bytes, &full[slot]);
+      bulk_load(dst, p.src + static_cast<int64_t>(r0) * K, bytes, &full[slot]);
     } else {  // strided rows: one copy per row, packed densely in the slot
-      for (int64_t r = 0; r < nrows; ++r)
-        bulk_load(dst + r * row_bytes, p.src + (r0 + r) * p.ldx, row_bytes, &full[slot]);
+      for (int r = 0; r < nrows; ++r)
+        bulk_load(dst + r * row_bytes, p.src + static_cast<int64_t>(r0 + r) * p.ldx, row_bytes, &full[slot]);
     }
     issued = it + 1;
   };
-  static_assert(kRqStages >= 2, "the block after the current one needs its own slot");
-  if (tid == 0) issue(0);
+  static_assert(S >= 2, "the block after the current one needs its own slot");
+  if (tid == 0)
+    for (int i = 0; i < S - 1; ++i) issue(i);
 
   // byte offset of the lane's first piece inside a slot (loop-invariant)
-  const uint32_t lane_off =
-      (static_cast<uint32_t>(row_in_cta) * static_cast<uint32_t>(p.K) + static_cast<uint32_t>(grp * G + 8 * l)) * 2u;
+  const uint32_t lane_off = (static_cast<uint32_t>(row_in_cta) * static_cast<uint32_t>(K) +
+                             static_cast<uint32_t>(grp * G + 8 * l)) * 2u;
+  // the g = 256 exchange region of this warp inside a slot
+  const uint32_t xoff = static_cast<uint32_t>(tid >> 5) * kX256RegionBytes;
 
-  int64_t it = 0;
+  int it = 0;
   int slot = 0;
   uint32_t ph = 0;
   int rsel = 0;  // which of the three row-maximum buffers this block uses
   bool timed_out = false;
-  for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x, ++it) {
-    const int64_t row = blk * rpc + row_in_cta;
-    const bool valid = lane_active && row < p.rows;
+  for (int blk = blockIdx.x; blk < nblocks; blk += gridDim.x, ++it) {
+    const int row = blk * rpc + row_in_cta;
+    const bool valid = lane_active && row < rows;
     // Row maxima rotate over three buffers: this block's, the next block's
     // (cleared now, before this block's barrier), and the previous block's,
     // which slower threads may still be reading.
@@ -141,12 +155,13 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
     if (tid < rpc) row_max[rnext][tid] = 0u;
 
     const bool ok = mbar_wait_bounded(&full[slot], ph, &abort_flag, p.timeout_ns);
-    // the slot of block it+1 was released by the barrier of block it-1
-    if (tid == 0 && ok) issue(it + 1);
+    // the slot of block it+S-1 was released by the barrier of block it-1
+    if (tid == 0 && ok) issue(it + S - 1);
     uint8_t* slot_mem = stage_mem + static_cast<size_t>(slot) * stage_bytes;
     // Every lane loads, also those of rows past the end or of padding
     // threads: their bytes lie inside the slot (stale but harmless) and only
-    // their stores are skipped.
+    // their stores are skipped. The stage on the top piece bit is taken
+    // straight from the input words.
     float2 v[4][8];
     {
       const uint8_t* src = slot_mem + lane_off;
@@ -157,28 +172,20 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 fa = widen2<F16IN>(aw[q]), fb = widen2<F16IN>(bw[q]);
-          v[jj][2 * q] = make_float2(fa.x, fb.x);
-          v[jj][2 * q + 1] = make_float2(fa.y, fb.y);
-        }
+        for (int q = 0; q < 4; ++q) fwht_first_pair<F16IN>(aw[q], widen2<F16IN>(bw[q]), v[jj][2 * q], v[jj][2 * q + 1]);
       }
     }
-    if (++slot == kRqStages) {
+    if (++slot == S) {
       slot = 0;
       ph ^= 1u;
     }
     rsel = rnext;
 
-    // transform; afterwards w holds the lane's values (layout per g below)
+    // the other stages; afterwards w holds the lane's values (layout per g below)
     float2 w[4][8];
-    // packed stages first, then the scalar one on the top piece bit: its
-    // results go straight to the 16-byte exchange stores (or the shuffles)
-    // without being re-paired
     fwht_lane_local(v);
-    fwht_pair_stage(v);
     if constexpr (G == 256) {
-      fwht256_exchange(v, w, slot_mem + static_cast<size_t>(tid >> 5) * kX256RegionBytes, (tid & 31) >> 2, l);
+      fwht256_exchange(v, w, slot_mem + xoff, (tid & 31) >> 2, l);
       // the slot is refilled by an asynchronous copy after the barrier below
       fence_proxy_async_smem();
       fwht256_after_exchange(w);
@@ -189,7 +196,7 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[jj][e] = v[jj][e];
     }
-    float m = absmax64(w);
+    float m = absmax64_v3(w);
 #pragma unroll
     for (int s = 1; s < LG; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
     // non-negative floats order like their bit patterns
@@ -208,27 +215,28 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
     }
     const float amax_u =
         (MODE == kRqActivation) ? __uint_as_float(rmax[row_in_cta]) : __uint_as_float(*p.tensor_absmax);
-    const QuantScale qs = make_scale<G>(amax_u);
+    // the stored scale, one correctly rounded division, by the one thread that stores it
     if (MODE == kRqActivation) {
-      if (valid && t == 0) p.scale[row] = qs.s;
+      if (valid && t == 0) p.scale[row] = scale_of<G>(amax_u);
     } else {
-      if (blk == 0 && tid == 0) *p.scale = qs.s;
+      if (blk == 0 && tid == 0) *p.scale = scale_of<G>(amax_u);
     }
     if (!valid) continue;
-    if (qs.pre != 1.0f) {  // tiny row: multiply by 2^64 first (exact), then by ci
-      const float2 pre2 = make_float2(qs.pre, qs.pre);
+    const CodeFactor cf = code_factor(amax_u);
+    if (cf.pre != 1.0f) {  // tiny row: multiply by 2^64 first (exact), then by ci
+      const float2 pre2 = make_float2(cf.pre, cf.pre);
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[jj][e] = __fmul2_rn(w[jj][e], pre2);
     }
     const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
-    int8_t* dst = p.dst + row * p.K + static_cast<int64_t>(grp) * G;
+    int8_t* dst = p.dst + static_cast<int64_t>(row) * K + grp * G;
     if constexpr (G == 256) {
       // the lane holds elements 32*l + (0..31) (.x) and 128 + 32*l + (0..31)
       // (.y), in the order w[src][e] = element 8*src + e of the run; the
       // piece-order flip left them multiplied by (-1)^(flip & l)
-      const float ci = (flip & l & 1) ? -qs.ci : qs.ci;
+      const float ci = (flip & l & 1) ? -cf.ci : cf.ci;
       const float2 ci2 = make_float2(ci, ci);
       uint32_t lo[8], hi[8];
 #pragma unroll
@@ -250,7 +258,7 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
       int8_t* d8 = dst + 8 * l;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
-        const float cij = (__popc(jj & flip) & 1) ? -qs.ci : qs.ci;
+        const float cij = (__popc(jj & flip) & 1) ? -cf.ci : cf.ci;
         const float2 ci2 = make_float2(cij, cij);
         float2 r[8];
 #pragma unroll
@@ -269,8 +277,8 @@ __global__ void __maxnreg__(112) rotate_quant_kernel(RotQuantParams p) {
   if (timed_out && tid == 0) {
     if (p.status != nullptr) atomicOr(p.status, kRqTimeoutStatus);
     // let the copies already issued land before the shared memory goes away
-    for (int64_t k = it; k < issued; ++k)
-      mbar_wait_bounded(&full[k % kRqStages], static_cast<uint32_t>((k / kRqStages) & 1), nullptr, p.timeout_ns);
+    for (int k = it; k < issued; ++k)
+      mbar_wait_bounded(&full[k % S], static_cast<uint32_t>((k / S) & 1), nullptr, p.timeout_ns);
   }
 }
 

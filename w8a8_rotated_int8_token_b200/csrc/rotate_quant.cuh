@@ -14,7 +14,10 @@ enum RotQuantMode : int {
 };
 
 constexpr int kMaxRowsPerCta = 256;
-constexpr int kRqStages = 2;          // input slots per CTA: the block computed and the next one
+#ifndef CONVROT_RQ_SLOTS
+#define CONVROT_RQ_SLOTS 2
+#endif
+constexpr int kRqStages = CONVROT_RQ_SLOTS;  // input slots per CTA: the block computed and the ones in flight
 constexpr int kRqTimeoutStatus = 5;   // CONVROT_ERR_DEVICE_TIMEOUT
 constexpr int kRotQuantMaxThreads = 512;  // K/64 threads per row: K <= 32768
 
