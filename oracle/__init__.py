@@ -4,6 +4,13 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package; the library never does.
 """
 
+from .attention_oracle import (  # noqa: F401
+    attention_exact,
+    attention_int8,
+    attention_logits,
+    quantize_heads,
+    softmax,
+)
 from .convrot_oracle import (  # noqa: F401
     QMAX,
     bf16_to_f64,

@@ -41,6 +41,37 @@ MUTATIONS = {
 }
 
 
+# mistakes planted in the attention oracle, caught by its own pins
+MUTATIONS_ATTENTION = {
+    "softmax_scale_dropped": ("        * np.float64(softmax_scale)", "        * 1.0"),
+    "keys_not_rotated": ("    kc, sk = quantize_heads(k, g)", "    kc, sk = quantize_per_token(np.asarray(k, np.float64))"),
+    "softmax_over_queries": ("    m = np.max(s, axis=-1, keepdims=True)\n    e = np.exp(s - m)\n    return e / np.sum(e, axis=-1, keepdims=True)",
+                             "    m = np.max(s, axis=-2, keepdims=True)\n    e = np.exp(s - m)\n    return e / np.sum(e, axis=-2, keepdims=True)"),
+    "probabilities_not_normalised": ("    return e / np.sum(e, axis=-1, keepdims=True)", "    return e"),
+    "key_scale_dropped": ("np.asarray(sk, np.float64)[..., None, :]) \\", "1.0) \\"),
+}
+
+
+def _run_mutated(tmp_path, file_name, old, new, test_file):
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__"))
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), tmp_path / "pytest.ini")
+    path = tmp_path / "oracle" / file_name
+    src = path.read_text()
+    assert old in src, "mutation target not found: the oracle changed, update this table"
+    path.write_text(src.replace(old, new))
+    return subprocess.run([sys.executable, "-m", "pytest", test_file, "-q", "-x"],
+                          cwd=tmp_path, capture_output=True, text=True, timeout=300)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS_ATTENTION))
+def test_attention_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTATIONS_ATTENTION[name]
+    r = _run_mutated(tmp_path, "attention_oracle.py", old, new, "tests/test_oracle_attention.py")
+    assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(name, tmp_path):
     old, new = MUTATIONS[name]
