@@ -328,7 +328,7 @@ def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, su
     torch.cuda.synchronize(dev)
     burst = []
     with ClockSampler(clock_index, 0.001) as clk_b:
-        for _ in range(5):
+        for _ in range(10):
             e0.record(stream)
             cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
             e1.record(stream)
@@ -345,13 +345,14 @@ def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, su
     if cr.convrot_read_device_status(ws) != 0:
         raise RuntimeError("int8 peak probe: a device wait timed out")
     b, s = clk_b.summary(), clk_s.summary()
-    return {"burst_tops": max(burst), "burst_tops_median": statistics.median(burst), "sustained_tops": sustained,
+    return {"peak_tops": max(max(burst), sustained),
+            "burst_tops": max(burst), "burst_tops_median": statistics.median(burst), "sustained_tops": sustained,
             "burst_clock_mhz": b["sm_mhz"], "sustained_clock_mhz": s["sm_mhz"],
             "reasons": sorted(set(b["reasons"]) | set(s["reasons"])),
             "ops_per_clk_per_sm_burst": (max(burst) * 1e12 / (b["sm_mhz"] * 1e6) / ctas) if b["sm_mhz"] else None,
             "probe": f"{pairs} CTA pairs x {iters} x 4 tcgen05.mma.cta_group::2.kind::i8 (256x256x32), "
-                     f"operands in shared memory, no global traffic; burst = best of 5 launches of ~{burst_ms:g} ms, "
-                     f"sustained = {n_sus} launches back to back",
+                     f"operands in shared memory, no global traffic; burst = best of 10 launches of ~{burst_ms:g} ms, "
+                     f"sustained = {n_sus} launches back to back; peak = the larger of the two",
             "context": {"nominal_dense_int8_tops": NOMINAL_INT8_TOPS}}
 
 
@@ -469,6 +470,59 @@ def bench_config(cr, L, name: str, dev, stream, reps: int, peaks: dict, i8_peak,
         out["layer_weight_stream_frac_hbm"] = gbytes / (t_b2b * 1e-3) / 1e9 / hbm
         out["gemm_weight_stream_frac_hbm"] = gbytes / (gg_med * 1e-3) / 1e9 / hbm
         out["algorithmic_bytes"] = gbytes
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
+SFU_EX2_PER_CLK_PER_SM = 16  # special-function unit throughput of exp2 per SM per clock (B200)
+
+
+def bench_attention(cr, dev, stream, reps: int, clock_index: int, i8_peak) -> dict:
+    """INT8 attention at the pages' shape: 4096 image + 128 prefix tokens, 32 heads, head dim 128."""
+    import torch
+
+    BH, S, D = 32, 4224, 128
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    ns = 4  # 4 x (Q, K, V, O) = 553 MB: no call finds its inputs in L2
+    sets = []
+    for _ in range(ns):
+        q, k, v = (torch.randn((BH, S, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(3))
+        ws = torch.empty((cr.convrot_attention_workspace_bytes(BH, S, S, D),), dtype=torch.uint8, device=dev)
+        sets.append((q, k, v, torch.empty_like(q), ws))
+
+    def call(i):
+        q, k, v, o, ws = sets[i % ns]
+        cr.convrot_attention_int8(q, k, v, O=o, ws=ws, stream=stream)
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(clock_index, 0.002) as clk:
+        e0.record(stream)
+        for i in range(reps):
+            call(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    t_ms = e0.elapsed_time(e1) / reps
+    for s in sets:
+        if cr.convrot_read_device_status(s[4]) != 0:
+            raise RuntimeError("attention: device status not OK")
+    ops = 4.0 * S * S * D * BH  # Q K^T and P V
+    exps = float(S) * S * BH
+    c = clk.summary()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965
+    sfu_peak = SFU_EX2_PER_CLK_PER_SM * sms * mhz * 1e6
+    out = {"BH": BH, "S": S, "D": D, "call_us": t_ms * 1e3, "tops": ops / (t_ms * 1e-3) / 1e12,
+           "bound": "alu", "exp2_per_s": exps / (t_ms * 1e-3), "exp2_peak_per_s": sfu_peak,
+           "frac_exp2_peak": exps / (t_ms * 1e-3) / sfu_peak, "clock_mhz": c["sm_mhz"],
+           "note": "one call = rotate+quantise of Q and of K, transposition of V, the attention kernel; "
+                   "exp2 peak = 16 per SM per clock at the sampled SM clock"}
+    if i8_peak:
+        out["tensor_floor_us"] = (2.0 * S * S * D * BH / i8_peak + 2.0 * S * S * D * BH / (i8_peak / 2.0)) / 1e6
     del sets
     torch.cuda.empty_cache()
     return out
@@ -718,9 +772,10 @@ def main():
     i8 = None
     if not args.no_peak:
         i8 = measure_i8_peak(cr, dev, stream, local)
-        i8["burst_tops"] = max_over_ranks(i8["burst_tops"])  # every rank runs it; the figure is per GPU
-    int8_peak = i8["burst_tops"] if i8 else peaks["bf16_tflops"] * INT8_OVER_BF16
-    int8_peak_src = ("measured int8 probe burst (tcgen05.mma.cta_group::2.kind::i8 from shared memory)" if i8 else
+        i8["peak_tops"] = max_over_ranks(i8["peak_tops"])  # every rank runs it; the figure is per GPU
+    int8_peak = i8["peak_tops"] if i8 else peaks["bf16_tflops"] * INT8_OVER_BF16
+    int8_peak_src = ("measured int8 probe (tcgen05.mma.cta_group::2.kind::i8 from shared memory; the larger of "
+                     "its burst and sustained rates)" if i8 else
                      f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
                      "(nominal int8:bf16 dense ratio)")
     layer_tops = ops / (t_layer * 1e-3) / 1e12
@@ -757,7 +812,9 @@ def main():
         order = CONFIG_NAMES[shift:] + CONFIG_NAMES[:shift]
         for name in order:
             configs[name] = bench_config(cr, L, name, dev, stream, args.config_reps, peaks,
-                                         i8["burst_tops"] if i8 else None, up_cache)
+                                         i8["peak_tops"] if i8 else None, up_cache)
+        configs["attention_int8_4224"] = bench_attention(cr, dev, stream, args.config_reps, local,
+                                                         i8["peak_tops"] if i8 else None)
         configs = {"order": order, "reps": args.config_reps,
                    "timing": "CUDA events on the launching stream; median and min over the repetitions; "
                              "layer_us from back-to-back calls", **configs}

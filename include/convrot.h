@@ -313,6 +313,32 @@ CONVROT_API convrot_status convrot_linear_noalloc(const void* X, int64_t M, int6
 CONVROT_API convrot_status convrot_read_device_status(const void* ws, convrot_stream_t stream);
 
 /*
+ * convrot_attention_int8 -- INT8 attention, O = softmax(S) V per (batch*head):
+ *   S[i, j] = (Qq[i] . Kq[j]) * s_q[i] * s_k[j] * softmax_scale, where Qq/Kq are
+ *   the per-token int8 codes of the head vectors of Q and K after the
+ *   normalised Walsh-Hadamard rotation along the head dimension (the same
+ *   rotate + quantise as convrot_quant_act with g = D), the integer dot products
+ *   exact; softmax over the keys in float32; P rounded to bf16 and P V
+ *   accumulated in float32; O rounded to bf16.
+ *   The Hugging Face discussion "INT8 ConvRot on 2xT4" (section "Attention
+ *   kernel alone") measures INT8 attention at 4096 + 128 tokens, 32 heads,
+ *   head dimension 128 against FP32 attention; the pages do not give the
+ *   quantisation scheme, which this entry point fixes as above.
+ *   Q [BH, Sq, D], K and V [BH, Skv, D], O [BH, Sq, D]: bf16, row-major (D
+ *   contiguous), device pointers, 16-byte aligned; BH = batch * heads
+ *   (<= 65535). D must be 128 (else CONVROT_ERR_UNSUPPORTED). Skv >= 1;
+ *   Sq = 0 or BH = 0 enqueues nothing. softmax_scale > 0 and finite (usually
+ *   1/sqrt(D)). ws: >= convrot_attention_workspace_bytes(BH, Sq, Skv, D),
+ *   256-byte aligned; its first word is the status word
+ *   (convrot_read_device_status). Launches a 4-byte memset and four kernels
+ *   (rotate+quantise of Q and of K, a transposition of V, the attention kernel).
+ */
+CONVROT_API size_t convrot_attention_workspace_bytes(int64_t BH, int64_t Sq, int64_t Skv, int64_t D);
+CONVROT_API convrot_status convrot_attention_int8(const void* Q, const void* K, const void* V, int64_t BH,
+                                                  int64_t Sq, int64_t Skv, int64_t D, float softmax_scale,
+                                                  void* O, void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
  * convrot_probe_i8_peak -- measurement aid for the GEMM's roofline (not part
  * of the layer): launches one CTA pair per two SMs, each issuing `iters`
  * times four tcgen05.mma.cta_group::2.kind::i8 instructions (M = 256, N = 256,

@@ -38,6 +38,8 @@ __all__ = [
     "convrot_read_device_status",
     "convrot_test_wait_timeout",
     "convrot_probe_i8_peak",
+    "convrot_attention_workspace_bytes",
+    "convrot_attention_int8",
     "ConvRotLinear",
     "lib",
 ]
@@ -355,6 +357,39 @@ def convrot_probe_i8_peak(iters: int, ws=None, stream=None) -> int:
         ws = torch.empty((256,), dtype=torch.uint8, device=torch.cuda.current_device())
     _check(L.convrot_probe_i8_peak(int(iters), _ptr(ws), ws.numel(), _stream_ptr(stream)), "convrot_probe_i8_peak")
     return int(L.convrot_probe_i8_peak_ctas())
+
+
+def convrot_attention_workspace_bytes(BH: int, Sq: int, Skv: int, D: int = 128) -> int:
+    return int(lib().convrot_attention_workspace_bytes(BH, Sq, Skv, D))
+
+
+def convrot_attention_int8(Q, K, V, softmax_scale=None, O=None, ws=None, stream=None):
+    """INT8 attention of bf16 Q [..., Sq, 128] with K, V [..., Skv, 128] (same leading
+    dims, flattened to batch*heads): O [..., Sq, 128] bf16 (see include/convrot.h)."""
+    import math
+
+    import torch
+
+    for t, name in ((Q, "Q"), (K, "K"), (V, "V")):
+        _require(t, torch.bfloat16, None, name)
+        if t.dim() < 2 or t.shape[-1] != 128:
+            raise ValueError(f"{name} must be [..., S, 128]")
+    lead = tuple(Q.shape[:-2])
+    if tuple(K.shape[:-2]) != lead or tuple(V.shape) != tuple(K.shape):
+        raise ValueError("Q, K and V must share their leading dimensions, and K and V their shape")
+    Sq, Skv, D = Q.shape[-2], K.shape[-2], Q.shape[-1]
+    BH = int(math.prod(lead)) if lead else 1
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16, device=Q.device)
+    _require(O, torch.bfloat16, tuple(Q.shape), "O")
+    need = convrot_attention_workspace_bytes(BH, Sq, Skv, D)
+    if ws is None:
+        ws = torch.empty((max(need, 256),), dtype=torch.uint8, device=Q.device)
+    _check(lib().convrot_attention_int8(_ptr(Q), _ptr(K), _ptr(V), BH, Sq, Skv, D, float(softmax_scale), _ptr(O),
+                                        _ptr(ws), ws.numel(), _stream_ptr(stream)), "convrot_attention_int8")
+    return O
 
 
 class ConvRotLinear:
