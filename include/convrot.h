@@ -158,10 +158,18 @@ CONVROT_API convrot_status convrot_linear(const void* X, int64_t M, int64_t K, i
  * measured slower than the two-kernel convrot_linear (137 against 110 us).
  * Same arguments, workspace and errors as convrot_linear, plus
  * CONVROT_ERR_UNSUPPORTED when K > 20480 (the worker warps of one CTA hold a
- * token) or K % 128 != 0. Not for CUDA graphs: the counters' per-call tag is
- * drawn on the host at each call, so a replayed graph would reuse it. A call
- * on a stream that is capturing returns CONVROT_ERR_UNSUPPORTED and enqueues
- * nothing.
+ * token) or K % 128 != 0, or when the device cannot hold one CTA of the kernel
+ * on every SM at once (checked on the host). Not for CUDA graphs: the counters'
+ * per-call tag is drawn on the host at each call, so a replayed graph would
+ * reuse it. A call on a stream that is capturing returns CONVROT_ERR_UNSUPPORTED
+ * and enqueues nothing.
+ * The GEMM roles of one CTA wait (bounded) for token blocks that worker warps
+ * of OTHER CTAs quantise, so every CTA of the grid (one per SM) must be
+ * resident at the same time. On a GPU whose SMs are partly held by other work
+ * (another process under MPS, a concurrent kernel), a CTA may not start until
+ * others finish, the wait runs out after about 2 s, and the call reports
+ * CONVROT_ERR_DEVICE_TIMEOUT through the status word without a fault; the
+ * two-kernel convrot_linear has no such dependency.
  */
 CONVROT_API convrot_status convrot_linear_one_launch(const void* X, int64_t M, int64_t K, int g,
                                                      const int8_t* Wq, const float* w_scale, int64_t N,

@@ -276,8 +276,13 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
     gp.x_scale_out = x_scale;
     gp.ready = reinterpret_cast<unsigned long long*>(wsb + lay.ready_off);
     gp.epoch = next_epoch();
+    // the status word is cleared before the launch, so that no CTA's report of a
+    // timed-out wait can come before the clear
+    if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
     if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return CONVROT_ERR_CUDA;
-    if (convrot::launch_linear_fused(g, Wq, Y, gp, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    const cudaError_t fe = convrot::launch_linear_fused(g, Wq, Y, gp, s);
+    if (fe == cudaErrorNotSupported) return CONVROT_ERR_UNSUPPORTED;  // the grid cannot be resident at once
+    if (fe != cudaSuccess) return CONVROT_ERR_CUDA;
     if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return CONVROT_ERR_CUDA;
     if (ev2 != nullptr && cudaEventRecord(ev2, s) != cudaSuccess) return CONVROT_ERR_CUDA;
     return CONVROT_OK;

@@ -534,7 +534,6 @@ __global__ void __launch_bounds__(FG ? kFusedMaxThreads : NUM_THREADS, 1)
   // outputs (and, fused, the workspace it may still read) are touched only
   // after this point.
   griddep_wait();
-  if (FG != 0 && blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0;
 
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
 
@@ -1275,6 +1274,14 @@ cudaError_t launch_impl(const int8_t* A, const int8_t* B, void* out, GemmParams 
   static std::atomic<int> attr_done[kMaxDevices];
   cudaError_t e = ensure_smem_attr(gemm_i8_kernel<EPI, FG>, smem, attr_done);
   if (e != cudaSuccess) return e;
+  if (FG != 0) {
+    // the fused form's CTAs wait for one another's quantised blocks: the whole
+    // grid (one CTA per SM) must fit on the device at once
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_i8_kernel<EPI, FG>, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1 || static_cast<int64_t>(per_sm) * sms < grid) return cudaErrorNotSupported;
+  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;

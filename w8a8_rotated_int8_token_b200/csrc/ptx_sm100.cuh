@@ -61,25 +61,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-#ifndef CONVROT_MBAR_SUSPEND_NS
-#define CONVROT_MBAR_SUSPEND_NS 0
-#endif
-
-// The same test, letting the hardware suspend the thread for up to `ns`
-// nanoseconds until the phase completes (it resumes as soon as it does), so
-// that a waiting warp takes no issue slots from the warps that have work.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
-      : "memory");
-  return done != 0;
-}
-
 // Wait until the phase with the given parity has completed, for at most
 // `timeout_ns`. Returns false if the wait ran out or if another thread of the
 // CTA raised `*abort` (then the caller unwinds; `abort` may be null). Never
@@ -89,11 +70,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-#if CONVROT_MBAR_SUSPEND_NS > 0
-    if (mbar_try_wait_suspend(bar, parity, CONVROT_MBAR_SUSPEND_NS)) return true;
-#else
     if (mbar_try_wait(bar, parity)) return true;
-#endif
     if ((it & 31u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) return false;
