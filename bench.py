@@ -515,12 +515,26 @@ def bench_attention(cr, dev, stream, reps: int, clock_index: int, i8_peak) -> di
     c = clk.summary()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965
-    sfu_peak = SFU_EX2_PER_CLK_PER_SM * sms * mhz * 1e6
+    nominal = SFU_EX2_PER_CLK_PER_SM * sms * mhz * 1e6
+    # the special-function unit's exp2 rate measured on this GPU (probe: independent ex2 chains)
+    L = cr.lib()
+    pws = torch.empty((256,), dtype=torch.float32, device=dev)
+    per_iter = float(L.convrot_probe_ex2_per_iter())
+    iters = 4096
+    for _ in range(2):
+        L.convrot_probe_ex2_peak(iters, pws.data_ptr(), pws.numel() * 4, stream.cuda_stream)
+    e0.record(stream)
+    for _ in range(5):
+        L.convrot_probe_ex2_peak(iters, pws.data_ptr(), pws.numel() * 4, stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    measured = per_iter * iters * 5 / (e0.elapsed_time(e1) * 1e-3)
     out = {"BH": BH, "S": S, "D": D, "call_us": t_ms * 1e3, "tops": ops / (t_ms * 1e-3) / 1e12,
-           "bound": "alu", "exp2_per_s": exps / (t_ms * 1e-3), "exp2_peak_per_s": sfu_peak,
-           "frac_exp2_peak": exps / (t_ms * 1e-3) / sfu_peak, "clock_mhz": c["sm_mhz"],
-           "note": "one call = rotate+quantise of Q and of K, transposition of V, the attention kernel; "
-                   "exp2 peak = 16 per SM per clock at the sampled SM clock"}
+           "bound": "alu", "exp2_per_s": exps / (t_ms * 1e-3), "exp2_peak_per_s": measured,
+           "frac_exp2_peak": exps / (t_ms * 1e-3) / measured, "clock_mhz": c["sm_mhz"],
+           "exp2_peak_source": "measured: independent ex2.approx chains over a full grid (convrot_probe_ex2_peak)",
+           "exp2_nominal_16_per_sm_clk": nominal,
+           "note": "one call = rotate+quantise of Q and of K, transposition of V, the attention kernel"}
     if i8_peak:
         out["tensor_floor_us"] = (2.0 * S * S * D * BH / i8_peak + 2.0 * S * S * D * BH / (i8_peak / 2.0)) / 1e6
     del sets

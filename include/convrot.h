@@ -363,6 +363,17 @@ CONVROT_API convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t
 CONVROT_API int convrot_probe_i8_peak_ctas(void);
 
 /*
+ * convrot_probe_ex2_peak -- measurement aid for the attention softmax's
+ * roofline (not part of the layer): a full grid in which every thread runs
+ * independent chains of the special-function unit's exp2 (ex2.approx), iters
+ * steps each, convrot_probe_ex2_per_iter() exp2 per step over the grid. The
+ * caller times it with events on `stream`. iters in [1, 2^24]; ws >= 1 KB,
+ * 256-byte aligned (never written in practice).
+ */
+CONVROT_API convrot_status convrot_probe_ex2_peak(int64_t iters, void* ws, size_t ws_bytes, convrot_stream_t stream);
+CONVROT_API int64_t convrot_probe_ex2_per_iter(void);
+
+/*
  * convrot_test_wait_timeout -- exercises the bounded device wait: launches one
  * CTA that waits on a barrier nothing will complete, for at most timeout_ns
  * nanoseconds (1e3 .. 1e9), then records CONVROT_ERR_DEVICE_TIMEOUT in the

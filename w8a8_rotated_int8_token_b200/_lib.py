@@ -51,6 +51,8 @@ SIGNATURES = {
     "convrot_attention_int8": (_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _i64, ctypes.c_float,
                                       _c_void_p, _c_void_p, _size, _c_void_p]),
     "convrot_probe_i8_peak_ctas": (_int, []),
+    "convrot_probe_ex2_peak": (_int, [_i64, _c_void_p, _size, _c_void_p]),
+    "convrot_probe_ex2_per_iter": (_i64, []),
 }
 
 _lib = None

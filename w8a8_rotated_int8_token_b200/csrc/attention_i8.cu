@@ -23,15 +23,22 @@
 //                      K = 4 x 32) into TMEM columns 0..127 and
 //                      O += P V (kind::f16 with bf16 operands, M = N = 128,
 //                      K = 8 x 16) into columns 128..255.
-//   warps 2..5       : softmax, one query row per thread (TMEM lane): S from
-//                      TMEM, t = c_i s_k[j] S_ij in base-2 units with
-//                      c_i = s_q[i] softmax_scale log2(e), p = 2^(t - m) in
-//                      float32, the row sum in float32, P rounded to bf16 into
-//                      128-byte-swizzled shared memory for the MMA. The
+//   warps 2..9       : softmax, two warps per query row (TMEM lane): one takes
+//                      keys 0..63 of every block and O columns 0..63, the
+//                      other keys 64..127 and O columns 64..127. S from TMEM,
+//                      t = c_i s_k[j] S_ij in base-2 units with
+//                      c_i = s_q[i] softmax_scale log2(e), the block maximum
+//                      of the row combined across the pair through shared
+//                      memory, p = 2^(t - m) in float32 (packed f32x2
+//                      arithmetic), the row sums in float32, P rounded to bf16
+//                      into 128-byte-swizzled shared memory for the MMA. The
 //                      reference maximum m moves only when a block raises it
 //                      by more than 8 (p <= 256), and then O is rescaled in
 //                      TMEM once the previous block's P V has finished. At
-//                      the end O / sum is rounded to bf16 and stored.
+//                      the end O / sum is rounded to bf16 and stored. The two
+//                      warps of a pair meet at a named barrier every block,
+//                      also after a timed-out wait (they then skip the work),
+//                      so neither can be left waiting for the other.
 // S is read out of TMEM before the next block's S is written, so the next
 // QK^T runs on the tensor cores while this block's softmax runs on the CUDA
 // cores. Every wait is bounded (status word + abort flag, as in the GEMM).
@@ -56,7 +63,8 @@ namespace {
 constexpr int AT_BQ = 128;  // queries per CTA tile
 constexpr int AT_BK = 128;  // keys per block
 constexpr int AT_D = 128;   // head dimension
-constexpr int AT_THREADS = 192;
+constexpr int AT_SOFTMAX_WARPS = 8;  // two per TMEM lane quarter: keys (and O columns) 0..63 and 64..127
+constexpr int AT_THREADS = 64 + 32 * AT_SOFTMAX_WARPS;
 constexpr int kQBytes = AT_BQ * AT_D;      // int8 query codes: 16 KB
 constexpr int kKBytes = AT_BK * AT_D;      // int8 key codes of one block: 16 KB
 constexpr int kHalf = 128 * 128;           // one 64-key half of a bf16 operand: 128 rows x 128 B
@@ -74,8 +82,10 @@ struct AttnSmem {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kKBytes;
   static constexpr int kOffP = kOffV + kVBytes;
-  static constexpr int kOffSk = kOffP + kPBytes;  // per softmax warp, two buffers of a block's key scales
-  static constexpr int kOffBar = kOffSk + 4 * 2 * AT_BK * 4;
+  static constexpr int kOffSk = kOffP + kPBytes;  // per softmax warp, two buffers of its 64 key scales
+  static constexpr int kOffMx = kOffSk + AT_SOFTMAX_WARPS * 2 * 64 * 4;  // [2 blocks][2 halves][128 rows] maxima
+  static constexpr int kOffLs = kOffMx + 2 * 2 * AT_BQ * 4;              // [2 halves][128 rows] row sums
+  static constexpr int kOffBar = kOffLs + 2 * AT_BQ * 4;
   // q_full, k_full, k_empty, v_full, v_empty, s_full, s_empty, p_full, o_done, drain
   static constexpr int kNumBars = 10;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
@@ -119,30 +129,68 @@ __device__ __forceinline__ float small_int_to_float(uint32_t acc) {
   return __uint_as_float(acc + 0x4B400000u) - 12582912.0f;
 }
 
-// The probabilities of one row for 64 keys (one half), packed to bf16 into the
-// row's 128-byte-swizzled shared-memory line; returns their float32 sum.
-template <bool MASKED>
-__device__ __forceinline__ float write_p_half(const float (&u)[128], int h, float c, float m_ref, int nvalid,
-                                              uint8_t* row, int sw) {
-  float sum = 0.0f;
+// One pass over this thread's 64 logits of a block, straight from TMEM in four
+// 16-column loads: t = c * s_k[key] * S[row, key] (base-2 units); with
+// WRITE_P the probabilities p = 2^(t - m_ref) are rounded to bf16 into the
+// row's 128-byte-swizzled shared-memory line and their float32 sum returned.
+// The maximum over the valid keys of s_k[key] * S[row, key] goes to *mh.
+template <bool WRITE_P, bool MASKED>
+__device__ __forceinline__ float softmax_pass(uint32_t t_s, const float* skb, float c, float m_ref, int nvalid,
+                                              uint8_t* row, int sw, float* mh) {
+  const float2 mg = make_float2(-12582912.0f, -12582912.0f);
+  const float2 c2 = make_float2(c, c);
+  const float2 nm2 = make_float2(-m_ref, -m_ref);
+  float2 sum2 = make_float2(0.0f, 0.0f);
+  float ma = -INFINITY, mc = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint32_t w[4];
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t a[16];
+    tmem_ld_32x32b_x16(t_s + ch * 16, a);
+    tmem_ld_wait_regs16(a);
+    uint32_t w[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = h * 64 + i * 8 + 2 * e;
-      float p0 = ex2_approx(fmaf(c, u[k], -m_ref));
-      float p1 = ex2_approx(fmaf(c, u[k + 1], -m_ref));
+    for (int i = 0; i < 8; ++i) {
+      const int k = ch * 16 + 2 * i;  // key (within this half) of the pair's first element
+      // float(acc) for |acc| < 2^22: the integer added to the bits of 1.5 * 2^23, minus 1.5 * 2^23
+      const float2 x = make_float2(__uint_as_float(a[2 * i] + 0x4B400000u), __uint_as_float(a[2 * i + 1] + 0x4B400000u));
+      const float2 u = __fmul2_rn(__fadd2_rn(x, mg), *reinterpret_cast<const float2*>(skb + k));
       if (MASKED) {
-        p0 = (k < nvalid) ? p0 : 0.0f;
-        p1 = (k + 1 < nvalid) ? p1 : 0.0f;
+        ma = (k < nvalid) ? fmaxf(ma, u.x) : ma;
+        mc = (k + 1 < nvalid) ? fmaxf(mc, u.y) : mc;
+      } else if (i & 1) {
+        mc = fwht::fmax3f(mc, u.x, u.y);
+      } else {
+        ma = fwht::fmax3f(ma, u.x, u.y);
       }
-      sum += p0 + p1;
-      w[e] = pack_bf16x2(p0, p1);
+      if (WRITE_P) {
+        const float2 t = __ffma2_rn(c2, u, nm2);
+        float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+        if (MASKED) {
+          pp.x = (k < nvalid) ? pp.x : 0.0f;
+          pp.y = (k + 1 < nvalid) ? pp.y : 0.0f;
+        }
+        sum2 = __fadd2_rn(sum2, pp);
+        w[i] = pack_bf16x2(pp.x, pp.y);
+      }
     }
-    *reinterpret_cast<uint4*>(row + ((i ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (WRITE_P) {  // keys 16 ch .. 16 ch + 15: 16-byte pieces 2 ch and 2 ch + 1
+      *reinterpret_cast<uint4*>(row + (((2 * ch) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(row + (((2 * ch + 1) ^ sw) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+    }
   }
-  return sum;
+  *mh = fmaxf(ma, mc);
+  return sum2.x + sum2.y;
+}
+
+template <bool WRITE_P>
+__device__ __forceinline__ float softmax_pass_any(uint32_t t_s, const float* skb, float c, float m_ref, int nvalid,
+                                                  uint8_t* row, int sw, float* mh) {
+  return nvalid == 64 ? softmax_pass<WRITE_P, false>(t_s, skb, c, m_ref, nvalid, row, sw, mh)
+                      : softmax_pass<WRITE_P, true>(t_s, skb, c, m_ref, nvalid, row, sw, mh);
+}
+
+__device__ __forceinline__ void pair_bar(int id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 2)
@@ -181,8 +229,8 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_empty, 4);  // the four softmax warps
-    mbar_init(p_full, 4);
+    mbar_init(s_empty, AT_SOFTMAX_WARPS);  // every softmax warp
+    mbar_init(p_full, AT_SOFTMAX_WARPS);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort = 0;
@@ -290,154 +338,122 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int qd = warp & 3;  // TMEM lane quarter this warp may access
+    const int hf = (warp - 2) >> 2;  // which 64 keys of a block (and O columns) this warp takes
+    const int qd = warp & 3;         // TMEM lane quarter this warp may access
     const int r = qd * 32 + lane;
     const int qrow = q0 + r;
+    const int bar_id = 1 + qd;  // the two warps of this lane quarter
     const float sqv = (qrow < p.Sq) ? __ldg(p.sq + static_cast<int64_t>(bh) * p.Sq + qrow) : 0.0f;
     const float c = sqv * p.c_scale;  // >= 0
-    const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
-    uint8_t* prow = smem + L::kOffP + r * 128;
+    const uint32_t t_row = (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(hf * 64);
+    uint8_t* prow = smem + L::kOffP + hf * kHalf + r * 128;
     const int sw = r & 7;
-    const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv;
-    // this warp's two buffers of a block's 128 key scales (no barrier across warps)
-    float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * AT_BK;
+    const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv + hf * 64;
+    float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * 64;
+    float* mxb = reinterpret_cast<float*>(smem + L::kOffMx);
+    float* lsb = reinterpret_cast<float*>(smem + L::kOffLs);
     float m_ref = 0.0f;
     float l = 0.0f;
     bool ok = true;
-    // lane loads keys 4 * lane .. 4 * lane + 3 of each block, one block ahead
-    float skn[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) skn[e] = (4 * lane + e < p.Skv) ? __ldg(skh + 4 * lane + e) : 0.0f;
+    // lane loads the scales of keys 2 * lane, 2 * lane + 1 of this warp's half, one block ahead
+    float2 skn;
+    skn.x = (hf * 64 + 2 * lane < p.Skv) ? __ldg(skh + 2 * lane) : 0.0f;
+    skn.y = (hf * 64 + 2 * lane + 1 < p.Skv) ? __ldg(skh + 2 * lane + 1) : 0.0f;
     for (int j = 0; j < J; ++j) {
-      float* skb = skw + (j & 1) * AT_BK;
-      *reinterpret_cast<float4*>(skb + 4 * lane) = make_float4(skn[0], skn[1], skn[2], skn[3]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kn = (j + 1) * AT_BK + 4 * lane + e;
-        skn[e] = (j + 1 < J && kn < p.Skv) ? __ldg(skh + kn) : 0.0f;
+      float* skb = skw + (j & 1) * 64;
+      *reinterpret_cast<float2*>(skb + 2 * lane) = skn;
+      {
+        const int kn = (j + 1) * AT_BK + hf * 64 + 2 * lane;
+        skn.x = (j + 1 < J && kn < p.Skv) ? __ldg(skh + (j + 1) * AT_BK + 2 * lane) : 0.0f;
+        skn.y = (j + 1 < J && kn + 1 < p.Skv) ? __ldg(skh + (j + 1) * AT_BK + 2 * lane + 1) : 0.0f;
       }
       __syncwarp();  // the block's key scales are in this warp's buffer
-      const int nvalid = (p.Skv - j * AT_BK) < AT_BK ? (p.Skv - j * AT_BK) : AT_BK;
+      int nvalid = p.Skv - j * AT_BK - hf * 64;  // valid keys among this warp's 64
+      nvalid = nvalid < 0 ? 0 : (nvalid > 64 ? 64 : nvalid);
 
-      if (!warp_wait_bounded(s_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
-        ok = false;
-        break;
+      // S_j is in TMEM; the previous block's P V has finished (O stable, P buffer free)
+      if (ok) ok = warp_wait_bounded(s_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns);
+      if (ok && j >= 1) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns);
+      if (ok) tc_fence_after();
+      const uint32_t t_s = tS + t_row;
+      float mh = -INFINITY;
+      float bl = 0.0f;
+      if (ok) {
+        if (j == 0)  // the first block sets the reference maximum: its maximum first
+          softmax_pass_any<false>(t_s, skb, c, 0.0f, nvalid, prow, sw, &mh);
+        else  // later blocks: probabilities against the current reference, maximum alongside
+          bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &mh);
       }
-      tc_fence_after();
-      float u[128];  // s_k[key] * S[row, key]: the logit without the row factor c
-      {
-        // two 32-column loads in flight at a time, converted as they land
-        uint32_t a0[32], a1[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld_32x32b_x32(tS + lane_off + half * 64, a0);
-          tmem_ld_32x32b_x32(tS + lane_off + half * 64 + 32, a1);
-          tmem_ld_wait_regs(a0);
-          tmem_ld_wait_regs(a1);
-          if (half == 1) {
-            // S has been read: the next block's QK^T may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty);
-          }
-#pragma unroll
-          for (int k4 = 0; k4 < 16; ++k4) {
-            const float4 s4 = *reinterpret_cast<const float4*>(skb + half * 64 + 4 * k4);
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 4 * k4 + e;
-              const uint32_t acc = (k < 32) ? a0[k] : a1[k - 32];
-              u[half * 64 + k] = small_int_to_float(acc) * sv[e];
-            }
-          }
-        }
-      }
-      // the block maximum over its valid keys, in base-2 units
-      float mb;
-      if (nvalid == AT_BK) {
-        // 128 -> 43 -> 15 -> 5 -> 1 with three-input maxima
-        float a[43], b[15], c5[5];
-#pragma unroll
-        for (int i = 0; i < 42; ++i) a[i] = fwht::fmax3f(u[3 * i], u[3 * i + 1], u[3 * i + 2]);
-        a[42] = fmaxf(u[126], u[127]);
-#pragma unroll
-        for (int i = 0; i < 14; ++i) b[i] = fwht::fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-        b[14] = a[42];
-#pragma unroll
-        for (int i = 0; i < 5; ++i) c5[i] = fwht::fmax3f(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
-        mb = fmaxf(fwht::fmax3f(c5[0], c5[1], c5[2]), fmaxf(c5[3], c5[4]));
-      } else {
-        mb = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < AT_BK; ++k) mb = (k < nvalid) ? fmaxf(mb, u[k]) : mb;
-      }
-      const float t_max = c * mb;
+      // the row's block maximum over both halves (every block has a valid key)
+      mxb[((j & 1) * 2 + hf) * AT_BQ + r] = mh;
+      pair_bar(bar_id);
+      const float t_max = c * fmaxf(mh, mxb[((j & 1) * 2 + (hf ^ 1)) * AT_BQ + r]);
       float alpha = 1.0f;
-      bool need = false;
+      bool need = false;   // O has to follow a raised reference
+      bool redo = j == 0;  // P has to be (re)written against the new reference
       if (j == 0) {
         m_ref = t_max;
       } else if (t_max > m_ref + kRescaleThreshold) {
         alpha = ex2_approx(m_ref - t_max);
         m_ref = t_max;
-        need = true;
+        need = redo = true;
       }
-      // the previous block's P V has finished: O is stable and the P buffer free
-      if (j >= 1 && !warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float bl;
-      if (nvalid == AT_BK) {
-        bl = write_p_half<false>(u, 0, c, m_ref, nvalid, prow, sw) +
-             write_p_half<false>(u, 1, c, m_ref, nvalid, prow + kHalf, sw);
-      } else {
-        bl = write_p_half<true>(u, 0, c, m_ref, nvalid, prow, sw) +
-             write_p_half<true>(u, 1, c, m_ref, nvalid, prow + kHalf, sw);
-      }
-      l = l * alpha + bl;
-      // O to the new reference maximum before this block's P V adds to it
-      // (after the P writes, so that the logits are no longer live)
-      if (__any_sync(0xFFFFFFFFu, need)) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tO + lane_off + ch * 32, o);
-          tmem_ld_wait_regs(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st_32x32b_x32(tO + lane_off + ch * 32, o);
+      if (ok) {
+        if (redo) {
+          float unused;
+          bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &unused);
         }
-        tmem_st_wait();
-      }
-      // P is read by the tensor cores (async proxy); O's rescale is complete
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (ok) {
-      if (!warp_wait_bounded(o_done, static_cast<uint32_t>((J - 1) & 1), abort, p.timeout_ns)) {
-        ok = false;
-      } else {
-        tc_fence_after();
-        const float inv = 1.0f / l;
-        uint16_t* orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qrow) * AT_D;
+        l = l * alpha + bl;
+        // S has been read: the next block's QK^T may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty);
+        // this warp's 64 columns of O to the new reference maximum before this block's P V adds to them
+        if (__any_sync(0xFFFFFFFFu, need)) {
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tO + lane_off + ch * 32, o);
-          tmem_ld_wait_regs(o);
-          uint32_t w[16];
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[16];
+            tmem_ld_32x32b_x16(tO + t_row + ch * 16, o);
+            tmem_ld_wait_regs16(o);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-          if (qrow < p.Sq) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2);
+              o[2 * i] = __float_as_uint(v.x);
+              o[2 * i + 1] = __float_as_uint(v.y);
+            }
+            tmem_st_32x32b_x16(tO + t_row + ch * 16, o);
           }
+          tmem_st_wait();
+        }
+        // P is read by the tensor cores (async proxy); O's rescale is complete
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+    }
+    if (ok) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((J - 1) & 1), abort, p.timeout_ns);
+    // the row sum over both halves
+    lsb[hf * AT_BQ + r] = l;
+    pair_bar(bar_id);
+    const float inv = 1.0f / (l + lsb[(hf ^ 1) * AT_BQ + r]);
+    if (ok) {
+      tc_fence_after();
+      uint16_t* orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qrow) * AT_D + hf * 64;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[16];
+        tmem_ld_32x32b_x16(tO + t_row + ch * 16, o);
+        tmem_ld_wait_regs16(o);
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        if (qrow < p.Sq) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 16);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
       }
     }

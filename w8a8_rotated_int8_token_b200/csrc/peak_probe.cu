@@ -1,9 +1,11 @@
-// Measured peak of the int8 tensor pipe: the same instruction the layer's GEMM
+// Measured peaks of the units the hot kernels are bound by. The int8 tensor pipe: the same instruction the layer's GEMM
 // issues (tcgen05.mma.cta_group::2.kind::i8, M = 256, N = 256, K = 32 per
 // instruction, both operands from shared memory) in a loop with no global
 // memory traffic, so that a timed launch gives the rate the tensor cores
-// sustain on this GPU at its current clock. It is a measurement aid for the
-// roofline of the GEMM; it computes nothing of the layer.
+// sustain on this GPU at its current clock. The special-function unit's exp2
+// (the unit the attention softmax is bound by): independent chains of
+// ex2.approx in every thread of a full grid. Measurement aids for the
+// rooflines; they compute nothing of the layer.
 
 #include <cuda_runtime.h>
 
@@ -67,11 +69,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, 256);
 }
 
+constexpr int kEx2Threads = 256;
+constexpr int kEx2CtasPerSm = 8;
+constexpr int kEx2Chains = 8;
+
+__global__ void __launch_bounds__(kEx2Threads) ex2_peak_kernel(int64_t iters, float* sink) {
+  float y[kEx2Chains];
+#pragma unroll
+  for (int i = 0; i < kEx2Chains; ++i) y[i] = 0.5f + 0.01f * static_cast<float>(threadIdx.x & 7) + 0.001f * i;
+  for (int64_t it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < kEx2Chains; ++i) y[i] = ex2_approx(-y[i]);  // stays in [0.5, 1)
+  }
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kEx2Chains; ++i) s += y[i];
+  if (s == 12345.0f) sink[threadIdx.x] = s;  // never true: keeps the chains live
+}
+
 }  // namespace
 
 }  // namespace convrot
 
 extern "C" {
+
+convrot_status convrot_probe_ex2_peak(int64_t iters, void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  if (iters < 1 || iters > (int64_t(1) << 24)) return CONVROT_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % 256) != 0 || ws_bytes < 256 * sizeof(float))
+    return CONVROT_ERR_WORKSPACE;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  convrot::ex2_peak_kernel<<<sms * convrot::kEx2CtasPerSm, convrot::kEx2Threads, 0,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(iters, static_cast<float*>(ws));
+  return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+int64_t convrot_probe_ex2_per_iter(void) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return static_cast<int64_t>(sms) * convrot::kEx2CtasPerSm * convrot::kEx2Threads * convrot::kEx2Chains;
+}
 
 convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t ws_bytes, convrot_stream_t stream) {
   // at most 2^20 x 512 tensor cycles (about 0.3 s at 1.9 GHz): well inside the 2 s bound of the final wait
