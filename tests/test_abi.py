@@ -52,13 +52,21 @@ def test_library_exports_nothing_else():
     assert exported == set(_declared_entry_points())
 
 
-def linear_ws_layout(M, K):
-    """Byte layout of convrot_linear's workspace, as include/convrot.h describes it."""
+def linear_ws_layout(M, K, N=None):
+    """Byte layout of convrot_linear's workspace, as include/convrot.h describes it
+    (the split buffers of the weight-streaming GEMM, for 1 <= M <= 64, when N is given)."""
     up = lambda v, a: (v + a - 1) // a * a  # noqa: E731
     ready = 256
     scale = up(ready + 8 * ((M + 127) // 128), 256)
     codes = up(scale + 4 * M, 1024)
-    return {"ready": ready, "scale": scale, "codes": codes, "total": up(codes + M * K, 256)}
+    total = up(codes + M * K, 256)
+    lay = {"ready": ready, "scale": scale, "codes": codes, "total": total}
+    if N is not None and 1 <= M <= 64 and (N + 127) // 128 <= 4096:
+        bnt = 16 if M <= 16 else (32 if M <= 32 else 64)
+        lay["split_count"] = total
+        lay["split_part"] = up(total + 4 * ((N + 127) // 128), 1024)
+        lay["total"] = up(lay["split_part"] + 2 * 160 * bnt * 128 * 4, 256)
+    return lay
 
 
 def test_status_strings_and_version(L):
@@ -73,12 +81,15 @@ def test_workspace_sizes(L):
     # [status 256 B | ready counters 8 B per 128 tokens | scales 4M | codes M*K]
     M, N, K = 4608, 9216, 3072
     need = L.convrot_linear_workspace_bytes(M, N, K, 256)
-    assert need == linear_ws_layout(M, K)["total"]
+    assert need == linear_ws_layout(M, K, N)["total"]
     assert need >= M * K + 4 * M + 8 * (M // 128) + 256
     assert L.convrot_linear_workspace_bytes(M, N, K, 64) == 0       # unsupported g
     assert L.convrot_linear_workspace_bytes(M, N, 3000, 256) == 0   # K % g != 0
     assert L.convrot_linear_workspace_bytes(M, 9212, K, 256) == 0   # N % 8 != 0
-    assert L.convrot_linear_workspace_bytes(0, N, K, 256) == linear_ws_layout(0, K)["total"]  # M = 0 is valid
+    assert L.convrot_linear_workspace_bytes(0, N, K, 256) == linear_ws_layout(0, K, N)["total"]  # M = 0 is valid
+    # the weight-streaming GEMM's split buffers (M <= 64)
+    for m in (1, 16, 17, 33, 64, 65):
+        assert L.convrot_linear_workspace_bytes(m, 12288, 4096, 128) == linear_ws_layout(m, 4096, 12288)["total"]
     assert L.convrot_linear_workspace_bytes(-1, N, K, 256) == 0
     assert L.convrot_gemm_workspace_bytes() == 256
     assert L.convrot_prepare_weight_workspace_bytes() >= 4

@@ -346,6 +346,33 @@ def test_linear_ragged_and_large_k(cr, M, N, K, g):
     _linear_case(cr, _random_layer(M, N, K, g))
 
 
+# The weight-streaming GEMM (M <= 64) split over all SMs: (weight tile, k-block)
+# units in equal contiguous ranges per CTA, partial tiles summed by the last CTA
+# to arrive. Cases: tiles shared by two and three CTAs (K = 12288: 96 k-blocks
+# per tile), one k-block per tile (every unit a whole tile), fewer units than
+# SMs, N not a multiple of 128 (the last tile's rows past N), M at 1, 17 and 64
+# (16-, 32- and 64-token MMA columns), and more tiles than SMs.
+@pytest.mark.parametrize("M,N,K,g", [(1, 12288, 4096, 128), (17, 1032, 12288, 256), (64, 384, 12288, 256),
+                                     (5, 8192, 128, 128), (3, 200, 256, 256), (40, 2056, 768, 256),
+                                     (9, 40960, 1024, 256)])
+def test_linear_weight_streaming_split(cr, M, N, K, g):
+    _linear_case(cr, _random_layer(M, N, K, g))
+
+
+def test_linear_weight_streaming_split_is_deterministic(cr):
+    # the partial sums meet in whatever order the CTAs arrive; integer sums make the
+    # result independent of it, so repeated calls give identical bits
+    import torch
+
+    d = _random_layer(16, 12288, 4096, 128)
+    Wq, sw = cr.convrot_prepare_weight(to_torch_bf16(d["w"]), 128)
+    X = to_torch_bf16(d["x"])
+    outs = [cr.convrot_linear(X, Wq, sw, 128, to_torch_bf16(d["bias"])) for _ in range(4)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
 @pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256),   # largest K of the one-launch form
                                      (1, 16, 384, 128), (385, 520, 1024, 256), (64, 256, 256, 256)])
 def test_linear_one_launch_matches_oracle(cr, M, N, K, g):

@@ -12,36 +12,41 @@
 //
 // One call: Q and K through the rotate+quantise kernel (codes + one scale per
 // token), V transposed once into key-contiguous rows (the K-major B operand of
-// the P V product), then one CTA per (batch*head, 128-query tile):
+// the P V product), then one CTA per SM at a time, each on one
+// (batch*head, 128-query tile):
 //   warp 0, one lane : TMA producer: the tile's 128 x 128 query codes once,
-//                      then per 128-key block the key codes (loaded as soon
-//                      as the previous block's S is computed) and the
-//                      transposed values (two 64-key halves, loaded as soon
-//                      as the previous block's P V is done).
-//   warp 1           : allocates 256 TMEM columns; one lane issues
-//                      S = Qq Kq^T (tcgen05.mma kind::i8, M = N = 128,
-//                      K = 4 x 32) into TMEM columns 0..127 and
-//                      O += P V (kind::f16 with bf16 operands, M = N = 128,
-//                      K = 8 x 16) into columns 128..255.
+//                      then per 128-key block j the key codes into stage j%2
+//                      (once S of block j-2 is computed) and the transposed
+//                      values, two 64-key halves, into stage j%2 (once P V of
+//                      block j-2 is done).
+//   warp 1           : allocates 512 TMEM columns; one lane issues
+//                      S_j = Qq Kq_j^T (tcgen05.mma kind::i8, M = N = 128,
+//                      K = 4 x 32) into S buffer j%2 (TMEM columns 0..127 or
+//                      128..255) and O += P_j V_j (kind::f16 with bf16
+//                      operands, M = N = 128, K = 8 x 16) into columns
+//                      256..383, in the order S_0, S_1, PV_0, S_2, PV_1, ...
 //   warps 2..9       : softmax, two warps per query row (TMEM lane): one takes
 //                      keys 0..63 of every block and O columns 0..63, the
-//                      other keys 64..127 and O columns 64..127. S from TMEM,
-//                      t = c_i s_k[j] S_ij in base-2 units with
-//                      c_i = s_q[i] softmax_scale log2(e), the block maximum
-//                      of the row combined across the pair through shared
-//                      memory, p = 2^(t - m) in float32 (packed f32x2
-//                      arithmetic), the row sums in float32, P rounded to bf16
-//                      into 128-byte-swizzled shared memory for the MMA. The
-//                      reference maximum m moves only when a block raises it
-//                      by more than 8 (p <= 256), and then O is rescaled in
-//                      TMEM once the previous block's P V has finished. At
-//                      the end O / sum is rounded to bf16 and stored. The two
-//                      warps of a pair meet at a named barrier every block,
-//                      also after a timed-out wait (they then skip the work),
-//                      so neither can be left waiting for the other.
-// S is read out of TMEM before the next block's S is written, so the next
-// QK^T runs on the tensor cores while this block's softmax runs on the CUDA
-// cores. Every wait is bounded (status word + abort flag, as in the GEMM).
+//                      other keys 64..127 and O columns 64..127. One pass per
+//                      block straight from TMEM: t = c_i s_k[j] S_ij in base-2
+//                      units (c_i = s_q[i] softmax_scale log2(e)),
+//                      p = 2^(t - m) against the current reference maximum m
+//                      (packed f32x2 arithmetic), P rounded to bf16 into the
+//                      128-byte-swizzled P buffer j%2, the row sums in
+//                      float32; the block maximum of the row is combined
+//                      across the pair through shared memory. When a block
+//                      raises the maximum by more than 8 (p would pass 256)
+//                      the reference moves, the block's pass is redone (S is
+//                      still in TMEM) and O is rescaled in TMEM once the
+//                      previous block's P V is done. The two warps of a pair
+//                      meet at a named barrier every block, also after a
+//                      timed-out wait (they then skip the work), so neither
+//                      can be left waiting for the other. At the end
+//                      O / (sum of both halves) is rounded to bf16 and stored.
+// Every buffer is double: the next block's QK^T and loads run while this
+// block's softmax runs on the CUDA cores and the previous block's P V on the
+// tensor cores. Every mbarrier is waited on phase by phase in order, and every
+// wait is bounded (status word + abort flag, as in the GEMM).
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -75,19 +80,17 @@ constexpr uint32_t IDESC_O = idesc_bf16(AT_BQ, AT_D);
 constexpr int kTimeoutStatus = 5;
 constexpr float kRescaleThreshold = 8.0f;  // base-2 units: probabilities stay below 2^8
 
-// 2 CTAs per SM: everything below (plus the alignment slack) stays under
-// half of the SM's 228 KB of shared memory.
 struct AttnSmem {
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kKBytes;
-  static constexpr int kOffP = kOffV + kVBytes;
-  static constexpr int kOffSk = kOffP + kPBytes;  // per softmax warp, two buffers of its 64 key scales
+  static constexpr int kOffK = kOffQ + kQBytes;       // two stages
+  static constexpr int kOffV = kOffK + 2 * kKBytes;   // two stages
+  static constexpr int kOffP = kOffV + 2 * kVBytes;   // two buffers
+  static constexpr int kOffSk = kOffP + 2 * kPBytes;  // per softmax warp, two buffers of its 64 key scales
   static constexpr int kOffMx = kOffSk + AT_SOFTMAX_WARPS * 2 * 64 * 4;  // [2 blocks][2 halves][128 rows] maxima
   static constexpr int kOffLs = kOffMx + 2 * 2 * AT_BQ * 4;              // [2 halves][128 rows] row sums
   static constexpr int kOffBar = kOffLs + 2 * AT_BQ * 4;
-  // q_full, k_full, k_empty, v_full, v_empty, s_full, s_empty, p_full, o_done, drain
-  static constexpr int kNumBars = 10;
+  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2], p_full, o_done, drain
+  static constexpr int kNumBars = 16;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 8;
   static constexpr int kBytes = kOffAbort + 8;
@@ -189,11 +192,13 @@ __device__ __forceinline__ float softmax_pass_any(uint32_t t_s, const float* skb
                       : softmax_pass<WRITE_P, true>(t_s, skb, c, m_ref, nvalid, row, sw, mh);
 }
 
+// The two softmax warps of one TMEM lane quarter (64 threads) meet here. The
+// non-aligned form: a warp need not arrive converged.
 __device__ __forceinline__ void pair_bar(int id) {
-  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+  asm volatile("barrier.sync %0, 64;" ::"r"(id) : "memory");
 }
 
-__global__ void __launch_bounds__(AT_THREADS, 2)
+__global__ void __launch_bounds__(AT_THREADS, 1)
     attention_i8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using L = AttnSmem;
@@ -201,15 +206,15 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 2;
-  uint64_t* v_full = bars + 3;
-  uint64_t* v_empty = bars + 4;
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_empty = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* o_done = bars + 8;
-  uint64_t* drain = bars + 9;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2]
+  uint64_t* s_empty = bars + 11;  // [2]
+  uint64_t* p_full = bars + 13;
+  uint64_t* o_done = bars + 14;
+  uint64_t* drain = bars + 15;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
 
@@ -224,12 +229,14 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     mbar_init(q_full, 1);
-    mbar_init(k_full, 1);
-    mbar_init(k_empty, 1);
-    mbar_init(v_full, 1);
-    mbar_init(v_empty, 1);
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, AT_SOFTMAX_WARPS);  // every softmax warp
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&k_full[b], 1);
+      mbar_init(&k_empty[b], 1);
+      mbar_init(&v_full[b], 1);
+      mbar_init(&v_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], AT_SOFTMAX_WARPS);  // every softmax warp
+    }
     mbar_init(p_full, AT_SOFTMAX_WARPS);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -237,91 +244,99 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_ptr, 256);
+    tmem_alloc(tmem_ptr, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
-  const uint32_t tS = tmem_base;        // S: columns 0..127
-  const uint32_t tO = tmem_base + 128;  // O: columns 128..255
+  const uint32_t tO = tmem_base + 256;  // O: columns 256..383; S buffer b: columns 128 b ..
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // Tensor-pipe order is S_0, S_1, PV_0, S_2, PV_1, ...: K_{j+1} goes out
-    // when S_j is done, V_{j+1} when PV_j is done.
     if (lane == 0) {
       bool ok = true;
       int issued_k = 0, issued_v = 0;
       auto load_k = [&](int j) {
-        mbar_arrive_expect_tx(k_full, kKBytes);
-        tma_load_3d(smem + L::kOffK, &tmK, k_full, 0, j * AT_BK, bh);
+        const int b = j & 1;
+        mbar_arrive_expect_tx(&k_full[b], kKBytes);
+        tma_load_3d(smem + L::kOffK + b * kKBytes, &tmK, &k_full[b], 0, j * AT_BK, bh);
         issued_k = j + 1;
       };
       auto load_v = [&](int j) {
-        mbar_arrive_expect_tx(v_full, kVBytes);
-        tma_load_3d(smem + L::kOffV, &tmV, v_full, j * AT_BK, 0, bh);
-        tma_load_3d(smem + L::kOffV + kHalf, &tmV, v_full, j * AT_BK + 64, 0, bh);
+        const int b = j & 1;
+        uint8_t* dst = smem + L::kOffV + b * kVBytes;
+        mbar_arrive_expect_tx(&v_full[b], kVBytes);
+        tma_load_3d(dst, &tmV, &v_full[b], j * AT_BK, 0, bh);
+        tma_load_3d(dst + kHalf, &tmV, &v_full[b], j * AT_BK + 64, 0, bh);
         issued_v = j + 1;
       };
       mbar_arrive_expect_tx(q_full, kQBytes);
       tma_load_3d(smem + L::kOffQ, &tmQ, q_full, 0, q0, bh);
       load_k(0);
       load_v(0);
-      for (int j = 0; j + 1 < J; ++j) {
-        if (!mbar_wait_bounded(k_empty, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
+      if (J > 1) {
+        load_k(1);
+        load_v(1);
+      }
+      for (int j = 0; j + 2 < J; ++j) {
+        // stage j%2 again once block j is done with it (the (j/2)-th use of the stage)
+        const uint32_t par = static_cast<uint32_t>((j >> 1) & 1);
+        if (!mbar_wait_bounded(&k_empty[j & 1], par, abort, p.timeout_ns)) {
           ok = false;
           break;
         }
-        load_k(j + 1);
-        if (!mbar_wait_bounded(v_empty, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
+        load_k(j + 2);
+        if (!mbar_wait_bounded(&v_empty[j & 1], par, abort, p.timeout_ns)) {
           ok = false;
           break;
         }
-        load_v(j + 1);
+        load_v(j + 2);
       }
       if (!ok) {
         attn_abort(abort, p.status);
         // every copy already issued lands before the shared memory goes away
         mbar_wait_bounded(q_full, 0u, nullptr, p.timeout_ns);
-        if (issued_k > 0) mbar_wait_bounded(k_full, static_cast<uint32_t>((issued_k - 1) & 1), nullptr, p.timeout_ns);
-        if (issued_v > 0) mbar_wait_bounded(v_full, static_cast<uint32_t>((issued_v - 1) & 1), nullptr, p.timeout_ns);
+        for (int j = (issued_k > 2 ? issued_k - 2 : 0); j < issued_k; ++j)
+          mbar_wait_bounded(&k_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), nullptr, p.timeout_ns);
+        for (int j = (issued_v > 2 ? issued_v - 2 : 0); j < issued_v; ++j)
+          mbar_wait_bounded(&v_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), nullptr, p.timeout_ns);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t qa = smem_addr(smem + L::kOffQ);
-      const uint32_t pa = smem_addr(smem + L::kOffP);
-      const uint32_t va = smem_addr(smem + L::kOffV);
-      const uint32_t kb = smem_addr(smem + L::kOffK);
       auto mma_s = [&](int j) -> bool {
-        if (!mbar_wait_bounded(k_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) return false;
+        const int b = j & 1;
+        const uint32_t par = static_cast<uint32_t>((j >> 1) & 1);
+        // S buffer b free (the softmax of block j-2 has read it) and K_j landed
+        if (j >= 2 && !mbar_wait_bounded(&s_empty[b], par ^ 1u, abort, p.timeout_ns)) return false;
+        if (!mbar_wait_bounded(&k_full[b], par, abort, p.timeout_ns)) return false;
         tc_fence_after();
+        const uint32_t kb = smem_addr(smem + L::kOffK + b * kKBytes);
+        const uint32_t ts = tmem_base + static_cast<uint32_t>(b * 128);
 #pragma unroll
         for (int k = 0; k < AT_D / 32; ++k)
-          mma_i8(tS, smem_desc_k_sw128(qa + k * 32), smem_desc_k_sw128(kb + k * 32), IDESC_S, k > 0 ? 1u : 0u);
-        mma_commit(s_full);
-        mma_commit(k_empty);
+          mma_i8(ts, smem_desc_k_sw128(qa + k * 32), smem_desc_k_sw128(kb + k * 32), IDESC_S, k > 0 ? 1u : 0u);
+        mma_commit(&s_full[b]);
+        mma_commit(&k_empty[b]);
         return true;
       };
       bool ok = mbar_wait_bounded(q_full, 0u, abort, p.timeout_ns);
       if (ok) ok = mma_s(0);
+      if (ok && J > 1) ok = mma_s(1);
       for (int j = 0; j < J && ok; ++j) {
-        if (j + 1 < J) {
-          // S_{j+1} once the softmax has read S_j out of TMEM
-          if (!mbar_wait_bounded(s_empty, static_cast<uint32_t>(j & 1), abort, p.timeout_ns) || !mma_s(j + 1)) {
-            ok = false;
-            break;
-          }
-        }
+        const int b = j & 1;
         if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns) ||
-            !mbar_wait_bounded(v_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
+            !mbar_wait_bounded(&v_full[b], static_cast<uint32_t>((j >> 1) & 1), abort, p.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t pa = smem_addr(smem + L::kOffP + b * kPBytes);
+        const uint32_t va = smem_addr(smem + L::kOffV + b * kVBytes);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -329,7 +344,11 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
             mma_bf16(tO, smem_desc_k_sw128(pa + h * kHalf + k * 32), smem_desc_k_sw128(va + h * kHalf + k * 32),
                      IDESC_O, (j | h | k) != 0 ? 1u : 0u);
         mma_commit(o_done);
-        mma_commit(v_empty);
+        mma_commit(&v_empty[b]);
+        if (j + 2 < J && !mma_s(j + 2)) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) attn_abort(abort, p.status);
       // every MMA this thread issued has finished before TMEM is released
@@ -346,7 +365,6 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
     const float sqv = (qrow < p.Sq) ? __ldg(p.sq + static_cast<int64_t>(bh) * p.Sq + qrow) : 0.0f;
     const float c = sqv * p.c_scale;  // >= 0
     const uint32_t t_row = (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(hf * 64);
-    uint8_t* prow = smem + L::kOffP + hf * kHalf + r * 128;
     const int sw = r & 7;
     const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv + hf * 64;
     float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * 64;
@@ -360,7 +378,8 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
     skn.x = (hf * 64 + 2 * lane < p.Skv) ? __ldg(skh + 2 * lane) : 0.0f;
     skn.y = (hf * 64 + 2 * lane + 1 < p.Skv) ? __ldg(skh + 2 * lane + 1) : 0.0f;
     for (int j = 0; j < J; ++j) {
-      float* skb = skw + (j & 1) * 64;
+      const int b = j & 1;
+      float* skb = skw + b * 64;
       *reinterpret_cast<float2*>(skb + 2 * lane) = skn;
       {
         const int kn = (j + 1) * AT_BK + hf * 64 + 2 * lane;
@@ -370,12 +389,13 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
       __syncwarp();  // the block's key scales are in this warp's buffer
       int nvalid = p.Skv - j * AT_BK - hf * 64;  // valid keys among this warp's 64
       nvalid = nvalid < 0 ? 0 : (nvalid > 64 ? 64 : nvalid);
+      uint8_t* prow = smem + L::kOffP + b * kPBytes + hf * kHalf + r * 128;
+      const uint32_t t_s = tmem_base + static_cast<uint32_t>(b * 128) + t_row;
 
-      // S_j is in TMEM; the previous block's P V has finished (O stable, P buffer free)
-      if (ok) ok = warp_wait_bounded(s_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns);
-      if (ok && j >= 1) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns);
+      // S_j is in TMEM. P buffer b was last read by P V of block j-2, which was
+      // done before this warp signalled block j-1 (it waited for it there).
+      if (ok) ok = warp_wait_bounded(&s_full[b], static_cast<uint32_t>((j >> 1) & 1), abort, p.timeout_ns);
       if (ok) tc_fence_after();
-      const uint32_t t_s = tS + t_row;
       float mh = -INFINITY;
       float bl = 0.0f;
       if (ok) {
@@ -385,9 +405,9 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
           bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &mh);
       }
       // the row's block maximum over both halves (every block has a valid key)
-      mxb[((j & 1) * 2 + hf) * AT_BQ + r] = mh;
+      mxb[(b * 2 + hf) * AT_BQ + r] = mh;
       pair_bar(bar_id);
-      const float t_max = c * fmaxf(mh, mxb[((j & 1) * 2 + (hf ^ 1)) * AT_BQ + r]);
+      const float t_max = c * fmaxf(mh, mxb[(b * 2 + (hf ^ 1)) * AT_BQ + r]);
       float alpha = 1.0f;
       bool need = false;   // O has to follow a raised reference
       bool redo = j == 0;  // P has to be (re)written against the new reference
@@ -399,15 +419,24 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
         need = redo = true;
       }
       if (ok) {
-        if (redo) {
+        // The pass reads TMEM with warp-collective loads, so the whole warp runs
+        // it when any of its rows needs it; for the others the reference did not
+        // move and the pass writes the same probabilities again.
+        if (__any_sync(0xFFFFFFFFu, redo)) {
           float unused;
-          bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &unused);
+          const float bl2 = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &unused);
+          if (redo) bl = bl2;
         }
         l = l * alpha + bl;
-        // S has been read: the next block's QK^T may overwrite it
+        // S_j has been read: its buffer may take S_{j+2}
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty);
+        if (lane == 0) mbar_arrive(&s_empty[b]);
+      }
+      // P V of block j-1 is done: O is stable (and, for block j+1, P buffer b^1 is free)
+      if (ok && j >= 1) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns);
+      if (ok) {
+        tc_fence_after();
         // this warp's 64 columns of O to the new reference maximum before this block's P V adds to them
         if (__any_sync(0xFFFFFFFFu, need)) {
           const float2 a2 = make_float2(alpha, alpha);
@@ -463,7 +492,7 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 256);
+    tmem_dealloc(tmem_base, 512);
   }
 }
 

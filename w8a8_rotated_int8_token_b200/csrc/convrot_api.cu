@@ -23,22 +23,37 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device
 // two kernels at the time), so it is offered only as its own entry point.
 
 // Workspace of convrot_linear:
-// [status word | 256 B][M-block ready counters, 8 B each][token scales][int8 codes].
+// [status word | 256 B][M-block ready counters, 8 B each][token scales][int8 codes]
+// and, for the weight-streaming GEMM (M <= 64) split over all SMs,
+// [arrival counters, one per 128 weight rows][int32 partial accumulators].
 constexpr size_t kStatusBytes = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct LinearWs {
-  size_t ready_off, scale_off, codes_off, total;
+  size_t ready_off, scale_off, codes_off, split_count_off, split_part_off, total;
+  bool split;
 };
 
-LinearWs linear_ws_layout(int64_t M, int64_t K) {
+// Whether convrot_linear runs the weight-streaming GEMM split over all SMs.
+bool linear_uses_split(int64_t M, int64_t N) {
+  return M >= 1 && M <= convrot::kSmallM && (N + 127) / 128 <= convrot::kMaxSplitTiles;
+}
+
+LinearWs linear_ws_layout(int64_t M, int64_t K, int64_t N) {
   LinearWs w;
   w.ready_off = kStatusBytes;
   const size_t mblocks = (static_cast<size_t>(M) + 127) / 128;
   w.scale_off = align_up(w.ready_off + 8 * mblocks, 256);
   w.codes_off = align_up(w.scale_off + 4 * static_cast<size_t>(M), 1024);
   w.total = align_up(w.codes_off + static_cast<size_t>(M) * static_cast<size_t>(K), 256);
+  w.split = linear_uses_split(M, N);
+  w.split_count_off = w.split_part_off = 0;
+  if (w.split) {
+    w.split_count_off = w.total;
+    w.split_part_off = align_up(w.split_count_off + convrot::split_count_bytes(N), 1024);
+    w.total = align_up(w.split_part_off + convrot::split_part_bytes(static_cast<int>(M)), 256);
+  }
   return w;
 }
 
@@ -96,8 +111,11 @@ struct EpiOptions {
 
 convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, int64_t M, int64_t N, int64_t K,
                         const float* x_scale, const float* w_scale, const void* bias, int* status,
-                        cudaStream_t stream, EpiOptions opt = EpiOptions()) {
+                        cudaStream_t stream, EpiOptions opt = EpiOptions(), int32_t* split_part = nullptr,
+                        unsigned* split_count = nullptr) {
   convrot::GemmParams p{};
+  p.split_part = split_part;
+  p.split_count = split_count;
   p.out_f16 = opt.out_f16;
   p.wscale_per_channel = opt.wscale_per_channel;
   p.addend = static_cast<const uint16_t*>(opt.addend);
@@ -210,7 +228,7 @@ convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K, int g, int
 
 size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
   if (check_rotation_shape(M, K, g) != CONVROT_OK || check_gemm_shape(M, N, K, 8) != CONVROT_OK) return 0;
-  return linear_ws_layout(M, K).total;
+  return linear_ws_layout(M, K, N).total;
 }
 
 }  // extern "C"
@@ -246,7 +264,7 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
       !aligned(Y, 16) || (bias != nullptr && !aligned(bias, 16)) ||
       (opt.addend != nullptr && !aligned(opt.addend, 16)))
     return CONVROT_ERR_INVALID_ARG;
-  const LinearWs lay = linear_ws_layout(M, K);
+  const LinearWs lay = linear_ws_layout(M, K, N);
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(wsb);
@@ -300,12 +318,23 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   p.status_reset = status;  // CTA 0 of the first kernel clears the status word of this call
   p.status = status;
   p.timeout_ns = kWaitTimeoutNs;
+  int32_t* split_part = nullptr;
+  unsigned* split_count = nullptr;
+  if (lay.split) {
+    // the weight-streaming GEMM split over all SMs: its arrival counters are
+    // zeroed by the first kernel, before the GEMM may start
+    split_part = reinterpret_cast<int32_t*>(wsb + lay.split_part_off);
+    split_count = reinterpret_cast<unsigned*>(wsb + lay.split_count_off);
+    p.zero_words = split_count;
+    p.zero_count = static_cast<int>((N + 127) / 128);
+  }
   if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   const int epi = opt.act ? convrot::kEpiDequantGenGelu
                            : (opt.general() ? convrot::kEpiDequantGen : convrot::kEpiDequantBf16);
-  const convrot_status st = run_gemm(epi, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s, opt);
+  const convrot_status st =
+      run_gemm(epi, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s, opt, split_part, split_count);
   if (st != CONVROT_OK) return st;
   if (ev2 != nullptr && cudaEventRecord(ev2, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   return CONVROT_OK;

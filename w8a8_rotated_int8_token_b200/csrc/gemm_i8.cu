@@ -948,21 +948,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 
 // ===================================================== small-M (swap-AB) form
 //
-// For at most 128 tokens the layer is bound by streaming the int8 weight. The
+// For at most 64 tokens the layer is bound by streaming the int8 weight. The
 // MMA then takes the weight as its M side (128 weight rows per tile) and the
-// tokens as its N side (16..128): D[n][m] = sum_k Wq[n][k] Xq[m][k]. One CTA
-// per 128 weight rows streams its 128 x K panel through a deep TMA ring (the
-// activation codes are tiny and stay in L2); the panel is prefetched into L2
+// tokens as its N side (16..64): D[n][m] = sum_k Wq[n][k] Xq[m][k]. The
+// weight streams through a deep TMA ring per CTA (the activation codes are
+// tiny and stay in L2); the weight loads of the first ring stages go out
 // before waiting on the previous kernel, so the weight streams while the
 // rotate+quantise kernel runs. TMEM lane n holds weight row n, so the
 // epilogue writes Y[m][n] with 32 consecutive n per warp store.
+//
+// Work split. Without split buffers, CTA c takes weight tiles c, c + grid,
+// ... whole (one CTA per 128 weight rows, so N/128 of the SMs stream). With
+// them, the (weight tile, 128-wide k-block) units are divided evenly into
+// contiguous ranges, one per CTA on every SM, so a tile's K loop may be
+// shared by two or three consecutive CTAs. A CTA that holds only part of a
+// tile's K stores its int32 partial accumulators in its own slot and counts
+// itself in at the tile's arrival counter; the CTA that arrives last adds the
+// other slots to its own partial and runs the epilogue. Integer addition is
+// exact, so the result does not depend on the order of arrival, and no CTA
+// ever waits for another.
 
 constexpr int SM_BW = 128;  // weight rows per tile
 
 template <int BNT>
 struct SmallSmem {
   static constexpr int kW = SM_BW * BK;  // 16 KB
-  static constexpr int kX = BNT * BK;    // 2..16 KB
+  static constexpr int kX = BNT * BK;    // 2..8 KB
   static constexpr int kFit = (200 * 1024) / (kW + kX);
 #ifdef CONVROT_SMALLM_STAGES
   static constexpr int kStages = CONVROT_SMALLM_STAGES < kFit ? CONVROT_SMALLM_STAGES : kFit;
@@ -975,9 +986,78 @@ struct SmallSmem {
   static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 8;
-  static constexpr int kBytes = kOffAbort + 8;
+  static constexpr int kOffLast = kOffAbort + 8;  // split form: "this CTA finishes the tile"
+  static constexpr int kBytes = kOffLast + 8;
   static constexpr int kAlloc = kBytes + 1024;
 };
+
+// The sequence of (weight tile, k-block range) segments a CTA works on; every
+// role of the CTA walks the same sequence.
+struct SmallSegments {
+  bool split;
+  int KB, tiles, G;
+  int64_t u, u1;  // split: the CTA's unit range [u, u1)
+  int next;       // no split: the next whole tile
+  __device__ __forceinline__ SmallSegments(const GemmParams& p, int num_tiles) {
+    split = p.split_part != nullptr;
+    KB = p.num_k_blocks;
+    tiles = num_tiles;
+    G = static_cast<int>(gridDim.x);
+    const int64_t U = static_cast<int64_t>(tiles) * KB;
+    u = static_cast<int64_t>(blockIdx.x) * U / G;
+    u1 = static_cast<int64_t>(blockIdx.x + 1) * U / G;
+    next = static_cast<int>(blockIdx.x);
+  }
+  __device__ __forceinline__ bool get(int& tile, int& k0, int& k1) {
+    if (split) {
+      if (u >= u1) return false;
+      tile = static_cast<int>(u / KB);
+      k0 = static_cast<int>(u - static_cast<int64_t>(tile) * KB);
+      const int64_t left = u1 - u;
+      k1 = (KB - k0) < left ? KB : k0 + static_cast<int>(left);
+      u += k1 - k0;
+      return true;
+    }
+    if (next >= tiles) return false;
+    tile = next;
+    k0 = 0;
+    k1 = KB;
+    next += G;
+    return true;
+  }
+  // split form: the CTA holding unit x, and the first unit of CTA c
+  __device__ __forceinline__ int cta_of(int64_t x) const {
+    const int64_t U = static_cast<int64_t>(tiles) * KB;
+    return static_cast<int>(((x + 1) * G - 1) / U);
+  }
+  __device__ __forceinline__ int64_t first_unit(int c) const {
+    return static_cast<int64_t>(c) * (static_cast<int64_t>(tiles) * KB) / G;
+  }
+};
+
+__device__ __forceinline__ void epi_named_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// One output value of the weight-streaming epilogue: token m, output channel n.
+template <int EPI>
+__device__ __forceinline__ void smallm_store(const GemmParams& p, void* out, int m, int n, int32_t acc, float sw,
+                                             float swn, float bn) {
+  if (EPI == kEpiDequantBf16) {
+    const float y = fmaf(static_cast<float>(acc), __ldg(p.x_scale + m) * sw, bn);
+    static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(y);
+  } else if (epi_is_general(EPI)) {
+    const int64_t at = static_cast<int64_t>(m) * (p.ldy ? p.ldy : p.N) + n;
+    float bias_add = bn;
+    if (p.addend != nullptr) bias_add += out16_to_f32(__ldg(p.addend + at), p.out_f16 != 0);
+    float y = fmaf(static_cast<float>(acc), __ldg(p.x_scale + m) * swn, bias_add);
+    if (EPI == kEpiDequantGenGelu) y = gelu_erf(y);
+    if (p.out_f16)
+      static_cast<__half*>(out)[at] = __float2half_rn(y);
+    else
+      static_cast<__nv_bfloat16*>(out)[at] = __float2bfloat16_rn(y);
+  } else {
+    static_cast<int32_t*>(out)[static_cast<int64_t>(m) * p.N + n] = acc;
+  }
+}
 
 template <int EPI, int BNT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -996,6 +1076,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* drain = tmem_empty + 2;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kOffLast);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1030,6 +1111,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      SmallSegments seg(p, num_tiles);
       int s = 0;
       uint32_t ph = 0;
       int pending_phase[S];
@@ -1044,8 +1126,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = 0; i < n_early; ++i)
           tma_load_2d(smem + L::kOffX + early_s[i] * L::kX, &tmX, &full[early_s[i]], early_kb[i] * BK, 0);
       };
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+      int tile, k0, k1;
+      while (ok && seg.get(tile, k0, k1)) {
+        for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort, p.timeout_ns)) {
             ok = false;
             break;
@@ -1077,11 +1160,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      SmallSegments seg(p, num_tiles);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      int tile, k0, k1;
+      while (ok && seg.get(tile, k0, k1)) {
         const int b = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait_bounded(&tmem_empty[b], (use & 1u) ^ 1u, abort, p.timeout_ns)) {
@@ -1090,7 +1175,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(b * 128);
-        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        for (int kb = k0; kb < k1; ++kb) {
           if (!mbar_wait_bounded(&full[s], ph, abort, p.timeout_ns)) {
             ok = false;
             break;
@@ -1101,7 +1186,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             mma_i8(d, smem_desc_k_sw128(w_base + k * UMMA_K), smem_desc_k_sw128(x_base + k * UMMA_K), kIdesc,
-                   (kb | k) != 0 ? 1u : 0u);
+                   (kb > k0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&empty[s]);
           if (++s == S) {
@@ -1111,67 +1196,93 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         mma_commit(&tmem_full[b]);
+        ++it;
       }
       if (!ok) raise_abort(abort, p.status);
       mma_commit(drain);
       mbar_wait_bounded(drain, 0u, nullptr, p.timeout_ns);
     }
   } else {
-    griddep_wait();  // the token scales come from the previous kernel
+    griddep_wait();  // the token scales (and the split counters' zeroing) come from the previous kernel
+    SmallSegments seg(p, num_tiles);
     const int q = warp & 3;
+    const int nl = q * 32 + lane;  // weight row within the tile (TMEM lane)
     const float sw = epi_weight_scale<EPI>(p);
     int it = 0;
+    int si = 0;  // segment index within this CTA
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    int tile, k0, k1;
+    while (seg.get(tile, k0, k1)) {
       const int b = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
-      const int n = tile * SM_BW + q * 32 + lane;
+      const int n = tile * SM_BW + nl;
+      const bool whole = (k0 == 0 && k1 == seg.KB);
       float bn = 0.0f;
       float swn = sw;  // this thread's output channel's weight scale
       if (epi_is_dequant(EPI) && n < p.N) {
         if (p.bias != nullptr) bn = out16_to_f32(__ldg(p.bias + n), epi_is_general(EPI) && p.out_f16 != 0);
         if (epi_is_general(EPI) && p.wscale_per_channel) swn = __ldg(p.w_scale + n);
       }
-      if (!mbar_wait_bounded(&tmem_full[b], use & 1u, abort, p.timeout_ns)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * 128);
-#pragma unroll 1
-      for (int c = 0; c < BNT / 16; ++c) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(c * 16), r);
-        tmem_ld_wait();
-        if (c == BNT / 16 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tmem_empty[b]);
-        }
-        if (n >= p.N) continue;
+      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tmem_full[b], use & 1u, abort, p.timeout_ns));
+      // the accumulators of this segment: token m of weight row n in acc[m]
+      int32_t acc[BNT];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = c * 16 + j;
-          if (m >= p.M) break;
-          if (EPI == kEpiDequantBf16) {
-            const float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * sw, bn);
-            const __nv_bfloat16 h = __float2bfloat16_rn(y);
-            static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = h;
-          } else if (epi_is_general(EPI)) {
-            const int64_t at = static_cast<int64_t>(m) * (p.ldy ? p.ldy : p.N) + n;
-            float bias_add = bn;
-            if (p.addend != nullptr) bias_add += out16_to_f32(__ldg(p.addend + at), p.out_f16 != 0);
-            float y = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), __ldg(p.x_scale + m) * swn, bias_add);
-            if (EPI == kEpiDequantGenGelu) y = gelu_erf(y);
-            if (p.out_f16)
-              static_cast<__half*>(out)[at] = __float2half_rn(y);
-            else
-              static_cast<__nv_bfloat16*>(out)[at] = __float2bfloat16_rn(y);
-          } else {
-            static_cast<int32_t*>(out)[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[j]);
+      for (int m = 0; m < BNT; ++m) acc[m] = 0;
+      if (ok) {
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * 128);
+#pragma unroll
+        for (int c = 0; c < BNT / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(t_row + static_cast<uint32_t>(c * 16), r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[c * 16 + j] = static_cast<int32_t>(r[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tmem_empty[b]);
+      }
+      bool write_out = whole;
+      if (!whole) {
+        // split form, part of a tile: this CTA's partial to its slot (slot 0:
+        // its first segment, 1: its last), counted in at the tile's counter
+        int32_t* part = p.split_part + static_cast<int64_t>(2 * blockIdx.x + (si == 0 ? 0 : 1)) * BNT * 128;
+        if (ok) {
+#pragma unroll
+          for (int m = 0; m < BNT; ++m) part[m * 128 + nl] = acc[m];
+        }
+        __threadfence();
+        epi_named_barrier();  // every epilogue thread's partial is stored (all four warps, also after a timeout)
+        if (threadIdx.x == 64) {
+          const int c_first = seg.cta_of(static_cast<int64_t>(tile) * seg.KB);
+          const int c_last = seg.cta_of(static_cast<int64_t>(tile) * seg.KB + seg.KB - 1);
+          const unsigned prev = atomicAdd(p.split_count + tile, 1u);
+          *last_flag = (prev == static_cast<unsigned>(c_last - c_first)) ? 1 : 0;
+        }
+        epi_named_barrier();
+        write_out = *last_flag != 0;
+        if (write_out && ok) {
+          __threadfence();
+          // add the other contributors' partials (read through L2)
+          const int c_first = seg.cta_of(static_cast<int64_t>(tile) * seg.KB);
+          const int c_last = seg.cta_of(static_cast<int64_t>(tile) * seg.KB + seg.KB - 1);
+          for (int c = c_first; c <= c_last; ++c) {
+            if (c == static_cast<int>(blockIdx.x)) continue;
+            const int slot = 2 * c + ((seg.first_unit(c) / seg.KB) == tile ? 0 : 1);
+            const int32_t* op = p.split_part + static_cast<int64_t>(slot) * BNT * 128;
+#pragma unroll
+            for (int m = 0; m < BNT; ++m) acc[m] += __ldcg(op + m * 128 + nl);
           }
         }
       }
+      if (write_out && ok && n < p.N) {
+#pragma unroll
+        for (int m = 0; m < BNT; ++m)
+          if (m < p.M) smallm_store<EPI>(p, out, m, n, acc[m], sw, swn, bn);
+      }
+      ++it;
+      ++si;
     }
     if (!ok && lane == 0) raise_abort(abort, p.status);
     __syncwarp();
@@ -1367,7 +1478,14 @@ cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmPar
   const int tiles = (p.N + SM_BW - 1) / SM_BW;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const int grid = tiles < sms ? tiles : sms;
+  int grid = tiles < sms ? tiles : sms;
+  if (p.split_part != nullptr) {
+    // every SM streams an equal share of the (tile, k-block) units
+    if (tiles > kMaxSplitTiles || BNT != smallm_bnt(p.M)) return cudaErrorInvalidValue;
+    const int64_t units = static_cast<int64_t>(tiles) * p.num_k_blocks;
+    const int cap = sms < kMaxSplitCtas ? sms : kMaxSplitCtas;
+    grid = static_cast<int>(units < cap ? units : cap);
+  }
   constexpr int smem = SmallSmem<BNT>::kAlloc;
   static std::atomic<int> attr_done[kMaxDevices];
   cudaError_t e = ensure_smem_attr(gemm_i8_smallm_kernel<EPI, BNT>, smem, attr_done);

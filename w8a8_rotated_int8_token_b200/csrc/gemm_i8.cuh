@@ -40,10 +40,26 @@ struct GemmParams {
   unsigned long long* ready;      // [num_m_blocks] epoch << 32 | rows quantised
   uint32_t epoch;                 // unique per call, never 0
   int q_threads_per_row, q_rows_per_pass;  // filled by the launcher
+  // weight-streaming form split over all SMs (launch_gemm_i8 with M <= kSmallM):
+  // null = one CTA per 128 weight rows; else the (weight tile, k-block) units
+  // are divided evenly over the CTAs, and partial tiles meet in these buffers
+  int32_t* split_part;            // [2 * kMaxSplitCtas][BNT][128] int32 partial accumulators
+  unsigned* split_count;          // [weight tiles] arrival counters, zero when the kernel starts
 };
 
 constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass (fused form)
 constexpr int kSmallM = 64;  // up to this many tokens the GEMM runs in the weight-streaming (swap-AB) form
+constexpr int kMaxSplitCtas = 160;    // CTAs of the split weight-streaming form (at most)
+constexpr int kMaxSplitTiles = 4096;  // weight tiles (128 rows each) the split form takes (N <= 524288)
+
+// Token columns of the weight-streaming form's MMA for M tokens (16, 32 or 64).
+__host__ __device__ constexpr int smallm_bnt(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+
+// Bytes of the split form's partial buffers and counters for M tokens and N outputs.
+__host__ __device__ constexpr size_t split_part_bytes(int M) {
+  return static_cast<size_t>(2 * kMaxSplitCtas) * smallm_bnt(M) * 128 * 4;
+}
+__host__ __device__ constexpr size_t split_count_bytes(int64_t N) { return static_cast<size_t>((N + 127) / 128) * 4; }
 
 // Worker layout of the fused kernel for a given K; false if K is not a
 // multiple of 128 or too large for one CTA's worker warps (then the layer runs

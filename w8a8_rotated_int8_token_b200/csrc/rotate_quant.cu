@@ -104,7 +104,15 @@ __global__ void __maxnreg__(rq_maxnreg<G>()) rotate_quant_kernel(RotQuantParams 
   // The input may be the previous kernel's output: wait for it (launches are
   // programmatic), then let the next kernel start its prologue early.
   griddep_wait();
-  if (MODE == kRqActivation && p.status_reset != nullptr && blockIdx.x == 0 && tid == 0) *p.status_reset = 0;
+  if (MODE == kRqActivation && blockIdx.x == 0) {
+    // words the next kernel of the call counts in (its split arrival counters),
+    // and the call's status word: cleared before the next kernel may start
+    if (p.zero_words != nullptr)
+      for (int i = tid; i < p.zero_count; i += blockDim.x) p.zero_words[i] = 0u;
+    if (p.status_reset != nullptr && tid == 0) *p.status_reset = 0;
+    __threadfence();
+    __syncthreads();
+  }
   griddep_launch_dependents();
 
   // The producer (thread 0) keeps S-1 row blocks of this CTA in flight: block

@@ -31,6 +31,8 @@ struct RotQuantParams {
   float* scale;             // [rows] (activation) or [1] (weight)
   unsigned* tensor_absmax;  // weight modes: float bits of the unnormalised absmax
   int* status_reset;        // activation mode: status word zeroed by CTA 0, or null
+  unsigned* zero_words;     // activation mode: words zeroed by CTA 0 for the next kernel (or null)
+  int zero_count;
   int* status;              // a timed-out wait ORs 5 into it (may be null)
   uint64_t timeout_ns;      // bound of every device-side wait
   int threads_per_row;      // filled by launch_rotate_quant
