@@ -25,24 +25,23 @@
 //                      128..255) and O += P_j V_j (kind::f16 with bf16
 //                      operands, M = N = 128, K = 8 x 16) into columns
 //                      256..383, in the order S_0, S_1, PV_0, S_2, PV_1, ...
-//   warps 2..9       : softmax, two warps per query row (TMEM lane): one takes
-//                      keys 0..63 of every block and O columns 0..63, the
-//                      other keys 64..127 and O columns 64..127. One pass per
+//   warps 2..17      : softmax, four warps per query row (TMEM lane), each
+//                      taking 32 keys of every block and 32 O columns. One pass per
 //                      block straight from TMEM: t = c_i s_k[j] S_ij in base-2
 //                      units (c_i = s_q[i] softmax_scale log2(e)),
 //                      p = 2^(t - m) against the current reference maximum m
 //                      (packed f32x2 arithmetic), P rounded to bf16 into the
 //                      128-byte-swizzled P buffer j%2, the row sums in
 //                      float32; the block maximum of the row is combined
-//                      across the pair through shared memory. When a block
+//                      across the four warps through shared memory. When a block
 //                      raises the maximum by more than 8 (p would pass 256)
 //                      the reference moves, the block's pass is redone (S is
 //                      still in TMEM) and O is rescaled in TMEM once the
-//                      previous block's P V is done. The two warps of a pair
+//                      previous block's P V is done. The four warps of a row
 //                      meet at a named barrier every block, also after a
-//                      timed-out wait (they then skip the work), so neither
-//                      can be left waiting for the other. At the end
-//                      O / (sum of both halves) is rounded to bf16 and stored.
+//                      timed-out wait (they then skip the work), so none can
+//                      be left waiting for another. At the end
+//                      O / (sum of the four parts) is rounded to bf16 and stored.
 // Every buffer is double: the next block's QK^T and loads run while this
 // block's softmax runs on the CUDA cores and the previous block's P V on the
 // tensor cores. Every mbarrier is waited on phase by phase in order, and every
@@ -68,7 +67,8 @@ namespace {
 constexpr int AT_BQ = 128;  // queries per CTA tile
 constexpr int AT_BK = 128;  // keys per block
 constexpr int AT_D = 128;   // head dimension
-constexpr int AT_SOFTMAX_WARPS = 8;  // two per TMEM lane quarter: keys (and O columns) 0..63 and 64..127
+constexpr int AT_SOFTMAX_WARPS = 16;  // four per TMEM lane quarter: 32 keys (and 32 O columns) each
+constexpr int AT_SUB = 32;            // keys of a block (and O columns) per softmax warp
 constexpr int AT_THREADS = 64 + 32 * AT_SOFTMAX_WARPS;
 constexpr int kQBytes = AT_BQ * AT_D;      // int8 query codes: 16 KB
 constexpr int kKBytes = AT_BK * AT_D;      // int8 key codes of one block: 16 KB
@@ -85,10 +85,10 @@ struct AttnSmem {
   static constexpr int kOffK = kOffQ + kQBytes;       // two stages
   static constexpr int kOffV = kOffK + 2 * kKBytes;   // two stages
   static constexpr int kOffP = kOffV + 2 * kVBytes;   // two buffers
-  static constexpr int kOffSk = kOffP + 2 * kPBytes;  // per softmax warp, two buffers of its 64 key scales
-  static constexpr int kOffMx = kOffSk + AT_SOFTMAX_WARPS * 2 * 64 * 4;  // [2 blocks][2 halves][128 rows] maxima
-  static constexpr int kOffLs = kOffMx + 2 * 2 * AT_BQ * 4;              // [2 halves][128 rows] row sums
-  static constexpr int kOffBar = kOffLs + 2 * AT_BQ * 4;
+  static constexpr int kOffSk = kOffP + 2 * kPBytes;  // per softmax warp, two buffers of its 32 key scales
+  static constexpr int kOffMx = kOffSk + AT_SOFTMAX_WARPS * 2 * AT_SUB * 4;  // [2 blocks][4 parts][128 rows] maxima
+  static constexpr int kOffLs = kOffMx + 2 * 4 * AT_BQ * 4;                  // [4 parts][128 rows] row sums
+  static constexpr int kOffBar = kOffLs + 4 * AT_BQ * 4;
   // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2], p_full, o_done, drain
   static constexpr int kNumBars = 16;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
@@ -132,30 +132,34 @@ __device__ __forceinline__ float small_int_to_float(uint32_t acc) {
   return __uint_as_float(acc + 0x4B400000u) - 12582912.0f;
 }
 
-// One pass over this thread's 64 logits of a block, straight from TMEM in four
-// 16-column loads: t = c * s_k[key] * S[row, key] (base-2 units); with
-// WRITE_P the probabilities p = 2^(t - m_ref) are rounded to bf16 into the
-// row's 128-byte-swizzled shared-memory line and their float32 sum returned.
-// The maximum over the valid keys of s_k[key] * S[row, key] goes to *mh.
+// One pass over this thread's 32 logits of a block, straight from TMEM (both
+// 16-column loads in flight together): t = c * s_k[key] * S[row, key] (base-2
+// units); with WRITE_P the probabilities p = 2^(t - m_ref) are rounded to bf16
+// into the four 16-byte pieces `piece0`.. of the row's 128-byte-swizzled
+// shared-memory line and their float32 sum returned. The maximum over the
+// valid keys of s_k[key] * S[row, key] goes to *mh.
 template <bool WRITE_P, bool MASKED>
 __device__ __forceinline__ float softmax_pass(uint32_t t_s, const float* skb, float c, float m_ref, int nvalid,
-                                              uint8_t* row, int sw, float* mh) {
+                                              uint8_t* row, int piece0, int sw, float* mh) {
   const float2 mg = make_float2(-12582912.0f, -12582912.0f);
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m_ref, -m_ref);
   float2 sum2 = make_float2(0.0f, 0.0f);
   float ma = -INFINITY, mc = -INFINITY;
+  uint32_t a[2][16];
+  tmem_ld_32x32b_x16(t_s, a[0]);
+  tmem_ld_32x32b_x16(t_s + 16, a[1]);
+  tmem_ld_wait_regs16(a[0]);
+  tmem_ld_wait_regs16(a[1]);
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-    uint32_t a[16];
-    tmem_ld_32x32b_x16(t_s + ch * 16, a);
-    tmem_ld_wait_regs16(a);
+  for (int ch = 0; ch < 2; ++ch) {
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int k = ch * 16 + 2 * i;  // key (within this half) of the pair's first element
+      const int k = ch * 16 + 2 * i;  // key (within this warp's 32) of the pair's first element
       // float(acc) for |acc| < 2^22: the integer added to the bits of 1.5 * 2^23, minus 1.5 * 2^23
-      const float2 x = make_float2(__uint_as_float(a[2 * i] + 0x4B400000u), __uint_as_float(a[2 * i + 1] + 0x4B400000u));
+      const float2 x =
+          make_float2(__uint_as_float(a[ch][2 * i] + 0x4B400000u), __uint_as_float(a[ch][2 * i + 1] + 0x4B400000u));
       const float2 u = __fmul2_rn(__fadd2_rn(x, mg), *reinterpret_cast<const float2*>(skb + k));
       if (MASKED) {
         ma = (k < nvalid) ? fmaxf(ma, u.x) : ma;
@@ -176,9 +180,9 @@ __device__ __forceinline__ float softmax_pass(uint32_t t_s, const float* skb, fl
         w[i] = pack_bf16x2(pp.x, pp.y);
       }
     }
-    if (WRITE_P) {  // keys 16 ch .. 16 ch + 15: 16-byte pieces 2 ch and 2 ch + 1
-      *reinterpret_cast<uint4*>(row + (((2 * ch) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(row + (((2 * ch + 1) ^ sw) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+    if (WRITE_P) {  // keys 16 ch .. 16 ch + 15 of this warp: pieces piece0 + 2 ch, piece0 + 2 ch + 1
+      *reinterpret_cast<uint4*>(row + (((piece0 + 2 * ch) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(row + (((piece0 + 2 * ch + 1) ^ sw) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
     }
   }
   *mh = fmaxf(ma, mc);
@@ -187,15 +191,15 @@ __device__ __forceinline__ float softmax_pass(uint32_t t_s, const float* skb, fl
 
 template <bool WRITE_P>
 __device__ __forceinline__ float softmax_pass_any(uint32_t t_s, const float* skb, float c, float m_ref, int nvalid,
-                                                  uint8_t* row, int sw, float* mh) {
-  return nvalid == 64 ? softmax_pass<WRITE_P, false>(t_s, skb, c, m_ref, nvalid, row, sw, mh)
-                      : softmax_pass<WRITE_P, true>(t_s, skb, c, m_ref, nvalid, row, sw, mh);
+                                                  uint8_t* row, int piece0, int sw, float* mh) {
+  return nvalid == AT_SUB ? softmax_pass<WRITE_P, false>(t_s, skb, c, m_ref, nvalid, row, piece0, sw, mh)
+                          : softmax_pass<WRITE_P, true>(t_s, skb, c, m_ref, nvalid, row, piece0, sw, mh);
 }
 
-// The two softmax warps of one TMEM lane quarter (64 threads) meet here. The
+// The four softmax warps of one TMEM lane quarter (128 threads) meet here. The
 // non-aligned form: a warp need not arrive converged.
-__device__ __forceinline__ void pair_bar(int id) {
-  asm volatile("barrier.sync %0, 64;" ::"r"(id) : "memory");
+__device__ __forceinline__ void quarter_bar(int id) {
+  asm volatile("barrier.sync %0, 128;" ::"r"(id) : "memory");
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
@@ -357,39 +361,37 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int hf = (warp - 2) >> 2;  // which 64 keys of a block (and O columns) this warp takes
-    const int qd = warp & 3;         // TMEM lane quarter this warp may access
+    const int sub = (warp - 2) >> 2;  // which 32 keys of a block (and O columns) this warp takes
+    const int qd = warp & 3;          // TMEM lane quarter this warp may access
     const int r = qd * 32 + lane;
     const int qrow = q0 + r;
-    const int bar_id = 1 + qd;  // the two warps of this lane quarter
+    const int bar_id = 1 + qd;  // the four warps of this lane quarter
     const float sqv = (qrow < p.Sq) ? __ldg(p.sq + static_cast<int64_t>(bh) * p.Sq + qrow) : 0.0f;
     const float c = sqv * p.c_scale;  // >= 0
-    const uint32_t t_row = (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(hf * 64);
+    const uint32_t t_row = (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(sub * AT_SUB);
     const int sw = r & 7;
-    const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv + hf * 64;
-    float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * 64;
+    const int piece0 = (sub & 1) * 4;  // this warp's 32 keys: four 16-byte pieces of a P half's row
+    const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv + sub * AT_SUB;
+    float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * AT_SUB;
     float* mxb = reinterpret_cast<float*>(smem + L::kOffMx);
     float* lsb = reinterpret_cast<float*>(smem + L::kOffLs);
     float m_ref = 0.0f;
     float l = 0.0f;
     bool ok = true;
-    // lane loads the scales of keys 2 * lane, 2 * lane + 1 of this warp's half, one block ahead
-    float2 skn;
-    skn.x = (hf * 64 + 2 * lane < p.Skv) ? __ldg(skh + 2 * lane) : 0.0f;
-    skn.y = (hf * 64 + 2 * lane + 1 < p.Skv) ? __ldg(skh + 2 * lane + 1) : 0.0f;
+    // lane loads the scale of key `lane` of this warp's 32, one block ahead
+    float skn = (sub * AT_SUB + lane < p.Skv) ? __ldg(skh + lane) : 0.0f;
     for (int j = 0; j < J; ++j) {
       const int b = j & 1;
-      float* skb = skw + b * 64;
-      *reinterpret_cast<float2*>(skb + 2 * lane) = skn;
+      float* skb = skw + b * AT_SUB;
+      skb[lane] = skn;
       {
-        const int kn = (j + 1) * AT_BK + hf * 64 + 2 * lane;
-        skn.x = (j + 1 < J && kn < p.Skv) ? __ldg(skh + (j + 1) * AT_BK + 2 * lane) : 0.0f;
-        skn.y = (j + 1 < J && kn + 1 < p.Skv) ? __ldg(skh + (j + 1) * AT_BK + 2 * lane + 1) : 0.0f;
+        const int kn = (j + 1) * AT_BK + sub * AT_SUB + lane;
+        skn = (j + 1 < J && kn < p.Skv) ? __ldg(skh + (j + 1) * AT_BK + lane) : 0.0f;
       }
       __syncwarp();  // the block's key scales are in this warp's buffer
-      int nvalid = p.Skv - j * AT_BK - hf * 64;  // valid keys among this warp's 64
-      nvalid = nvalid < 0 ? 0 : (nvalid > 64 ? 64 : nvalid);
-      uint8_t* prow = smem + L::kOffP + b * kPBytes + hf * kHalf + r * 128;
+      int nvalid = p.Skv - j * AT_BK - sub * AT_SUB;  // valid keys among this warp's 32
+      nvalid = nvalid < 0 ? 0 : (nvalid > AT_SUB ? AT_SUB : nvalid);
+      uint8_t* prow = smem + L::kOffP + b * kPBytes + (sub >> 1) * kHalf + r * 128;
       const uint32_t t_s = tmem_base + static_cast<uint32_t>(b * 128) + t_row;
 
       // S_j is in TMEM. P buffer b was last read by P V of block j-2, which was
@@ -400,14 +402,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       float bl = 0.0f;
       if (ok) {
         if (j == 0)  // the first block sets the reference maximum: its maximum first
-          softmax_pass_any<false>(t_s, skb, c, 0.0f, nvalid, prow, sw, &mh);
+          softmax_pass_any<false>(t_s, skb, c, 0.0f, nvalid, prow, piece0, sw, &mh);
         else  // later blocks: probabilities against the current reference, maximum alongside
-          bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &mh);
+          bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, piece0, sw, &mh);
       }
-      // the row's block maximum over both halves (every block has a valid key)
-      mxb[(b * 2 + hf) * AT_BQ + r] = mh;
-      pair_bar(bar_id);
-      const float t_max = c * fmaxf(mh, mxb[(b * 2 + (hf ^ 1)) * AT_BQ + r]);
+      // the row's block maximum over its four parts (every block has a valid key)
+      mxb[(b * 4 + sub) * AT_BQ + r] = mh;
+      quarter_bar(bar_id);
+      const float* mrow = mxb + b * 4 * AT_BQ + r;
+      const float t_max = c * fmaxf(fmaxf(mrow[0], mrow[AT_BQ]), fmaxf(mrow[2 * AT_BQ], mrow[3 * AT_BQ]));
       float alpha = 1.0f;
       bool need = false;   // O has to follow a raised reference
       bool redo = j == 0;  // P has to be (re)written against the new reference
@@ -424,7 +427,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         // move and the pass writes the same probabilities again.
         if (__any_sync(0xFFFFFFFFu, redo)) {
           float unused;
-          const float bl2 = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, sw, &unused);
+          const float bl2 = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, piece0, sw, &unused);
           if (redo) bl = bl2;
         }
         l = l * alpha + bl;
@@ -437,22 +440,19 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       if (ok && j >= 1) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns);
       if (ok) {
         tc_fence_after();
-        // this warp's 64 columns of O to the new reference maximum before this block's P V adds to them
+        // this warp's 32 columns of O to the new reference maximum before this block's P V adds to them
         if (__any_sync(0xFFFFFFFFu, need)) {
           const float2 a2 = make_float2(alpha, alpha);
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tO + t_row, o);
+          tmem_ld_wait_regs(o);
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o[16];
-            tmem_ld_32x32b_x16(tO + t_row + ch * 16, o);
-            tmem_ld_wait_regs16(o);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2);
-              o[2 * i] = __float_as_uint(v.x);
-              o[2 * i + 1] = __float_as_uint(v.y);
-            }
-            tmem_st_32x32b_x16(tO + t_row + ch * 16, o);
+          for (int i = 0; i < 16; ++i) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2);
+            o[2 * i] = __float_as_uint(v.x);
+            o[2 * i + 1] = __float_as_uint(v.y);
           }
+          tmem_st_32x32b_x32(tO + t_row, o);
           tmem_st_wait();
         }
         // P is read by the tensor cores (async proxy); O's rescale is complete
@@ -463,27 +463,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
     }
     if (ok) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((J - 1) & 1), abort, p.timeout_ns);
-    // the row sum over both halves
-    lsb[hf * AT_BQ + r] = l;
-    pair_bar(bar_id);
-    const float inv = 1.0f / (l + lsb[(hf ^ 1) * AT_BQ + r]);
+    // the row sum over the four parts
+    lsb[sub * AT_BQ + r] = l;
+    quarter_bar(bar_id);
+    const float inv = 1.0f / ((lsb[r] + lsb[AT_BQ + r]) + (lsb[2 * AT_BQ + r] + lsb[3 * AT_BQ + r]));
     if (ok) {
       tc_fence_after();
-      uint16_t* orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qrow) * AT_D + hf * 64;
+      uint16_t* orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qrow) * AT_D + sub * AT_SUB;
+      uint32_t o[32];
+      tmem_ld_32x32b_x32(tO + t_row, o);
+      tmem_ld_wait_regs(o);
+      uint32_t w[16];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t o[16];
-        tmem_ld_32x32b_x16(tO + t_row + ch * 16, o);
-        tmem_ld_wait_regs16(o);
-        uint32_t w[8];
+      for (int i = 0; i < 16; ++i)
+        w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+      if (qrow < p.Sq) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (qrow < p.Sq) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 16);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
     if (!ok && lane == 0) attn_abort(abort, p.status);

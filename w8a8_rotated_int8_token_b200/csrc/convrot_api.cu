@@ -35,9 +35,14 @@ struct LinearWs {
   bool split;
 };
 
+#ifndef CONVROT_SMALLM_SPLIT
+#define CONVROT_SMALLM_SPLIT 1
+#endif
+
 // Whether convrot_linear runs the weight-streaming GEMM split over all SMs.
 bool linear_uses_split(int64_t M, int64_t N) {
-  return M >= 1 && M <= convrot::kSmallM && (N + 127) / 128 <= convrot::kMaxSplitTiles;
+  return CONVROT_SMALLM_SPLIT != 0 && M >= 1 && M <= convrot::kSmallM &&
+         (N + 127) / 128 <= convrot::kMaxSplitTiles;
 }
 
 LinearWs linear_ws_layout(int64_t M, int64_t K, int64_t N) {
