@@ -138,10 +138,10 @@ CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K
  *   ws       device workspace, 256-byte aligned, ws_bytes >=
  *            convrot_linear_workspace_bytes(M, N, K, g). It holds the status
  *            word, per-128-token readiness counters, the token scales and the
- *            int8 activation codes of this call, and for M <= 64 (the
- *            weight-streaming GEMM, split over all SMs) one arrival counter per
- *            128 weight rows and 2 * 160 slots of 128 x (16, 32 or 64) int32
- *            partial sums; calls that may run at the same time need separate
+ *            int8 activation codes of this call, and for M <= 64 with
+ *            N <= 8192 (the weight-streaming GEMM split over all SMs) one
+ *            arrival counter per 128 weight rows and 2 * 160 slots of
+ *            128 x (16, 32 or 64) int32 partial sums; calls that may run at the same time need separate
  *            workspaces. Its contents need no initialisation (the readiness
  *            counters carry a per-call tag; the first kernel of a call zeroes
  *            the arrival counters).

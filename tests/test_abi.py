@@ -54,14 +54,15 @@ def test_library_exports_nothing_else():
 
 def linear_ws_layout(M, K, N=None):
     """Byte layout of convrot_linear's workspace, as include/convrot.h describes it
-    (the split buffers of the weight-streaming GEMM, for 1 <= M <= 64, when N is given)."""
+    (the split buffers of the weight-streaming GEMM, for 1 <= M <= 64 and at most 64 weight
+    tiles of 128 rows, when N is given)."""
     up = lambda v, a: (v + a - 1) // a * a  # noqa: E731
     ready = 256
     scale = up(ready + 8 * ((M + 127) // 128), 256)
     codes = up(scale + 4 * M, 1024)
     total = up(codes + M * K, 256)
     lay = {"ready": ready, "scale": scale, "codes": codes, "total": total}
-    if N is not None and 1 <= M <= 64 and (N + 127) // 128 <= 4096:
+    if N is not None and 1 <= M <= 64 and (N + 127) // 128 <= 64:
         bnt = 16 if M <= 16 else (32 if M <= 32 else 64)
         lay["split_count"] = total
         lay["split_part"] = up(total + 4 * ((N + 127) // 128), 1024)
@@ -89,7 +90,8 @@ def test_workspace_sizes(L):
     assert L.convrot_linear_workspace_bytes(0, N, K, 256) == linear_ws_layout(0, K, N)["total"]  # M = 0 is valid
     # the weight-streaming GEMM's split buffers (M <= 64)
     for m in (1, 16, 17, 33, 64, 65):
-        assert L.convrot_linear_workspace_bytes(m, 12288, 4096, 128) == linear_ws_layout(m, 4096, 12288)["total"]
+        for n in (12288, 4096, 8192, 8200):
+            assert L.convrot_linear_workspace_bytes(m, n, 4096, 128) == linear_ws_layout(m, 4096, n)["total"]
     assert L.convrot_linear_workspace_bytes(-1, N, K, 256) == 0
     assert L.convrot_gemm_workspace_bytes() == 256
     assert L.convrot_prepare_weight_workspace_bytes() >= 4

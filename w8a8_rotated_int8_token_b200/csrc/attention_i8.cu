@@ -12,40 +12,29 @@
 //
 // One call: Q and K through the rotate+quantise kernel (codes + one scale per
 // token), V transposed once into key-contiguous rows (the K-major B operand of
-// the P V product), then one CTA per SM at a time, each on one
-// (batch*head, 128-query tile):
+// the P V product), then one CTA per (batch*head, 128-query tile):
 //   warp 0, one lane : TMA producer: the tile's 128 x 128 query codes once,
-//                      then per 128-key block j the key codes into stage j%2
-//                      (once S of block j-2 is computed) and the transposed
-//                      values, two 64-key halves, into stage j%2 (once P V of
-//                      block j-2 is done).
-//   warp 1           : allocates 512 TMEM columns; one lane issues
-//                      S_j = Qq Kq_j^T (tcgen05.mma kind::i8, M = N = 128,
-//                      K = 4 x 32) into S buffer j%2 (TMEM columns 0..127 or
-//                      128..255) and O += P_j V_j (kind::f16 with bf16
-//                      operands, M = N = 128, K = 8 x 16) into columns
-//                      256..383, in the order S_0, S_1, PV_0, S_2, PV_1, ...
-//   warps 2..17      : softmax, four warps per query row (TMEM lane), each
-//                      taking 32 keys of every block and 32 O columns. One pass per
-//                      block straight from TMEM: t = c_i s_k[j] S_ij in base-2
-//                      units (c_i = s_q[i] softmax_scale log2(e)),
-//                      p = 2^(t - m) against the current reference maximum m
-//                      (packed f32x2 arithmetic), P rounded to bf16 into the
-//                      128-byte-swizzled P buffer j%2, the row sums in
-//                      float32; the block maximum of the row is combined
-//                      across the four warps through shared memory. When a block
-//                      raises the maximum by more than 8 (p would pass 256)
-//                      the reference moves, the block's pass is redone (S is
-//                      still in TMEM) and O is rescaled in TMEM once the
-//                      previous block's P V is done. The four warps of a row
-//                      meet at a named barrier every block, also after a
-//                      timed-out wait (they then skip the work), so none can
-//                      be left waiting for another. At the end
-//                      O / (sum of the four parts) is rounded to bf16 and stored.
-// Every buffer is double: the next block's QK^T and loads run while this
-// block's softmax runs on the CUDA cores and the previous block's P V on the
-// tensor cores. Every mbarrier is waited on phase by phase in order, and every
-// wait is bounded (status word + abort flag, as in the GEMM).
+//                      then per 128-key block the key codes (loaded as soon
+//                      as the previous block's S is computed) and the
+//                      transposed values (two 64-key halves, loaded as soon
+//                      as the previous block's P V is done).
+//   warp 1           : allocates 256 TMEM columns; one lane issues
+//                      S = Qq Kq^T (tcgen05.mma kind::i8, M = N = 128,
+//                      K = 4 x 32) into TMEM columns 0..127 and
+//                      O += P V (kind::f16 with bf16 operands, M = N = 128,
+//                      K = 8 x 16) into columns 128..255.
+//   warps 2..5       : softmax, one query row per thread (TMEM lane): S from
+//                      TMEM, t = c_i s_k[j] S_ij in base-2 units with
+//                      c_i = s_q[i] softmax_scale log2(e), p = 2^(t - m) in
+//                      float32, the row sum in float32, P rounded to bf16 into
+//                      128-byte-swizzled shared memory for the MMA. The
+//                      reference maximum m moves only when a block raises it
+//                      by more than 8 (p <= 256), and then O is rescaled in
+//                      TMEM once the previous block's P V has finished. At
+//                      the end O / sum is rounded to bf16 and stored.
+// S is read out of TMEM before the next block's S is written, so the next
+// QK^T runs on the tensor cores while this block's softmax runs on the CUDA
+// cores. Every wait is bounded (status word + abort flag, as in the GEMM).
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -67,9 +56,7 @@ namespace {
 constexpr int AT_BQ = 128;  // queries per CTA tile
 constexpr int AT_BK = 128;  // keys per block
 constexpr int AT_D = 128;   // head dimension
-constexpr int AT_SOFTMAX_WARPS = 16;  // four per TMEM lane quarter: 32 keys (and 32 O columns) each
-constexpr int AT_SUB = 32;            // keys of a block (and O columns) per softmax warp
-constexpr int AT_THREADS = 64 + 32 * AT_SOFTMAX_WARPS;
+constexpr int AT_THREADS = 192;
 constexpr int kQBytes = AT_BQ * AT_D;      // int8 query codes: 16 KB
 constexpr int kKBytes = AT_BK * AT_D;      // int8 key codes of one block: 16 KB
 constexpr int kHalf = 128 * 128;           // one 64-key half of a bf16 operand: 128 rows x 128 B
@@ -80,17 +67,17 @@ constexpr uint32_t IDESC_O = idesc_bf16(AT_BQ, AT_D);
 constexpr int kTimeoutStatus = 5;
 constexpr float kRescaleThreshold = 8.0f;  // base-2 units: probabilities stay below 2^8
 
+// 2 CTAs per SM: everything below (plus the alignment slack) stays under
+// half of the SM's 228 KB of shared memory.
 struct AttnSmem {
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;       // two stages
-  static constexpr int kOffV = kOffK + 2 * kKBytes;   // two stages
-  static constexpr int kOffP = kOffV + 2 * kVBytes;   // two buffers
-  static constexpr int kOffSk = kOffP + 2 * kPBytes;  // per softmax warp, two buffers of its 32 key scales
-  static constexpr int kOffMx = kOffSk + AT_SOFTMAX_WARPS * 2 * AT_SUB * 4;  // [2 blocks][4 parts][128 rows] maxima
-  static constexpr int kOffLs = kOffMx + 2 * 4 * AT_BQ * 4;                  // [4 parts][128 rows] row sums
-  static constexpr int kOffBar = kOffLs + 4 * AT_BQ * 4;
-  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2], p_full, o_done, drain
-  static constexpr int kNumBars = 16;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kKBytes;
+  static constexpr int kOffP = kOffV + kVBytes;
+  static constexpr int kOffSk = kOffP + kPBytes;  // per softmax warp, two buffers of a block's key scales
+  static constexpr int kOffBar = kOffSk + 4 * 2 * AT_BK * 4;
+  // q_full, k_full, k_empty, v_full, v_empty, s_full, s_empty, p_full, o_done, drain
+  static constexpr int kNumBars = 10;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 8;
   static constexpr int kBytes = kOffAbort + 8;
@@ -132,77 +119,36 @@ __device__ __forceinline__ float small_int_to_float(uint32_t acc) {
   return __uint_as_float(acc + 0x4B400000u) - 12582912.0f;
 }
 
-// One pass over this thread's 32 logits of a block, straight from TMEM (both
-// 16-column loads in flight together): t = c * s_k[key] * S[row, key] (base-2
-// units); with WRITE_P the probabilities p = 2^(t - m_ref) are rounded to bf16
-// into the four 16-byte pieces `piece0`.. of the row's 128-byte-swizzled
-// shared-memory line and their float32 sum returned. The maximum over the
-// valid keys of s_k[key] * S[row, key] goes to *mh.
-template <bool WRITE_P, bool MASKED>
-__device__ __forceinline__ float softmax_pass(uint32_t t_s, const float* skb, float c, float m_ref, int nvalid,
-                                              uint8_t* row, int piece0, int sw, float* mh) {
-  const float2 mg = make_float2(-12582912.0f, -12582912.0f);
+// The probabilities of one row for 64 keys (one half), packed to bf16 into the
+// row's 128-byte-swizzled shared-memory line; returns their float32 sum.
+template <bool MASKED>
+__device__ __forceinline__ float write_p_half(const float (&u)[128], int h, float c, float m_ref, int nvalid,
+                                              uint8_t* row, int sw) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m_ref, -m_ref);
   float2 sum2 = make_float2(0.0f, 0.0f);
-  float ma = -INFINITY, mc = -INFINITY;
-  uint32_t a[2][16];
-  tmem_ld_32x32b_x16(t_s, a[0]);
-  tmem_ld_32x32b_x16(t_s + 16, a[1]);
-  tmem_ld_wait_regs16(a[0]);
-  tmem_ld_wait_regs16(a[1]);
 #pragma unroll
-  for (int ch = 0; ch < 2; ++ch) {
-    uint32_t w[8];
+  for (int i = 0; i < 8; ++i) {
+    uint32_t w[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int k = ch * 16 + 2 * i;  // key (within this warp's 32) of the pair's first element
-      // float(acc) for |acc| < 2^22: the integer added to the bits of 1.5 * 2^23, minus 1.5 * 2^23
-      const float2 x =
-          make_float2(__uint_as_float(a[ch][2 * i] + 0x4B400000u), __uint_as_float(a[ch][2 * i + 1] + 0x4B400000u));
-      const float2 u = __fmul2_rn(__fadd2_rn(x, mg), *reinterpret_cast<const float2*>(skb + k));
+    for (int e = 0; e < 4; ++e) {
+      const int k = h * 64 + i * 8 + 2 * e;
+      // t = c u - m for two keys at once, then p = 2^t
+      const float2 t = __ffma2_rn(c2, make_float2(u[k], u[k + 1]), nm2);
+      float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
       if (MASKED) {
-        ma = (k < nvalid) ? fmaxf(ma, u.x) : ma;
-        mc = (k + 1 < nvalid) ? fmaxf(mc, u.y) : mc;
-      } else if (i & 1) {
-        mc = fwht::fmax3f(mc, u.x, u.y);
-      } else {
-        ma = fwht::fmax3f(ma, u.x, u.y);
+        pp.x = (k < nvalid) ? pp.x : 0.0f;
+        pp.y = (k + 1 < nvalid) ? pp.y : 0.0f;
       }
-      if (WRITE_P) {
-        const float2 t = __ffma2_rn(c2, u, nm2);
-        float2 pp = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-        if (MASKED) {
-          pp.x = (k < nvalid) ? pp.x : 0.0f;
-          pp.y = (k + 1 < nvalid) ? pp.y : 0.0f;
-        }
-        sum2 = __fadd2_rn(sum2, pp);
-        w[i] = pack_bf16x2(pp.x, pp.y);
-      }
+      sum2 = __fadd2_rn(sum2, pp);
+      w[e] = pack_bf16x2(pp.x, pp.y);
     }
-    if (WRITE_P) {  // keys 16 ch .. 16 ch + 15 of this warp: pieces piece0 + 2 ch, piece0 + 2 ch + 1
-      *reinterpret_cast<uint4*>(row + (((piece0 + 2 * ch) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(row + (((piece0 + 2 * ch + 1) ^ sw) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
-    }
+    *reinterpret_cast<uint4*>(row + ((i ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  *mh = fmaxf(ma, mc);
   return sum2.x + sum2.y;
 }
 
-template <bool WRITE_P>
-__device__ __forceinline__ float softmax_pass_any(uint32_t t_s, const float* skb, float c, float m_ref, int nvalid,
-                                                  uint8_t* row, int piece0, int sw, float* mh) {
-  return nvalid == AT_SUB ? softmax_pass<WRITE_P, false>(t_s, skb, c, m_ref, nvalid, row, piece0, sw, mh)
-                          : softmax_pass<WRITE_P, true>(t_s, skb, c, m_ref, nvalid, row, piece0, sw, mh);
-}
-
-// The four softmax warps of one TMEM lane quarter (128 threads) meet here. The
-// non-aligned form: a warp need not arrive converged.
-__device__ __forceinline__ void quarter_bar(int id) {
-  asm volatile("barrier.sync %0, 128;" ::"r"(id) : "memory");
-}
-
-__global__ void __launch_bounds__(AT_THREADS, 1)
+__global__ void __launch_bounds__(AT_THREADS, 2)
     attention_i8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using L = AttnSmem;
@@ -210,15 +156,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2]
-  uint64_t* s_empty = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* o_done = bars + 14;
-  uint64_t* drain = bars + 15;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_empty = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* o_done = bars + 8;
+  uint64_t* drain = bars + 9;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
 
@@ -233,114 +179,104 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     mbar_init(q_full, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&k_full[b], 1);
-      mbar_init(&k_empty[b], 1);
-      mbar_init(&v_full[b], 1);
-      mbar_init(&v_empty[b], 1);
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], AT_SOFTMAX_WARPS);  // every softmax warp
-    }
-    mbar_init(p_full, AT_SOFTMAX_WARPS);
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 4);  // the four softmax warps
+    mbar_init(p_full, 4);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_ptr, 512);
+    tmem_alloc(tmem_ptr, 256);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
-  const uint32_t tO = tmem_base + 256;  // O: columns 256..383; S buffer b: columns 128 b ..
+  const uint32_t tS = tmem_base;        // S: columns 0..127
+  const uint32_t tO = tmem_base + 128;  // O: columns 128..255
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Tensor-pipe order is S_0, S_1, PV_0, S_2, PV_1, ...: K_{j+1} goes out
+    // when S_j is done, V_{j+1} when PV_j is done.
     if (lane == 0) {
       bool ok = true;
       int issued_k = 0, issued_v = 0;
       auto load_k = [&](int j) {
-        const int b = j & 1;
-        mbar_arrive_expect_tx(&k_full[b], kKBytes);
-        tma_load_3d(smem + L::kOffK + b * kKBytes, &tmK, &k_full[b], 0, j * AT_BK, bh);
+        mbar_arrive_expect_tx(k_full, kKBytes);
+        tma_load_3d(smem + L::kOffK, &tmK, k_full, 0, j * AT_BK, bh);
         issued_k = j + 1;
       };
       auto load_v = [&](int j) {
-        const int b = j & 1;
-        uint8_t* dst = smem + L::kOffV + b * kVBytes;
-        mbar_arrive_expect_tx(&v_full[b], kVBytes);
-        tma_load_3d(dst, &tmV, &v_full[b], j * AT_BK, 0, bh);
-        tma_load_3d(dst + kHalf, &tmV, &v_full[b], j * AT_BK + 64, 0, bh);
+        mbar_arrive_expect_tx(v_full, kVBytes);
+        tma_load_3d(smem + L::kOffV, &tmV, v_full, j * AT_BK, 0, bh);
+        tma_load_3d(smem + L::kOffV + kHalf, &tmV, v_full, j * AT_BK + 64, 0, bh);
         issued_v = j + 1;
       };
       mbar_arrive_expect_tx(q_full, kQBytes);
       tma_load_3d(smem + L::kOffQ, &tmQ, q_full, 0, q0, bh);
       load_k(0);
       load_v(0);
-      if (J > 1) {
-        load_k(1);
-        load_v(1);
-      }
-      for (int j = 0; j + 2 < J; ++j) {
-        // stage j%2 again once block j is done with it (the (j/2)-th use of the stage)
-        const uint32_t par = static_cast<uint32_t>((j >> 1) & 1);
-        if (!mbar_wait_bounded(&k_empty[j & 1], par, abort, p.timeout_ns)) {
+      for (int j = 0; j + 1 < J; ++j) {
+        if (!mbar_wait_bounded(k_empty, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
           ok = false;
           break;
         }
-        load_k(j + 2);
-        if (!mbar_wait_bounded(&v_empty[j & 1], par, abort, p.timeout_ns)) {
+        load_k(j + 1);
+        if (!mbar_wait_bounded(v_empty, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
           ok = false;
           break;
         }
-        load_v(j + 2);
+        load_v(j + 1);
       }
       if (!ok) {
         attn_abort(abort, p.status);
         // every copy already issued lands before the shared memory goes away
         mbar_wait_bounded(q_full, 0u, nullptr, p.timeout_ns);
-        for (int j = (issued_k > 2 ? issued_k - 2 : 0); j < issued_k; ++j)
-          mbar_wait_bounded(&k_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), nullptr, p.timeout_ns);
-        for (int j = (issued_v > 2 ? issued_v - 2 : 0); j < issued_v; ++j)
-          mbar_wait_bounded(&v_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), nullptr, p.timeout_ns);
+        if (issued_k > 0) mbar_wait_bounded(k_full, static_cast<uint32_t>((issued_k - 1) & 1), nullptr, p.timeout_ns);
+        if (issued_v > 0) mbar_wait_bounded(v_full, static_cast<uint32_t>((issued_v - 1) & 1), nullptr, p.timeout_ns);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t qa = smem_addr(smem + L::kOffQ);
+      const uint32_t pa = smem_addr(smem + L::kOffP);
+      const uint32_t va = smem_addr(smem + L::kOffV);
+      const uint32_t kb = smem_addr(smem + L::kOffK);
       auto mma_s = [&](int j) -> bool {
-        const int b = j & 1;
-        const uint32_t par = static_cast<uint32_t>((j >> 1) & 1);
-        // S buffer b free (the softmax of block j-2 has read it) and K_j landed
-        if (j >= 2 && !mbar_wait_bounded(&s_empty[b], par ^ 1u, abort, p.timeout_ns)) return false;
-        if (!mbar_wait_bounded(&k_full[b], par, abort, p.timeout_ns)) return false;
+        if (!mbar_wait_bounded(k_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) return false;
         tc_fence_after();
-        const uint32_t kb = smem_addr(smem + L::kOffK + b * kKBytes);
-        const uint32_t ts = tmem_base + static_cast<uint32_t>(b * 128);
 #pragma unroll
         for (int k = 0; k < AT_D / 32; ++k)
-          mma_i8(ts, smem_desc_k_sw128(qa + k * 32), smem_desc_k_sw128(kb + k * 32), IDESC_S, k > 0 ? 1u : 0u);
-        mma_commit(&s_full[b]);
-        mma_commit(&k_empty[b]);
+          mma_i8(tS, smem_desc_k_sw128(qa + k * 32), smem_desc_k_sw128(kb + k * 32), IDESC_S, k > 0 ? 1u : 0u);
+        mma_commit(s_full);
+        mma_commit(k_empty);
         return true;
       };
       bool ok = mbar_wait_bounded(q_full, 0u, abort, p.timeout_ns);
       if (ok) ok = mma_s(0);
-      if (ok && J > 1) ok = mma_s(1);
       for (int j = 0; j < J && ok; ++j) {
-        const int b = j & 1;
+        if (j + 1 < J) {
+          // S_{j+1} once the softmax has read S_j out of TMEM
+          if (!mbar_wait_bounded(s_empty, static_cast<uint32_t>(j & 1), abort, p.timeout_ns) || !mma_s(j + 1)) {
+            ok = false;
+            break;
+          }
+        }
         if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns) ||
-            !mbar_wait_bounded(&v_full[b], static_cast<uint32_t>((j >> 1) & 1), abort, p.timeout_ns)) {
+            !mbar_wait_bounded(v_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t pa = smem_addr(smem + L::kOffP + b * kPBytes);
-        const uint32_t va = smem_addr(smem + L::kOffV + b * kVBytes);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -348,11 +284,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             mma_bf16(tO, smem_desc_k_sw128(pa + h * kHalf + k * 32), smem_desc_k_sw128(va + h * kHalf + k * 32),
                      IDESC_O, (j | h | k) != 0 ? 1u : 0u);
         mma_commit(o_done);
-        mma_commit(&v_empty[b]);
-        if (j + 2 < J && !mma_s(j + 2)) {
-          ok = false;
-          break;
-        }
+        mma_commit(v_empty);
       }
       if (!ok) attn_abort(abort, p.status);
       // every MMA this thread issued has finished before TMEM is released
@@ -361,126 +293,161 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int sub = (warp - 2) >> 2;  // which 32 keys of a block (and O columns) this warp takes
-    const int qd = warp & 3;          // TMEM lane quarter this warp may access
+    const int qd = warp & 3;  // TMEM lane quarter this warp may access
     const int r = qd * 32 + lane;
     const int qrow = q0 + r;
-    const int bar_id = 1 + qd;  // the four warps of this lane quarter
     const float sqv = (qrow < p.Sq) ? __ldg(p.sq + static_cast<int64_t>(bh) * p.Sq + qrow) : 0.0f;
     const float c = sqv * p.c_scale;  // >= 0
-    const uint32_t t_row = (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(sub * AT_SUB);
+    const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
+    uint8_t* prow = smem + L::kOffP + r * 128;
     const int sw = r & 7;
-    const int piece0 = (sub & 1) * 4;  // this warp's 32 keys: four 16-byte pieces of a P half's row
-    const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv + sub * AT_SUB;
-    float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * AT_SUB;
-    float* mxb = reinterpret_cast<float*>(smem + L::kOffMx);
-    float* lsb = reinterpret_cast<float*>(smem + L::kOffLs);
+    const float* skh = p.sk + static_cast<int64_t>(bh) * p.Skv;
+    // this warp's two buffers of a block's 128 key scales (no barrier across warps)
+    float* skw = reinterpret_cast<float*>(smem + L::kOffSk) + (warp - 2) * 2 * AT_BK;
     float m_ref = 0.0f;
     float l = 0.0f;
     bool ok = true;
-    // lane loads the scale of key `lane` of this warp's 32, one block ahead
-    float skn = (sub * AT_SUB + lane < p.Skv) ? __ldg(skh + lane) : 0.0f;
+    // lane loads keys 4 * lane .. 4 * lane + 3 of each block, one block ahead
+    float skn[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) skn[e] = (4 * lane + e < p.Skv) ? __ldg(skh + 4 * lane + e) : 0.0f;
     for (int j = 0; j < J; ++j) {
-      const int b = j & 1;
-      float* skb = skw + b * AT_SUB;
-      skb[lane] = skn;
-      {
-        const int kn = (j + 1) * AT_BK + sub * AT_SUB + lane;
-        skn = (j + 1 < J && kn < p.Skv) ? __ldg(skh + (j + 1) * AT_BK + lane) : 0.0f;
+      float* skb = skw + (j & 1) * AT_BK;
+      *reinterpret_cast<float4*>(skb + 4 * lane) = make_float4(skn[0], skn[1], skn[2], skn[3]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kn = (j + 1) * AT_BK + 4 * lane + e;
+        skn[e] = (j + 1 < J && kn < p.Skv) ? __ldg(skh + kn) : 0.0f;
       }
       __syncwarp();  // the block's key scales are in this warp's buffer
-      int nvalid = p.Skv - j * AT_BK - sub * AT_SUB;  // valid keys among this warp's 32
-      nvalid = nvalid < 0 ? 0 : (nvalid > AT_SUB ? AT_SUB : nvalid);
-      uint8_t* prow = smem + L::kOffP + b * kPBytes + (sub >> 1) * kHalf + r * 128;
-      const uint32_t t_s = tmem_base + static_cast<uint32_t>(b * 128) + t_row;
+      const int nvalid = (p.Skv - j * AT_BK) < AT_BK ? (p.Skv - j * AT_BK) : AT_BK;
 
-      // S_j is in TMEM. P buffer b was last read by P V of block j-2, which was
-      // done before this warp signalled block j-1 (it waited for it there).
-      if (ok) ok = warp_wait_bounded(&s_full[b], static_cast<uint32_t>((j >> 1) & 1), abort, p.timeout_ns);
-      if (ok) tc_fence_after();
-      float mh = -INFINITY;
-      float bl = 0.0f;
-      if (ok) {
-        if (j == 0)  // the first block sets the reference maximum: its maximum first
-          softmax_pass_any<false>(t_s, skb, c, 0.0f, nvalid, prow, piece0, sw, &mh);
-        else  // later blocks: probabilities against the current reference, maximum alongside
-          bl = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, piece0, sw, &mh);
+      if (!warp_wait_bounded(s_full, static_cast<uint32_t>(j & 1), abort, p.timeout_ns)) {
+        ok = false;
+        break;
       }
-      // the row's block maximum over its four parts (every block has a valid key)
-      mxb[(b * 4 + sub) * AT_BQ + r] = mh;
-      quarter_bar(bar_id);
-      const float* mrow = mxb + b * 4 * AT_BQ + r;
-      const float t_max = c * fmaxf(fmaxf(mrow[0], mrow[AT_BQ]), fmaxf(mrow[2 * AT_BQ], mrow[3 * AT_BQ]));
+      tc_fence_after();
+      float u[128];  // s_k[key] * S[row, key]: the logit without the row factor c
+      {
+        // two 32-column loads in flight at a time, converted as they land
+        uint32_t a0[32], a1[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld_32x32b_x32(tS + lane_off + half * 64, a0);
+          tmem_ld_32x32b_x32(tS + lane_off + half * 64 + 32, a1);
+          tmem_ld_wait_regs(a0);
+          tmem_ld_wait_regs(a1);
+          if (half == 1) {
+            // S has been read: the next block's QK^T may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty);
+          }
+          // u = float(acc) * s_k, two keys per packed f32x2 operation
+          const float2 mg = make_float2(-12582912.0f, -12582912.0f);
+#pragma unroll
+          for (int k4 = 0; k4 < 16; ++k4) {
+            const float4 s4 = *reinterpret_cast<const float4*>(skb + half * 64 + 4 * k4);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int k = 4 * k4 + 2 * e;
+              const uint32_t acc0 = (k < 32) ? a0[k] : a1[k - 32];
+              const uint32_t acc1 = (k + 1 < 32) ? a0[k + 1] : a1[k - 31];
+              // float(acc) for |acc| < 2^22: the integer added to the bits of 1.5 * 2^23, minus 1.5 * 2^23
+              const float2 x = make_float2(__uint_as_float(acc0 + 0x4B400000u), __uint_as_float(acc1 + 0x4B400000u));
+              const float2 v = __fmul2_rn(__fadd2_rn(x, mg), e == 0 ? make_float2(s4.x, s4.y) : make_float2(s4.z, s4.w));
+              u[half * 64 + k] = v.x;
+              u[half * 64 + k + 1] = v.y;
+            }
+          }
+        }
+      }
+      // the block maximum over its valid keys, in base-2 units
+      float mb;
+      if (nvalid == AT_BK) {
+        // 128 -> 43 -> 15 -> 5 -> 1 with three-input maxima
+        float a[43], b[15], c5[5];
+#pragma unroll
+        for (int i = 0; i < 42; ++i) a[i] = fwht::fmax3f(u[3 * i], u[3 * i + 1], u[3 * i + 2]);
+        a[42] = fmaxf(u[126], u[127]);
+#pragma unroll
+        for (int i = 0; i < 14; ++i) b[i] = fwht::fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        b[14] = a[42];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) c5[i] = fwht::fmax3f(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+        mb = fmaxf(fwht::fmax3f(c5[0], c5[1], c5[2]), fmaxf(c5[3], c5[4]));
+      } else {
+        mb = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < AT_BK; ++k) mb = (k < nvalid) ? fmaxf(mb, u[k]) : mb;
+      }
+      const float t_max = c * mb;
       float alpha = 1.0f;
-      bool need = false;   // O has to follow a raised reference
-      bool redo = j == 0;  // P has to be (re)written against the new reference
+      bool need = false;
       if (j == 0) {
         m_ref = t_max;
       } else if (t_max > m_ref + kRescaleThreshold) {
         alpha = ex2_approx(m_ref - t_max);
         m_ref = t_max;
-        need = redo = true;
+        need = true;
       }
-      if (ok) {
-        // The pass reads TMEM with warp-collective loads, so the whole warp runs
-        // it when any of its rows needs it; for the others the reference did not
-        // move and the pass writes the same probabilities again.
-        if (__any_sync(0xFFFFFFFFu, redo)) {
-          float unused;
-          const float bl2 = softmax_pass_any<true>(t_s, skb, c, m_ref, nvalid, prow, piece0, sw, &unused);
-          if (redo) bl = bl2;
-        }
-        l = l * alpha + bl;
-        // S_j has been read: its buffer may take S_{j+2}
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[b]);
+      // the previous block's P V has finished: O is stable and the P buffer free
+      if (j >= 1 && !warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns)) {
+        ok = false;
+        break;
       }
-      // P V of block j-1 is done: O is stable (and, for block j+1, P buffer b^1 is free)
-      if (ok && j >= 1) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((j - 1) & 1), abort, p.timeout_ns);
-      if (ok) {
-        tc_fence_after();
-        // this warp's 32 columns of O to the new reference maximum before this block's P V adds to them
-        if (__any_sync(0xFFFFFFFFu, need)) {
-          const float2 a2 = make_float2(alpha, alpha);
+      tc_fence_after();
+      float bl;
+      if (nvalid == AT_BK) {
+        bl = write_p_half<false>(u, 0, c, m_ref, nvalid, prow, sw) +
+             write_p_half<false>(u, 1, c, m_ref, nvalid, prow + kHalf, sw);
+      } else {
+        bl = write_p_half<true>(u, 0, c, m_ref, nvalid, prow, sw) +
+             write_p_half<true>(u, 1, c, m_ref, nvalid, prow + kHalf, sw);
+      }
+      l = l * alpha + bl;
+      // O to the new reference maximum before this block's P V adds to it
+      // (after the P writes, so that the logits are no longer live)
+      if (__any_sync(0xFFFFFFFFu, need)) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
           uint32_t o[32];
-          tmem_ld_32x32b_x32(tO + t_row, o);
+          tmem_ld_32x32b_x32(tO + lane_off + ch * 32, o);
           tmem_ld_wait_regs(o);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2);
-            o[2 * i] = __float_as_uint(v.x);
-            o[2 * i + 1] = __float_as_uint(v.y);
-          }
-          tmem_st_32x32b_x32(tO + t_row, o);
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_32x32b_x32(tO + lane_off + ch * 32, o);
         }
-        // P is read by the tensor cores (async proxy); O's rescale is complete
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        tmem_st_wait();
       }
+      // P is read by the tensor cores (async proxy); O's rescale is complete
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok) ok = warp_wait_bounded(o_done, static_cast<uint32_t>((J - 1) & 1), abort, p.timeout_ns);
-    // the row sum over the four parts
-    lsb[sub * AT_BQ + r] = l;
-    quarter_bar(bar_id);
-    const float inv = 1.0f / ((lsb[r] + lsb[AT_BQ + r]) + (lsb[2 * AT_BQ + r] + lsb[3 * AT_BQ + r]));
     if (ok) {
-      tc_fence_after();
-      uint16_t* orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qrow) * AT_D + sub * AT_SUB;
-      uint32_t o[32];
-      tmem_ld_32x32b_x32(tO + t_row, o);
-      tmem_ld_wait_regs(o);
-      uint32_t w[16];
+      if (!warp_wait_bounded(o_done, static_cast<uint32_t>((J - 1) & 1), abort, p.timeout_ns)) {
+        ok = false;
+      } else {
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        uint16_t* orow = p.O + (static_cast<int64_t>(bh) * p.Sq + qrow) * AT_D;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-      if (qrow < p.Sq) {
-        uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tO + lane_off + ch * 32, o);
+          tmem_ld_wait_regs(o);
+          uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+          if (qrow < p.Sq) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
       }
     }
     if (!ok && lane == 0) attn_abort(abort, p.status);
@@ -489,7 +456,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, 256);
   }
 }
 

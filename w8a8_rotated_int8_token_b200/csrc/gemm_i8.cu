@@ -970,11 +970,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 
 constexpr int SM_BW = 128;  // weight rows per tile
 
-template <int BNT>
+// KPS: consecutive 128-byte k-blocks per ring stage (one TMA box each), so
+// that each weight row is read in runs of KPS * 128 bytes.
+#ifndef CONVROT_SMALLM_KPS
+#define CONVROT_SMALLM_KPS 2
+#endif
+
+template <int BNT, int KPS = 1>
 struct SmallSmem {
-  static constexpr int kW = SM_BW * BK;  // 16 KB
-  static constexpr int kX = BNT * BK;    // 2..8 KB
-  static constexpr int kFit = (200 * 1024) / (kW + kX);
+  static constexpr int kW1 = SM_BW * BK;  // 16 KB: one weight k-block
+  static constexpr int kX1 = BNT * BK;    // 2..8 KB: one token k-block
+  static constexpr int kW = kW1 * KPS;
+  static constexpr int kX = kX1 * KPS;
+  static constexpr int kFit = (KPS == 1 ? 200 * 1024 : 216 * 1024) / (kW + kX);
 #ifdef CONVROT_SMALLM_STAGES
   static constexpr int kStages = CONVROT_SMALLM_STAGES < kFit ? CONVROT_SMALLM_STAGES : kFit;
 #else
@@ -1059,11 +1067,11 @@ __device__ __forceinline__ void smallm_store(const GemmParams& p, void* out, int
   }
 }
 
-template <int EPI, int BNT>
+template <int EPI, int BNT, int KPS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                           void* __restrict__ out, const int8_t* __restrict__ Wq, const GemmParams p) {
-  using L = SmallSmem<BNT>;
+  using L = SmallSmem<BNT, KPS>;
   constexpr int S = L::kStages;
   constexpr uint32_t kIdesc = idesc_i8(SM_BW, BNT);
   extern __shared__ uint8_t smem_raw[];
@@ -1120,23 +1128,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int early_s[S], early_kb[S];
       int n_early = 0;
       bool waited = false;
+      auto load_x = [&](int st, int kb) {
+#pragma unroll
+        for (int i = 0; i < KPS; ++i)
+          tma_load_2d(smem + L::kOffX + st * L::kX + i * L::kX1, &tmX, &full[st], (kb + i) * BK, 0);
+      };
       auto release_early = [&]() {
         griddep_wait();
         waited = true;
-        for (int i = 0; i < n_early; ++i)
-          tma_load_2d(smem + L::kOffX + early_s[i] * L::kX, &tmX, &full[early_s[i]], early_kb[i] * BK, 0);
+        for (int i = 0; i < n_early; ++i) load_x(early_s[i], early_kb[i]);
       };
       int tile, k0, k1;
       while (ok && seg.get(tile, k0, k1)) {
-        for (int kb = k0; kb < k1; ++kb) {
+        // KPS k-blocks per stage (blocks past K arrive as zeros: whole tiles only when KPS > 1)
+        for (int kb = k0; kb < k1; kb += KPS) {
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, abort, p.timeout_ns)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[s], L::kW + L::kX);
-          tma_load_2d(smem + L::kOffW + s * L::kW, &tmW, &full[s], kb * BK, tile * SM_BW);
+#pragma unroll
+          for (int i = 0; i < KPS; ++i)
+            tma_load_2d(smem + L::kOffW + s * L::kW + i * L::kW1, &tmW, &full[s], (kb + i) * BK, tile * SM_BW);
           if (waited) {
-            tma_load_2d(smem + L::kOffX + s * L::kX, &tmX, &full[s], kb * BK, 0);
+            load_x(s, kb);
           } else {
             early_s[n_early] = s;
             early_kb[n_early] = kb;
@@ -1175,18 +1190,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(b * 128);
-        for (int kb = k0; kb < k1; ++kb) {
+        for (int kb = k0; kb < k1; kb += KPS) {
           if (!mbar_wait_bounded(&full[s], ph, abort, p.timeout_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t w_base = smem_addr(smem + L::kOffW + s * L::kW);
-          const uint32_t x_base = smem_addr(smem + L::kOffX + s * L::kX);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            mma_i8(d, smem_desc_k_sw128(w_base + k * UMMA_K), smem_desc_k_sw128(x_base + k * UMMA_K), kIdesc,
-                   (kb > k0 || k > 0) ? 1u : 0u);
+          for (int i = 0; i < KPS; ++i) {
+            const uint32_t w_base = smem_addr(smem + L::kOffW + s * L::kW + i * L::kW1);
+            const uint32_t x_base = smem_addr(smem + L::kOffX + s * L::kX + i * L::kX1);
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              mma_i8(d, smem_desc_k_sw128(w_base + k * UMMA_K), smem_desc_k_sw128(x_base + k * UMMA_K), kIdesc,
+                     (kb > k0 || i > 0 || k > 0) ? 1u : 0u);
+            }
           }
           mma_commit(&empty[s]);
           if (++s == S) {
@@ -1468,7 +1486,7 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
 
 namespace {
 
-template <int EPI, int BNT>
+template <int EPI, int BNT, int KPS>
 cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
   CUtensorMap tw, tx;
   if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, SM_BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1486,9 +1504,9 @@ cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmPar
     const int cap = sms < kMaxSplitCtas ? sms : kMaxSplitCtas;
     grid = static_cast<int>(units < cap ? units : cap);
   }
-  constexpr int smem = SmallSmem<BNT>::kAlloc;
+  constexpr int smem = SmallSmem<BNT, KPS>::kAlloc;
   static std::atomic<int> attr_done[kMaxDevices];
-  cudaError_t e = ensure_smem_attr(gemm_i8_smallm_kernel<EPI, BNT>, smem, attr_done);
+  cudaError_t e = ensure_smem_attr(gemm_i8_smallm_kernel<EPI, BNT, KPS>, smem, attr_done);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1500,15 +1518,22 @@ cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmPar
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_smallm_kernel<EPI, BNT>, tw, tx, out, B, p);
+  return cudaLaunchKernelEx(&cfg, gemm_i8_smallm_kernel<EPI, BNT, KPS>, tw, tx, out, B, p);
+}
+
+template <int EPI, int KPS>
+cudaError_t launch_smallm_k(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
+  if (p.M <= 16) return launch_smallm_t<EPI, 16, KPS>(A, B, out, p, stream);
+  if (p.M <= 32) return launch_smallm_t<EPI, 32, KPS>(A, B, out, p, stream);
+  return launch_smallm_t<EPI, 64, KPS>(A, B, out, p, stream);
 }
 
 template <int EPI>
 cudaError_t launch_smallm(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
-  if (p.M <= 16) return launch_smallm_t<EPI, 16>(A, B, out, p, stream);
-  if (p.M <= 32) return launch_smallm_t<EPI, 32>(A, B, out, p, stream);
-  if (p.M <= 64) return launch_smallm_t<EPI, 64>(A, B, out, p, stream);
-  return launch_smallm_t<EPI, 128>(A, B, out, p, stream);
+  // several k-blocks per stage only for whole tiles (the split form walks single k-blocks)
+  if (p.split_part == nullptr && CONVROT_SMALLM_KPS > 1)
+    return launch_smallm_k<EPI, CONVROT_SMALLM_KPS>(A, B, out, p, stream);
+  return launch_smallm_k<EPI, 1>(A, B, out, p, stream);
 }
 
 }  // namespace

@@ -50,7 +50,11 @@ struct GemmParams {
 constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass (fused form)
 constexpr int kSmallM = 64;  // up to this many tokens the GEMM runs in the weight-streaming (swap-AB) form
 constexpr int kMaxSplitCtas = 160;    // CTAs of the split weight-streaming form (at most)
-constexpr int kMaxSplitTiles = 4096;  // weight tiles (128 rows each) the split form takes (N <= 524288)
+// The split pays a partial-tile epilogue (a store, a fence, a counter and the
+// last CTA's sum) at the end of most CTAs' ranges: on the 96-tile text-encoder
+// layer it measured slower than whole tiles on 96 SMs, so it is used only where
+// whole tiles would leave most SMs idle.
+constexpr int kMaxSplitTiles = 64;  // weight tiles (128 rows each) up to which the split form is used (N <= 8192)
 
 // Token columns of the weight-streaming form's MMA for M tokens (16, 32 or 64).
 __host__ __device__ constexpr int smallm_bnt(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }

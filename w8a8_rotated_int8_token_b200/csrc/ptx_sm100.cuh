@@ -61,6 +61,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// mbar_try_wait, letting the hardware suspend the thread for up to `ns`
+// nanoseconds until the phase completes (it resumes as soon as it does): a
+// waiting warp then takes no issue slots from the warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return done != 0;
+}
+
 // Wait until the phase with the given parity has completed, for at most
 // `timeout_ns`. Returns false if the wait ran out or if another thread of the
 // CTA raised `*abort` (then the caller unwinds; `abort` may be null). Never
