@@ -36,7 +36,7 @@ struct LinearWs {
 };
 
 #ifndef CONVROT_SMALLM_SPLIT
-#define CONVROT_SMALLM_SPLIT 1
+#define CONVROT_SMALLM_SPLIT 0
 #endif
 
 // Whether convrot_linear runs the weight-streaming GEMM split over all SMs.
