@@ -39,11 +39,15 @@ struct LinearWs {
 #define CONVROT_SMALLM_SPLIT 0
 #endif
 
-// Whether convrot_linear runs the weight-streaming GEMM split over all SMs.
-bool linear_uses_split(int64_t M, int64_t N) {
-  return CONVROT_SMALLM_SPLIT != 0 && M >= 1 && M <= convrot::kSmallM &&
-         (N + 127) / 128 <= convrot::kMaxSplitTiles;
+// Whether the workspace of a shape holds the split buffers of the
+// weight-streaming GEMM (the layout depends on the shape only) ...
+bool linear_has_split_buffers(int64_t M, int64_t N) {
+  return M >= 1 && M <= convrot::kSmallM && (N + 127) / 128 <= convrot::kMaxSplitTiles;
 }
+
+// ... and whether convrot_linear uses them (the split is compiled out by default:
+// it measured slower than whole tiles on every shape tried).
+bool linear_uses_split(int64_t M, int64_t N) { return CONVROT_SMALLM_SPLIT != 0 && linear_has_split_buffers(M, N); }
 
 LinearWs linear_ws_layout(int64_t M, int64_t K, int64_t N) {
   LinearWs w;
@@ -52,7 +56,7 @@ LinearWs linear_ws_layout(int64_t M, int64_t K, int64_t N) {
   w.scale_off = align_up(w.ready_off + 8 * mblocks, 256);
   w.codes_off = align_up(w.scale_off + 4 * static_cast<size_t>(M), 1024);
   w.total = align_up(w.codes_off + static_cast<size_t>(M) * static_cast<size_t>(K), 256);
-  w.split = linear_uses_split(M, N);
+  w.split = linear_has_split_buffers(M, N);
   w.split_count_off = w.split_part_off = 0;
   if (w.split) {
     w.split_count_off = w.total;
@@ -325,7 +329,7 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   p.timeout_ns = kWaitTimeoutNs;
   int32_t* split_part = nullptr;
   unsigned* split_count = nullptr;
-  if (lay.split) {
+  if (lay.split && linear_uses_split(M, N)) {
     // the weight-streaming GEMM split over all SMs: its arrival counters are
     // zeroed by the first kernel, before the GEMM may start
     split_part = reinterpret_cast<int32_t*>(wsb + lay.split_part_off);
