@@ -13,9 +13,13 @@ g=256, with bias.
 Besides the headline the line carries:
   * ``int8_peak``: the int8 tensor pipe's rate measured on this GPU by a probe
     that issues the GEMM's own instruction (tcgen05.mma.cta_group::2.kind::i8,
-    256x256x32) from shared memory with no global traffic, in bursts (the
-    denominator of the GEMM's roofline) and in a longer loop under the power
-    limit (sustained);
+    256x256x32) from shared memory with no global traffic, in bursts and in a
+    longer loop under the power limit (sustained), on zero operands and on
+    operand tiles copied from the layer's own codes. The tensor cores draw more
+    power on real codes and the GPU lowers its clock sooner, so the rate on the
+    codes (the larger of its burst and sustained figures) is the GEMM's roofline
+    denominator; the zero-operand rate and the fraction against it are reported
+    beside it;
   * ``configs``: every layer shape of the workload table timed by CUDA events
     (median and min over the repetitions, inputs rotated over enough buffer
     sets to exceed L2): the layer's time per call, TOPS, the GEMM's TOPS and
@@ -54,6 +58,7 @@ L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200 (context only)
 NOMINAL_INT8_TOPS = 4500.0  # datasheet dense int8 (context only)
+PEAK_BURST_REGION_MS = 50.0  # timed regions up to this long are compared with the probe's burst rate
 SMALL_M = 64  # up to this many tokens the layer's GEMM is the weight-streaming form
 PROBE_OPS_PER_ITER_PER_PAIR = 2.0 * 256 * 256 * 128  # four 256x256x32 MMAs
 
@@ -89,8 +94,8 @@ def gemm_traffic(config: str):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="dit_qkv_1024")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
@@ -301,36 +306,51 @@ def bits_to_dev(bits, dev, dtype=None):
     return t if dtype is None or dtype == torch.bfloat16 else t.to(dtype)
 
 
-def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, sustained_s: float = 0.4) -> dict:
+def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, sustained_s: float = 0.4,
+                    operands=None) -> dict:
     """The int8 tensor pipe's rate on this GPU (probe of the GEMM's own instruction, no global traffic).
 
     burst: single launches of about `burst_ms`, timed by events, after two warm-up
     launches (the GEMM is timed the same way, alone or inside short steps);
     sustained: launches back to back for about `sustained_s` under the power limit.
+    With `operands` (the layer's own codes) the same two figures are taken again on
+    them: the tensor cores draw more power on real codes than on zeros, and the GPU
+    lowers its clock under its power limit sooner.
     """
     import torch
 
     ws = torch.empty((256,), dtype=torch.uint8, device=dev)
-    ctas = cr.convrot_probe_i8_peak(64, ws=ws, stream=stream)
+    r = _probe_i8_rates(cr, dev, stream, clock_index, ws, None, burst_ms, sustained_s)
+    if operands is not None:
+        c = _probe_i8_rates(cr, dev, stream, clock_index, ws, operands, burst_ms, sustained_s)
+        r["on_layer_codes"] = {k: c[k] for k in ("burst_tops", "burst_tops_median", "sustained_tops",
+                                                 "burst_clock_mhz", "sustained_clock_mhz", "reasons")}
+    return r
+
+
+def _probe_i8_rates(cr, dev, stream, clock_index: int, ws, operands, burst_ms: float, sustained_s: float) -> dict:
+    import torch
+
+    ctas = cr.convrot_probe_i8_peak(64, operands=operands, ws=ws, stream=stream)
     torch.cuda.synchronize(dev)
     pairs = ctas // 2
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # calibrate the iteration count to about burst_ms per launch
     iters = 1024
     e0.record(stream)
-    cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+    cr.convrot_probe_i8_peak(iters, operands=operands, ws=ws, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     iters = int(max(256, min(1 << 20, iters * burst_ms / max(e0.elapsed_time(e1), 1e-3))))
     ops = PROBE_OPS_PER_ITER_PER_PAIR * iters * pairs
     for _ in range(2):
-        cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+        cr.convrot_probe_i8_peak(iters, operands=operands, ws=ws, stream=stream)
     torch.cuda.synchronize(dev)
     burst = []
     with ClockSampler(clock_index, 0.001) as clk_b:
         for _ in range(10):
             e0.record(stream)
-            cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+            cr.convrot_probe_i8_peak(iters, operands=operands, ws=ws, stream=stream)
             e1.record(stream)
             torch.cuda.synchronize(dev)
             burst.append(ops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
@@ -338,7 +358,7 @@ def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, su
     with ClockSampler(clock_index, 0.005) as clk_s:
         e0.record(stream)
         for _ in range(n_sus):
-            cr.convrot_probe_i8_peak(iters, ws=ws, stream=stream)
+            cr.convrot_probe_i8_peak(iters, operands=operands, ws=ws, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
     sustained = ops * n_sus / (e0.elapsed_time(e1) * 1e-3) / 1e12
@@ -351,8 +371,8 @@ def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, su
             "reasons": sorted(set(b["reasons"]) | set(s["reasons"])),
             "ops_per_clk_per_sm_burst": (max(burst) * 1e12 / (b["sm_mhz"] * 1e6) / ctas) if b["sm_mhz"] else None,
             "probe": f"{pairs} CTA pairs x {iters} x 4 tcgen05.mma.cta_group::2.kind::i8 (256x256x32), "
-                     f"operands in shared memory, no global traffic; burst = best of 10 launches of ~{burst_ms:g} ms, "
-                     f"sustained = {n_sus} launches back to back; peak = the larger of the two",
+                     f"zero operands in shared memory, no global traffic; burst = best of 10 launches of "
+                     f"~{burst_ms:g} ms, sustained = {n_sus} launches back to back; peak = the larger of the two",
             "context": {"nominal_dense_int8_tops": NOMINAL_INT8_TOPS}}
 
 
@@ -775,7 +795,6 @@ def main():
     n_alone = max(1, min(args.steps, 200))
     t_q = time_loop(q_only, n_alone)
     t_g = None if variant else time_loop(g_only, n_alone)
-    del xq, xsc
     if variant:
         t_layer = t_ms / args.steps
         t_first = t_q
@@ -785,13 +804,44 @@ def main():
     # ---- the int8 tensor pipe's measured peak (the GEMM's roofline denominator)
     i8 = None
     if not args.no_peak:
-        i8 = measure_i8_peak(cr, dev, stream, local)
+        # the probe's operand tiles on the layer's own codes: 16 KB of activation codes
+        # and 16 KB of weight codes per CTA
+        n_ctas = int(L.convrot_probe_i8_peak_ctas())
+        half = 16384
+        codes = torch.stack([xq[0].view(-1)[: n_ctas * half].view(torch.uint8).view(n_ctas, half),
+                             sets[0]["Wq"].view(-1)[: n_ctas * half].view(torch.uint8).view(n_ctas, half)],
+                            1).contiguous() if M * K >= n_ctas * half and N * K >= n_ctas * half else None
+        i8 = measure_i8_peak(cr, dev, stream, local, operands=codes)
+        del codes
         i8["peak_tops"] = max_over_ranks(i8["peak_tops"])  # every rank runs it; the figure is per GPU
-    int8_peak = i8["peak_tops"] if i8 else peaks["bf16_tflops"] * INT8_OVER_BF16
-    int8_peak_src = ("measured int8 probe (tcgen05.mma.cta_group::2.kind::i8 from shared memory; the larger of "
-                     "its burst and sustained rates)" if i8 else
-                     f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
-                     "(nominal int8:bf16 dense ratio)")
+    del xq, xsc
+    # The roofline denominator: the probe's rate on the layer's own codes (the data the
+    # GEMM multiplies: the tensor cores draw more power on it than on zeros, and the GPU
+    # holds a lower clock); the zero-operand rate is reported beside it.
+    # A timed region of at most PEAK_BURST_REGION_MS is compared with the probe's burst
+    # rate (single launches of ~5 ms), a longer one with its sustained rate (0.4 s back
+    # to back), since the GPU lowers its clock under its power limit within tens of ms.
+    int8_peak_zero = i8["peak_tops"] if i8 else None
+    int8_peak_codes = None
+    region_ms = t_ms
+    peak_kind = "burst" if region_ms <= PEAK_BURST_REGION_MS else "sustained"
+    int8_peak_short = int8_peak_zero  # for the configs' short repetitions: the burst rate on codes
+    if i8 and "on_layer_codes" in i8:
+        int8_peak_codes = max_over_ranks(i8["on_layer_codes"][f"{peak_kind}_tops"])
+        int8_peak_short = max_over_ranks(i8["on_layer_codes"]["burst_tops"])
+    if int8_peak_codes is not None:
+        int8_peak = int8_peak_codes
+        int8_peak_src = (f"measured int8 probe on the layer's own codes, {peak_kind} rate (the timed region lasted "
+                         f"{region_ms:.1f} ms): tcgen05.mma.cta_group::2.kind::i8 from shared memory, operand tiles "
+                         "copied from this layer's activation and weight codes")
+    elif i8:
+        int8_peak = int8_peak_zero
+        int8_peak_src = ("measured int8 probe on zero operands (tcgen05.mma.cta_group::2.kind::i8 from shared memory; "
+                         "the larger of its burst and sustained rates)")
+    else:
+        int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+        int8_peak_src = (f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
+                         "(nominal int8:bf16 dense ratio)")
     layer_tops = ops / (t_layer * 1e-3) / 1e12
     gemm_tops = None if t_g is None else ops / (t_g * 1e-3) / 1e12
     q_bytes = 3.0 * M * K + 4.0 * M
@@ -826,12 +876,14 @@ def main():
         order = CONFIG_NAMES[shift:] + CONFIG_NAMES[:shift]
         for name in order:
             configs[name] = bench_config(cr, L, name, dev, stream, args.config_reps, peaks,
-                                         i8["peak_tops"] if i8 else None, up_cache)
+                                         int8_peak_short if i8 else None, up_cache)
         configs["attention_int8_4224"] = bench_attention(cr, dev, stream, args.config_reps, local,
-                                                         i8["peak_tops"] if i8 else None)
+                                                         int8_peak_short if i8 else None)
         configs = {"order": order, "reps": args.config_reps,
                    "timing": "CUDA events on the launching stream; median and min over the repetitions; "
-                             "layer_us from back-to-back calls", **configs}
+                             "layer_us from back-to-back calls",
+                   "int8_peak_tops": int8_peak_short,
+                   "int8_peak_source": "the int8 probe's burst rate on the default layer's codes", **configs}
         del up_cache
 
     if world > 1:
@@ -856,6 +908,8 @@ def main():
                      "us_source": ("layer time minus the standalone rotate+quantise kernel" if variant
                                    else "CUDA events around the GEMM launch inside each step (mean)"),
                      "peak_source": int8_peak_src,
+                     "peak_zero_operands": int8_peak_zero,
+                     "frac_zero_operands": (dom_tops / int8_peak_zero) if int8_peak_zero else None,
                      "peak_context": {"nominal_dense_int8_tops": NOMINAL_INT8_TOPS,
                                       "bf16_x2_tops": peaks["bf16_tflops"] * INT8_OVER_BF16,
                                       "bf16_source": peak_src}},

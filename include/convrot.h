@@ -354,15 +354,21 @@ CONVROT_API convrot_status convrot_attention_int8(const void* Q, const void* K, 
  * convrot_probe_i8_peak -- measurement aid for the GEMM's roofline (not part
  * of the layer): launches one CTA pair per two SMs, each issuing `iters`
  * times four tcgen05.mma.cta_group::2.kind::i8 instructions (M = 256, N = 256,
- * K = 32: the instruction the layer's GEMM uses) on zeroed shared-memory
- * operands, with no global memory traffic. The caller times the launch with
+ * K = 32: the instruction the layer's GEMM uses) on shared-memory operands,
+ * with no global memory traffic in the loop. The caller times the launch with
  * events on `stream`; the work is 2 * 256 * 256 * 128 * iters operations per
- * pair, convrot_probe_i8_peak_ctas() / 2 pairs. iters in [1, 2^20]. `ws`
- * (>= 256 bytes, 256-byte aligned) receives the status word
- * (CONVROT_ERR_DEVICE_TIMEOUT if the final wait ran out).
+ * pair, convrot_probe_i8_peak_ctas() / 2 pairs. iters in [1, 2^20].
+ * operands: null (zero operands) or a device buffer of operand_bytes bytes
+ * (16-byte aligned, a positive multiple of 16) from which every CTA copies its
+ * 32 KB of A and B tiles once, before the loop (wrapping around the buffer).
+ * The rate at a fixed clock does not depend on the values, but the power
+ * drawn does: the layer's own codes give the clock the GPU holds under its
+ * power limit while the GEMM runs. `ws` (>= 256 bytes, 256-byte aligned)
+ * receives the status word (CONVROT_ERR_DEVICE_TIMEOUT if the final wait ran
+ * out).
  */
-CONVROT_API convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t ws_bytes,
-                                                 convrot_stream_t stream);
+CONVROT_API convrot_status convrot_probe_i8_peak(int64_t iters, const void* operands, size_t operand_bytes,
+                                                 void* ws, size_t ws_bytes, convrot_stream_t stream);
 /* CTAs that convrot_probe_i8_peak launches on the current device (0 on error). */
 CONVROT_API int convrot_probe_i8_peak_ctas(void);
 

@@ -346,16 +346,24 @@ def convrot_test_wait_timeout(ws, timeout_ns: int, stream=None) -> None:
            "convrot_test_wait_timeout")
 
 
-def convrot_probe_i8_peak(iters: int, ws=None, stream=None) -> int:
+def convrot_probe_i8_peak(iters: int, operands=None, ws=None, stream=None) -> int:
     """Enqueue the int8 tensor-pipe peak probe (one CTA pair per two SMs, `iters` x 4
-    tcgen05.mma.cta_group::2.kind::i8 of 256x256x32 each, no global traffic); returns
-    the number of CTAs launched. The caller times it with events on `stream`."""
+    tcgen05.mma.cta_group::2.kind::i8 of 256x256x32 each, no global traffic in the loop);
+    returns the number of CTAs launched. `operands`: None (zero operands) or a contiguous
+    device tensor whose bytes fill the CTAs' operand tiles. The caller times it with
+    events on `stream`."""
     import torch
 
     L = lib()
     if ws is None:
         ws = torch.empty((256,), dtype=torch.uint8, device=torch.cuda.current_device())
-    _check(L.convrot_probe_i8_peak(int(iters), _ptr(ws), ws.numel(), _stream_ptr(stream)), "convrot_probe_i8_peak")
+    op_ptr, op_bytes = None, 0
+    if operands is not None:
+        if not operands.is_contiguous():
+            raise ValueError("operands must be contiguous")
+        op_ptr, op_bytes = _ptr(operands), operands.numel() * operands.element_size()
+    _check(L.convrot_probe_i8_peak(int(iters), op_ptr, op_bytes, _ptr(ws), ws.numel(), _stream_ptr(stream)),
+           "convrot_probe_i8_peak")
     return int(L.convrot_probe_i8_peak_ctas())
 
 

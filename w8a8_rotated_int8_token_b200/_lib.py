@@ -46,7 +46,7 @@ SIGNATURES = {
                                       _c_void_p, _c_void_p, _c_void_p]),
     "convrot_read_device_status": (_int, [_c_void_p, _c_void_p]),
     "convrot_test_wait_timeout": (_int, [_c_void_p, _size, _i64, _c_void_p]),
-    "convrot_probe_i8_peak": (_int, [_i64, _c_void_p, _size, _c_void_p]),
+    "convrot_probe_i8_peak": (_int, [_i64, _c_void_p, _size, _c_void_p, _size, _c_void_p]),
     "convrot_attention_workspace_bytes": (_size, [_i64, _i64, _i64, _i64]),
     "convrot_attention_int8": (_int, [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _i64, ctypes.c_float,
                                       _c_void_p, _c_void_p, _size, _c_void_p]),

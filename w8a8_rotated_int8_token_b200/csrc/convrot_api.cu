@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 7;
+constexpr int kAbiVersion = 8;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
 // convrot_linear runs two kernels chained with programmatic dependent launch.
 // The one-launch form (rotate+quantise worker warps inside the GEMM kernel,

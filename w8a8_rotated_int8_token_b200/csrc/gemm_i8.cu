@@ -343,10 +343,11 @@ __device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmOut, const Ge
       }
       uint32_t packed[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float y0 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e])), sc, bv[2 * e]);
-        const float y1 = fmaf(static_cast<float>(static_cast<int32_t>(r[2 * e + 1])), sc, bv[2 * e + 1]);
-        packed[e] = bf16x2(y0, y1);
+      for (int e = 0; e < 16; ++e) {  // two fused multiply-adds per packed instruction (each rounded once)
+        const float2 y = __ffma2_rn(make_float2(static_cast<float>(static_cast<int32_t>(r[2 * e])),
+                                                static_cast<float>(static_cast<int32_t>(r[2 * e + 1]))),
+                                    make_float2(sc, sc), make_float2(bv[2 * e], bv[2 * e + 1]));
+        packed[e] = bf16x2(y.x, y.y);
       }
       // 32 rows x 64 bytes, 64-byte swizzle: 16-byte piece j of row r at piece j ^ ((r >> 1) & 3)
       uint8_t* rowp = ebuf + lane * 64;
@@ -701,7 +702,7 @@ constexpr int PAIR_THREADS = 64 + 32 * PAIR_EPI_WARPS;
 #define CONVROT_PAIR_STAGES 6
 #endif
 #ifndef CONVROT_PAIR_GROUP_M
-#define CONVROT_PAIR_GROUP_M 8
+#define CONVROT_PAIR_GROUP_M 16
 #endif
 constexpr int PAIR_STAGES = CONVROT_PAIR_STAGES;
 constexpr int PA_STAGE_BYTES = BM * BK;       // 16 KB: this CTA's 128 rows of A

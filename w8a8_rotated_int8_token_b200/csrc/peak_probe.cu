@@ -2,7 +2,10 @@
 // issues (tcgen05.mma.cta_group::2.kind::i8, M = 256, N = 256, K = 32 per
 // instruction, both operands from shared memory) in a loop with no global
 // memory traffic, so that a timed launch gives the rate the tensor cores
-// sustain on this GPU at its current clock. The special-function unit's exp2
+// sustain on this GPU at its current clock. The operands are zero or copied
+// from a caller buffer (the layer's own codes): the rate at a fixed clock does
+// not depend on them, but the power drawn does, and with it the clock the
+// GPU holds under its power limit. The special-function unit's exp2
 // (the unit the attention softmax is bound by): independent chains of
 // ex2.approx in every thread of a full grid. Measurement aids for the
 // rooflines; they compute nothing of the layer.
@@ -23,7 +26,8 @@ constexpr int kProbeThreads = 128;
 constexpr int kTimeoutStatus = 5;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
-    i8_peak_pair_kernel(int64_t iters, int* status, uint64_t timeout_ns) {
+    i8_peak_pair_kernel(int64_t iters, const uint4* operands, int64_t operand_chunks, int* status,
+                        uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t done;
   __shared__ uint32_t tmem_ptr;
@@ -32,10 +36,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
   const int lane = threadIdx.x & 31;
   const bool leader = cluster_ctarank() == 0;
 
-  // zero operands (their values do not change the rate); the tensor cores read
-  // them through the async proxy
-  for (int i = threadIdx.x; i < 2 * kProbeTile / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // this CTA's A and B tiles: zeros, or 2 * kProbeTile consecutive bytes of the
+  // caller's buffer starting at chunk (blockIdx.x * 2 * kProbeTile / 16) modulo
+  // its length (16-byte chunks); the tensor cores read them through the async proxy
+  constexpr int kChunks = 2 * kProbeTile / 16;
+  for (int i = threadIdx.x; i < kChunks; i += blockDim.x) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (operands != nullptr) v = operands[(static_cast<int64_t>(blockIdx.x) * kChunks + i) % operand_chunks];
+    reinterpret_cast<uint4*>(smem)[i] = v;
+  }
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     mbar_init(&done, 1);
@@ -112,9 +121,13 @@ int64_t convrot_probe_ex2_per_iter(void) {
   return static_cast<int64_t>(sms) * convrot::kEx2CtasPerSm * convrot::kEx2Threads * convrot::kEx2Chains;
 }
 
-convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t ws_bytes, convrot_stream_t stream) {
+convrot_status convrot_probe_i8_peak(int64_t iters, const void* operands, size_t operand_bytes, void* ws,
+                                     size_t ws_bytes, convrot_stream_t stream) {
   // at most 2^20 x 512 tensor cycles (about 0.3 s at 1.9 GHz): well inside the 2 s bound of the final wait
   if (iters < 1 || iters > (int64_t(1) << 20)) return CONVROT_ERR_INVALID_ARG;
+  if (operands != nullptr &&
+      ((reinterpret_cast<uintptr_t>(operands) % 16) != 0 || operand_bytes < 16 || (operand_bytes % 16) != 0))
+    return CONVROT_ERR_INVALID_ARG;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % 256) != 0 || ws_bytes < 256) return CONVROT_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int dev = 0, sms = 0;
@@ -127,8 +140,8 @@ convrot_status convrot_probe_i8_peak(int64_t iters, void* ws, size_t ws_bytes, c
   int* status = static_cast<int*>(ws);
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
   // one CTA pair per two SMs, every SM busy
-  convrot::i8_peak_pair_kernel<<<(sms / 2) * 2, convrot::kProbeThreads, smem, s>>>(iters, status,
-                                                                                    2000000000ull);
+  convrot::i8_peak_pair_kernel<<<(sms / 2) * 2, convrot::kProbeThreads, smem, s>>>(
+      iters, static_cast<const uint4*>(operands), static_cast<int64_t>(operand_bytes / 16), status, 2000000000ull);
   return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
