@@ -104,6 +104,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config table")
     ap.add_argument("--no-peak", action="store_true", help="skip the int8 peak probe")
     ap.add_argument("--config-reps", type=int, default=30, help="timed repetitions per config")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="time only the INT8 attention call (--config-reps calls) and print its figures")
     # layer variants (convrot_linear_ex); the defaults are the headline layer
     ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16", help="dtype of X, W, bias and Y")
     ap.add_argument("--wscale", choices=["tensor", "channel"], default="tensor", help="weight-scale granularity")
@@ -656,6 +658,14 @@ def main():
 
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, dev)
+
+    if args.attention_only:
+        att = bench_attention(cr, dev, torch.cuda.current_stream(dev), args.config_reps, local, None)
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"attention_int8_4224": att}), flush=True)
+        return 0
 
     d = synth.make_workload(args.config)
     w = d["workload"]
