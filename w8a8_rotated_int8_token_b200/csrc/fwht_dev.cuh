@@ -247,11 +247,22 @@ __device__ __forceinline__ QuantScale make_scale(float amax_u) {
 }
 
 // The stored scale of a row (or tensor): float32(absmax(X R) / 127) =
-// absmax_u / (127 sqrt(g)), one correctly rounded division (for g = 256 the
-// divisor 2032 is exact; for g = 128 it is the nearest float to 127 sqrt(128)).
+// absmax_u / (127 sqrt(g)), correctly rounded (for g = 256 the divisor 2032 is
+// exact; for g = 128 it is the nearest float to 127 sqrt(128)). From 2^-100 up
+// the quotient is the product with the rounded reciprocal r of the divisor,
+// corrected once by the exact remainder (two fused multiply-adds); that this
+// equals the correctly rounded quotient for every float in that range is
+// checked exhaustively on the CPU by the test suite. Below 2^-100 (where the
+// remainder could leave the normal range) it is the plain division.
 template <int G>
 __device__ __forceinline__ float scale_of(float amax_u) {
-  const float div = (G == 256) ? 2032.0f : 1436.8409423828125f;
+  constexpr float div = (G == 256) ? 2032.0f : 1436.8409423828125f;
+  constexpr float r = (G == 256) ? 0x1.020408p-11f : 0x1.6ce3aep-11f;  // nearest floats to 1/div
+  if (amax_u >= 0x1p-100f) {
+    const float q0 = __fmul_rn(amax_u, r);
+    const float e = fmaf(-q0, div, amax_u);  // exact remainder amax_u - q0 * div
+    return fmaf(e, r, q0);
+  }
   return amax_u / div;
 }
 
