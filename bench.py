@@ -58,6 +58,7 @@ L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B200 (context only)
 NOMINAL_INT8_TOPS = 4500.0  # datasheet dense int8 (context only)
+WS_CLOCK_RECORD_OFFSET = 64  # CONVROT_WS_CLOCK_RECORD_OFFSET in include/convrot.h
 PEAK_BURST_REGION_MS = 50.0  # timed regions up to this long are compared with the probe's burst rate
 SMALL_M = 64  # up to this many tokens the layer's GEMM is the weight-streaming form
 PROBE_OPS_PER_ITER_PER_PAIR = 2.0 * 256 * 256 * 128  # four 256x256x32 MMAs
@@ -326,8 +327,20 @@ def measure_i8_peak(cr, dev, stream, clock_index: int, burst_ms: float = 5.0, su
     if operands is not None:
         c = _probe_i8_rates(cr, dev, stream, clock_index, ws, operands, burst_ms, sustained_s)
         r["on_layer_codes"] = {k: c[k] for k in ("burst_tops", "burst_tops_median", "sustained_tops",
-                                                 "burst_clock_mhz", "sustained_clock_mhz", "reasons")}
+                                                 "burst_clock_mhz", "sustained_clock_mhz", "reasons",
+                                                 "burst_sm_mhz_in_kernel", "sustained_sm_mhz_in_kernel",
+                                                 "ops_per_clk_per_sm_in_kernel")}
     return r
+
+
+def kernel_clock_mhz(ws) -> float | None:
+    """The SM clock a GEMM or probe launch ran at, from the clock record it left in its workspace
+    (%clock64 and %globaltimer twice; include/convrot.h, CONVROT_WS_CLOCK_RECORD_OFFSET)."""
+    import torch
+
+    rec = ws[WS_CLOCK_RECORD_OFFSET:WS_CLOCK_RECORD_OFFSET + 32].view(torch.int64).tolist()
+    dc, dt = rec[2] - rec[0], rec[3] - rec[1]
+    return dc / dt * 1e3 if dc > 0 and dt > 0 else None
 
 
 def _probe_i8_rates(cr, dev, stream, clock_index: int, ws, operands, burst_ms: float, sustained_s: float) -> dict:
@@ -348,7 +361,7 @@ def _probe_i8_rates(cr, dev, stream, clock_index: int, ws, operands, burst_ms: f
     for _ in range(2):
         cr.convrot_probe_i8_peak(iters, operands=operands, ws=ws, stream=stream)
     torch.cuda.synchronize(dev)
-    burst = []
+    burst, burst_mhz = [], []
     with ClockSampler(clock_index, 0.001) as clk_b:
         for _ in range(10):
             e0.record(stream)
@@ -356,6 +369,7 @@ def _probe_i8_rates(cr, dev, stream, clock_index: int, ws, operands, burst_ms: f
             e1.record(stream)
             torch.cuda.synchronize(dev)
             burst.append(ops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+            burst_mhz.append(kernel_clock_mhz(ws))
     n_sus = int(max(1, sustained_s * 1e3 / burst_ms))
     with ClockSampler(clock_index, 0.005) as clk_s:
         e0.record(stream)
@@ -364,6 +378,7 @@ def _probe_i8_rates(cr, dev, stream, clock_index: int, ws, operands, burst_ms: f
         e1.record(stream)
         torch.cuda.synchronize(dev)
     sustained = ops * n_sus / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    sustained_mhz = kernel_clock_mhz(ws)  # the last launch of the loop
     if cr.convrot_read_device_status(ws) != 0:
         raise RuntimeError("int8 peak probe: a device wait timed out")
     b, s = clk_b.summary(), clk_s.summary()
@@ -372,6 +387,10 @@ def _probe_i8_rates(cr, dev, stream, clock_index: int, ws, operands, burst_ms: f
             "burst_clock_mhz": b["sm_mhz"], "sustained_clock_mhz": s["sm_mhz"],
             "reasons": sorted(set(b["reasons"]) | set(s["reasons"])),
             "ops_per_clk_per_sm_burst": (max(burst) * 1e12 / (b["sm_mhz"] * 1e6) / ctas) if b["sm_mhz"] else None,
+            "burst_sm_mhz_in_kernel": burst_mhz[burst.index(max(burst))],
+            "sustained_sm_mhz_in_kernel": sustained_mhz,
+            "ops_per_clk_per_sm_in_kernel": ((max(burst) * 1e12 / (burst_mhz[burst.index(max(burst))] * 1e6) / ctas)
+                                             if burst_mhz[burst.index(max(burst))] else None),
             "probe": f"{pairs} CTA pairs x {iters} x 4 tcgen05.mma.cta_group::2.kind::i8 (256x256x32), "
                      f"zero operands in shared memory, no global traffic; burst = best of 10 launches of "
                      f"~{burst_ms:g} ms, sustained = {n_sus} launches back to back; peak = the larger of the two",
@@ -768,6 +787,11 @@ def main():
         t_second = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
         t_second_med = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in ev))
         t_second_min = max_over_ranks(min(e[1].elapsed_time(e[2]) for e in ev))
+        # the SM clock the GEMM ran at inside the steps: the clock record of each set's last call
+        gemm_mhz = [m for m in (kernel_clock_mhz(s["ws"]) for s in sets) if m]
+        gemm_mhz = statistics.median(gemm_mhz) if gemm_mhz else None
+    else:
+        gemm_mhz = None
     # (variants: no per-launch events; the GEMM's time is the layer's minus the
     # standalone rotate+quantise kernel's, below)
 
@@ -941,6 +965,17 @@ def main():
     if not variant:
         out["roofline"]["us_per_launch_median"] = t_second_med * 1e3
         out["roofline"]["us_per_launch_min"] = t_second_min * 1e3
+        out["roofline"]["sm_mhz_in_kernel"] = gemm_mhz
+        opc = (i8 or {}).get("on_layer_codes", {}).get("ops_per_clk_per_sm_in_kernel")
+        if gemm_mhz and opc and M > SMALL_M:
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            at_clock = opc * sms * gemm_mhz * 1e6 / 1e12
+            out["roofline"]["peak_at_kernel_clock"] = at_clock
+            out["roofline"]["frac_at_kernel_clock"] = dom_tops / at_clock
+            out["roofline"]["clock_note"] = (
+                "sm_mhz_in_kernel: the SM clock the GEMM ran at inside the steps (its %clock64 against "
+                "%globaltimer); peak_at_kernel_clock: the probe's int8 rate per SM clock on the layer's codes "
+                "times that clock; NVML's clock samples do not follow these changes")
     if i8:
         out["int8_peak"] = i8
     if M <= SMALL_M:

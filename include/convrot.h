@@ -84,6 +84,19 @@ typedef enum {
 /* Largest K the rotation/quantisation kernels take (one CTA holds a token). */
 #define CONVROT_MAX_K 32768
 
+/*
+ * Byte offset, inside the workspace of convrot_linear, convrot_linear_timed,
+ * convrot_gemm_dequant and convrot_gemm_s32, of a measurement record the
+ * tensor-core GEMM for M > 64 writes on every call: four uint64, the SM clock
+ * counter (%clock64) and the global timer in ns (%globaltimer) read by one
+ * thread of its first CTA when that CTA's first operands have landed, then
+ * again after it has issued its last tile's MMAs. (clock difference) / (time
+ * difference) is the SM clock the GEMM ran at, in GHz. The weight-streaming
+ * GEMM (M <= 64) and the one-launch form leave the record untouched. Not
+ * part of any result; no call reads it.
+ */
+#define CONVROT_WS_CLOCK_RECORD_OFFSET 64
+
 /* Version of this ABI; bumped when a signature or a layout changes. */
 CONVROT_API int convrot_abi_version(void);
 
@@ -365,7 +378,8 @@ CONVROT_API convrot_status convrot_attention_int8(const void* Q, const void* K, 
  * drawn does: the layer's own codes give the clock the GPU holds under its
  * power limit while the GEMM runs. `ws` (>= 256 bytes, 256-byte aligned)
  * receives the status word (CONVROT_ERR_DEVICE_TIMEOUT if the final wait ran
- * out).
+ * out) and, at CONVROT_WS_CLOCK_RECORD_OFFSET, the same clock record as the
+ * GEMM's (one CTA: before its first MMA and after its last has completed).
  */
 CONVROT_API convrot_status convrot_probe_i8_peak(int64_t iters, const void* operands, size_t operand_bytes,
                                                  void* ws, size_t ws_bytes, convrot_stream_t stream);

@@ -71,7 +71,7 @@ def linear_ws_layout(M, K, N=None):
 
 
 def test_status_strings_and_version(L):
-    assert L.convrot_abi_version() == 8
+    assert L.convrot_abi_version() == 9
     for code in range(6):
         s = L.convrot_status_string(code)
         assert s and s != b"unknown status"

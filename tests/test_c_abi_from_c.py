@@ -37,7 +37,7 @@ static int fails = 0;
 int main(void) {
   void* fake = (void*)(uintptr_t)0x10000; /* aligned, never dereferenced: every call below returns on the host */
   size_t need = convrot_linear_workspace_bytes(4608, 9216, 3072, 256);
-  CHECK(convrot_abi_version() == 8);
+  CHECK(convrot_abi_version() == 9);
   CHECK(strcmp(convrot_status_string(CONVROT_OK), "ok") == 0);
   CHECK(strcmp(convrot_status_string(99), "unknown status") == 0);
   CHECK(need >= (size_t)4608 * 3072 + 4 * 4608);

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 8;
+constexpr int kAbiVersion = 9;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
 // convrot_linear runs two kernels chained with programmatic dependent launch.
 // The one-launch form (rotate+quantise worker warps inside the GEMM kernel,
@@ -136,6 +136,9 @@ convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, 
   p.w_scale = w_scale;
   p.bias = static_cast<const uint16_t*>(bias);
   p.status = status;
+  p.clock_rec = status == nullptr ? nullptr
+                                  : reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(status) +
+                                                                          CONVROT_WS_CLOCK_RECORD_OFFSET);
   p.timeout_ns = kWaitTimeoutNs;
   p.group_m = 0;
   return from_cuda(convrot::launch_gemm_i8(epi, Xq, Wq, out, p, stream));

@@ -45,6 +45,10 @@ struct GemmParams {
   // are divided evenly over the CTAs, and partial tiles meet in these buffers
   int32_t* split_part;            // [2 * kMaxSplitCtas][BNT][128] int32 partial accumulators
   unsigned* split_count;          // [weight tiles] arrival counters, zero when the kernel starts
+  // pair form: CTA 0's MMA issuer writes {%clock64, %globaltimer} when its first
+  // tile's first operands have landed and again after its last tile's MMAs are
+  // issued (the SM clock the kernel ran at), or null
+  unsigned long long* clock_rec;
 };
 
 constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass (fused form)

@@ -27,7 +27,7 @@ constexpr int kTimeoutStatus = 5;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
     i8_peak_pair_kernel(int64_t iters, const uint4* operands, int64_t operand_chunks, int* status,
-                        uint64_t timeout_ns) {
+                        unsigned long long* clock_rec, uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t done;
   __shared__ uint32_t tmem_ptr;
@@ -63,6 +63,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
     const uint32_t a_base = smem_addr(smem);
     const uint32_t b_base = smem_addr(smem + kProbeTile);
     constexpr uint32_t idesc = idesc_i8(256, 256);
+    if (blockIdx.x == 0) {
+      clock_rec[0] = clock64();
+      clock_rec[1] = global_timer_ns();
+    }
     for (int64_t i = 0; i < iters; ++i) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -71,7 +75,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProbeThreads, 1)
     }
     mma_commit_pair_mc(&done, 0x3);  // both CTAs learn that every MMA has finished
   }
-  if (threadIdx.x == 0 && !mbar_wait_bounded(&done, 0u, nullptr, timeout_ns)) atomicOr(status, kTimeoutStatus);
+  if (threadIdx.x == 0) {
+    if (!mbar_wait_bounded(&done, 0u, nullptr, timeout_ns)) {
+      atomicOr(status, kTimeoutStatus);
+    } else if (blockIdx.x == 0) {
+      clock_rec[2] = clock64();
+      clock_rec[3] = global_timer_ns();
+    }
+  }
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();
@@ -141,7 +152,8 @@ convrot_status convrot_probe_i8_peak(int64_t iters, const void* operands, size_t
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
   // one CTA pair per two SMs, every SM busy
   convrot::i8_peak_pair_kernel<<<(sms / 2) * 2, convrot::kProbeThreads, smem, s>>>(
-      iters, static_cast<const uint4*>(operands), static_cast<int64_t>(operand_bytes / 16), status, 2000000000ull);
+      iters, static_cast<const uint4*>(operands), static_cast<int64_t>(operand_bytes / 16), status,
+      reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + CONVROT_WS_CLOCK_RECORD_OFFSET), 2000000000ull);
   return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
