@@ -1498,7 +1498,12 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
   p.num_m_blocks = (p.M + 2 * BM - 1) / (2 * BM);  // 256-row pair blocks
   p.num_n_blocks = (p.N + BN - 1) / BN;
   p.num_k_blocks = (p.K + BK - 1) / BK;
-  if (p.group_m <= 0) p.group_m = CONVROT_PAIR_GROUP_M;
+  // Activation codes of at most 32 MiB stay in L2 for the whole launch: then one
+  // group over every pair-row reads each weight panel from DRAM once (2-3 % faster
+  // on the 4608-token layers than groups of 16, whose remainder group reads the
+  // weight again); larger ones go in groups of 16 pair-rows.
+  if (p.group_m <= 0)
+    p.group_m = static_cast<int64_t>(p.M) * p.K <= (int64_t(32) << 20) ? p.num_m_blocks : CONVROT_PAIR_GROUP_M;
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int sms = sm_count();
   if (sms < 2) return cudaErrorInvalidDevice;
