@@ -576,7 +576,7 @@ def bench_attention(cr, dev, stream, reps: int, clock_index: int, i8_peak) -> di
            "frac_exp2_peak": exps / (t_ms * 1e-3) / measured, "clock_mhz": c["sm_mhz"],
            "exp2_peak_source": "measured: independent ex2.approx chains over a full grid (convrot_probe_ex2_peak)",
            "exp2_nominal_16_per_sm_clk": nominal,
-           "note": "one call = rotate+quantise of Q and of K, transposition of V, the attention kernel"}
+           "note": "one call = rotate+quantise of Q and of K, the attention kernel"}
     if i8_peak:
         out["tensor_floor_us"] = (2.0 * S * S * D * BH / i8_peak + 2.0 * S * S * D * BH / (i8_peak / 2.0)) / 1e6
     del sets

@@ -361,8 +361,9 @@ CONVROT_API convrot_status convrot_read_device_status(const void* ws, convrot_st
  *   Sq = 0 or BH = 0 enqueues nothing. softmax_scale > 0 and finite (usually
  *   1/sqrt(D)). ws: >= convrot_attention_workspace_bytes(BH, Sq, Skv, D),
  *   256-byte aligned; its first word is the status word
- *   (convrot_read_device_status). Launches a 4-byte memset and four kernels
- *   (rotate+quantise of Q and of K, a transposition of V, the attention kernel).
+ *   (convrot_read_device_status). Launches a 4-byte memset and three kernels
+ *   (rotate+quantise of Q and of K, the attention kernel, which reads V as
+ *   given).
  */
 CONVROT_API size_t convrot_attention_workspace_bytes(int64_t BH, int64_t Sq, int64_t Skv, int64_t D);
 CONVROT_API convrot_status convrot_attention_int8(const void* Q, const void* K, const void* V, int64_t BH,

@@ -11,13 +11,13 @@
 // layer is applied to Q and K, and P V runs in bf16 with float32 accumulation.
 //
 // One call: Q and K through the rotate+quantise kernel (codes + one scale per
-// token), V transposed once into key-contiguous rows (the K-major B operand of
-// the P V product), then one CTA per (batch*head, 128-query tile):
+// token), then one CTA per (batch*head, 128-query tile):
 //   warp 0, one lane : TMA producer: the tile's 128 x 128 query codes once,
 //                      then per 128-key block the key codes (loaded as soon
-//                      as the previous block's S is computed) and the
-//                      transposed values (two 64-key halves, loaded as soon
-//                      as the previous block's P V is done).
+//                      as the previous block's S is computed) and the values
+//                      as given (two 64-column halves of the head dimension,
+//                      the MN-major B operand of P V, loaded as soon as the
+//                      previous block's P V is done).
 //   warp 1           : allocates 256 TMEM columns; one lane issues
 //                      S = Qq Kq^T (tcgen05.mma kind::i8, M = N = 128,
 //                      K = 4 x 32) into TMEM columns 0..127 and
@@ -59,11 +59,13 @@ constexpr int AT_D = 128;   // head dimension
 constexpr int AT_THREADS = 192;
 constexpr int kQBytes = AT_BQ * AT_D;      // int8 query codes: 16 KB
 constexpr int kKBytes = AT_BK * AT_D;      // int8 key codes of one block: 16 KB
-constexpr int kHalf = 128 * 128;           // one 64-key half of a bf16 operand: 128 rows x 128 B
-constexpr int kVBytes = 2 * kHalf;         // transposed values of one block: 32 KB
+constexpr int kHalf = 128 * 128;           // 128 rows x 128 B: one half of a block's bf16 operand
+constexpr int kVBytes = 2 * kHalf;         // values of one block: 32 KB (two 64-column halves)
 constexpr int kPBytes = 2 * kHalf;         // probabilities of one block (bf16): 32 KB
 constexpr uint32_t IDESC_S = idesc_i8(AT_BQ, AT_BK);
-constexpr uint32_t IDESC_O = idesc_bf16(AT_BQ, AT_D);
+// P V: A = P (K-major), B = V as stored, keys along K and the head dimension
+// along N contiguous (MN-major: bit 16 of the instruction descriptor)
+constexpr uint32_t IDESC_O = idesc_bf16(AT_BQ, AT_D) | (1u << 16);
 constexpr int kTimeoutStatus = 5;
 constexpr float kRescaleThreshold = 8.0f;  // base-2 units: probabilities stay below 2^8
 
@@ -216,8 +218,8 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
       };
       auto load_v = [&](int j) {
         mbar_arrive_expect_tx(v_full, kVBytes);
-        tma_load_3d(smem + L::kOffV, &tmV, v_full, j * AT_BK, 0, bh);
-        tma_load_3d(smem + L::kOffV + kHalf, &tmV, v_full, j * AT_BK + 64, 0, bh);
+        tma_load_3d(smem + L::kOffV, &tmV, v_full, 0, j * AT_BK, bh);
+        tma_load_3d(smem + L::kOffV + kHalf, &tmV, v_full, 64, j * AT_BK, bh);
         issued_v = j + 1;
       };
       mbar_arrive_expect_tx(q_full, kQBytes);
@@ -277,12 +279,15 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
           break;
         }
         tc_fence_after();
+        // 16 keys per MMA: P's K-major rows advance 32 B inside a 64-key half; V's
+        // MN-major atoms are 8 keys x 64 columns (1 KB apart along the keys, the
+        // second 64 columns 16 KB on)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16(tO, smem_desc_k_sw128(pa + h * kHalf + k * 32), smem_desc_k_sw128(va + h * kHalf + k * 32),
-                     IDESC_O, (j | h | k) != 0 ? 1u : 0u);
+            mma_bf16(tO, smem_desc_k_sw128(pa + h * kHalf + k * 32),
+                     smem_desc_mn_sw128(va + (4 * h + k) * 2048, kHalf, 1024), IDESC_O, (j | h | k) != 0 ? 1u : 0u);
         mma_commit(o_done);
         mma_commit(v_empty);
       }
@@ -460,39 +465,6 @@ __global__ void __launch_bounds__(AT_THREADS, 2)
   }
 }
 
-// V [BH, Skv, 128] -> Vt [BH, 128, Skv_pad] (keys contiguous), zero beyond Skv.
-// CTA: one head and 64 keys; 256 threads.
-__global__ void __launch_bounds__(256) transpose_v_kernel(const uint16_t* __restrict__ V, uint16_t* __restrict__ Vt,
-                                                          int Skv, int Skv_pad) {
-  __shared__ __align__(16) uint16_t tile[64][AT_D + 8];
-  const int bh = blockIdx.y;
-  const int k0 = blockIdx.x * 64;
-  const uint16_t* src = V + static_cast<int64_t>(bh) * Skv * AT_D;
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int c = threadIdx.x + it * 256;  // 16-byte chunk: row c / 16, columns 8 * (c % 16) ..
-    const int row = c >> 4;
-    const int col = (c & 15) * 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (k0 + row < Skv) v = __ldg(reinterpret_cast<const uint4*>(src + static_cast<int64_t>(k0 + row) * AT_D + col));
-    *reinterpret_cast<uint4*>(&tile[row][col]) = v;
-  }
-  __syncthreads();
-  uint16_t* dst = Vt + static_cast<int64_t>(bh) * AT_D * Skv_pad;
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int c = threadIdx.x + it * 256;  // 8 keys of one head dimension: d = c / 8, keys 8 * (c % 8) ..
-    const int d = c >> 3;
-    const int kc = (c & 7) * 8;
-    if (k0 + kc >= Skv_pad) continue;
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      w[e] = static_cast<uint32_t>(tile[kc + 2 * e][d]) | (static_cast<uint32_t>(tile[kc + 2 * e + 1][d]) << 16);
-    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(d) * Skv_pad + k0 + kc) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 attn_tensor_map_encoder() {
@@ -524,19 +496,16 @@ bool encode_3d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct AttnWs {
-  size_t qq, sq, kq, sk, vt, total;
-  int64_t skv_pad;
+  size_t qq, sq, kq, sk, total;
 };
 
 AttnWs attn_ws_layout(int64_t BH, int64_t Sq, int64_t Skv) {
   AttnWs w;
-  w.skv_pad = (Skv + 7) / 8 * 8;
   w.qq = 256;
   w.sq = align_up(w.qq + static_cast<size_t>(BH * Sq) * AT_D, 256);
   w.kq = align_up(w.sq + 4 * static_cast<size_t>(BH * Sq), 1024);
   w.sk = align_up(w.kq + static_cast<size_t>(BH * Skv) * AT_D, 256);
-  w.vt = align_up(w.sk + 4 * static_cast<size_t>(BH * Skv), 1024);
-  w.total = align_up(w.vt + 2 * static_cast<size_t>(BH) * AT_D * static_cast<size_t>(w.skv_pad), 256);
+  w.total = align_up(w.sk + 4 * static_cast<size_t>(BH * Skv), 256);
   return w;
 }
 
@@ -577,13 +546,11 @@ convrot_status convrot_attention_int8(const void* Q, const void* K, const void* 
   float* sq = reinterpret_cast<float*>(wsb + lay.sq);
   int8_t* Kq = reinterpret_cast<int8_t*>(wsb + lay.kq);
   float* sk = reinterpret_cast<float*>(wsb + lay.sk);
-  uint16_t* Vt = reinterpret_cast<uint16_t*>(wsb + lay.vt);
 
   CUtensorMap tq, tk, tv;
   if (!encode_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Qq, AT_D, Sq, BH, AT_D, Sq * AT_D, AT_D, AT_BQ) ||
       !encode_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, Kq, AT_D, Skv, BH, AT_D, Skv * AT_D, AT_D, AT_BK) ||
-      !encode_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Vt, lay.skv_pad, AT_D, BH, 2 * lay.skv_pad,
-                 2 * AT_D * lay.skv_pad, 64, AT_D))
+      !encode_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, AT_D, Skv, BH, 2 * AT_D, 2 * AT_D * Skv, 64, AT_BK))
     return CONVROT_ERR_INVALID_ARG;
 
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return CONVROT_ERR_CUDA;
@@ -606,9 +573,6 @@ convrot_status convrot_attention_int8(const void* Q, const void* K, const void* 
   rq.dst = Kq;
   rq.scale = sk;
   if (launch_rotate_quant(AT_D, kRqActivation, rq, s) != cudaSuccess) return CONVROT_ERR_CUDA;
-  transpose_v_kernel<<<dim3(static_cast<unsigned>((lay.skv_pad + 63) / 64), static_cast<unsigned>(BH)), 256, 0, s>>>(
-      static_cast<const uint16_t*>(V), Vt, static_cast<int>(Skv), static_cast<int>(lay.skv_pad));
-  if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
 
   AttnParams ap{};
   ap.BH = static_cast<int>(BH);
