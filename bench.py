@@ -72,7 +72,7 @@ PROBE_OPS_PER_ITER_PER_PAIR = 2.0 * 256 * 256 * 128  # four 256x256x32 MMAs
 GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh"]
 GEMM_TRAFFIC = {
     "dit_qkv_1024": {"bytes": 42615808 + 42857728,
-                     "sources_sha256": "1c8ee27f2c5a355a7837004bfc0cba699331b36299585fe8e28a2be9d0e8bafa"},
+                     "sources_sha256": "65f86525711b6149634edf86e9fb88da44e85bdf0578f03d98f8d15e288097aa"},
 }
 
 # Every layer shape of the workload table, timed after the headline.
