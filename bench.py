@@ -435,7 +435,7 @@ def bench_config(cr, L, name: str, dev, stream, reps: int, peaks: dict, i8_peak,
     ns = sets_for(per_set)
     sets = [{"X": X0 if i == 0 else X0.clone(), "Wq": Wq0 if i == 0 else Wq0.clone(),
              "Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
-             "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=dev),
+             "ws": torch.zeros((ws_bytes,), dtype=torch.uint8, device=dev),
              "Xq": torch.empty((M, K), dtype=torch.int8, device=dev),
              "sx": torch.empty((M,), dtype=torch.float32, device=dev)} for i in range(ns)]
     sp = stream.cuda_stream
@@ -531,7 +531,7 @@ def bench_attention(cr, dev, stream, reps: int, clock_index: int, i8_peak) -> di
     sets = []
     for _ in range(ns):
         q, k, v = (torch.randn((BH, S, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(3))
-        ws = torch.empty((cr.convrot_attention_workspace_bytes(BH, S, S, D),), dtype=torch.uint8, device=dev)
+        ws = torch.zeros((cr.convrot_attention_workspace_bytes(BH, S, S, D),), dtype=torch.uint8, device=dev)
         sets.append((q, k, v, torch.empty_like(q), ws))
 
     def call(i):
@@ -715,7 +715,7 @@ def main():
         sets.append({
             "X": X0.clone(), "Wq": Wq0.clone(),
             "Y": torch.empty((M, N), dtype=io_dtype, device=dev),
-            "ws": torch.empty((ws_bytes,), dtype=torch.uint8, device=dev),
+            "ws": torch.zeros((ws_bytes,), dtype=torch.uint8, device=dev),
         })
     del X0
     stream = torch.cuda.current_stream(dev)
