@@ -128,7 +128,10 @@ __device__ __forceinline__ float write_p_half(const float (&u)[128], int h, floa
                                               uint8_t* row, int sw) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m_ref, -m_ref);
-  float2 sum2 = make_float2(0.0f, 0.0f);
+  // four partial sums: one chain of 64 dependent adds per half would leave its
+  // latency exposed with two softmax warps per scheduler (3 % of the call)
+  float2 sum2[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                    make_float2(0.0f, 0.0f)};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     uint32_t w[4];
@@ -142,12 +145,13 @@ __device__ __forceinline__ float write_p_half(const float (&u)[128], int h, floa
         pp.x = (k < nvalid) ? pp.x : 0.0f;
         pp.y = (k + 1 < nvalid) ? pp.y : 0.0f;
       }
-      sum2 = __fadd2_rn(sum2, pp);
+      sum2[e] = __fadd2_rn(sum2[e], pp);
       w[e] = pack_bf16x2(pp.x, pp.y);
     }
     *reinterpret_cast<uint4*>(row + ((i ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  return sum2.x + sum2.y;
+  const float2 st = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
+  return st.x + st.y;
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 2)
