@@ -60,7 +60,8 @@ INT8_OVER_BF16 = 4.5 / 2.25  # nominal dense int8 : dense bf16 tensor rate on B2
 NOMINAL_INT8_TOPS = 4500.0  # datasheet dense int8 (context only)
 WS_CLOCK_RECORD_OFFSET = 64  # CONVROT_WS_CLOCK_RECORD_OFFSET in include/convrot.h
 PEAK_BURST_REGION_MS = 50.0
-IDLE_BEFORE_REGION_S = 0.5  # idle time before the per-launch timed region  # timed regions up to this long are compared with the probe's burst rate
+IDLE_BEFORE_REGION_S = 0.5  # idle time before the per-launch timed region
+WARMUP_AFTER_IDLE = 30  # untimed steps between that idle time and the region  # timed regions up to this long are compared with the probe's burst rate
 SMALL_M = 64  # up to this many tokens the layer's GEMM is the weight-streaming form
 PROBE_OPS_PER_ITER_PER_PAIR = 2.0 * 256 * 256 * 128  # four 256x256x32 MMAs
 
@@ -779,7 +780,7 @@ def main():
         # after the headline loop the GPU still holds the lower clock its power limit
         # set there (the clock record below says which clock the GEMM ran at).
         time.sleep(IDLE_BEFORE_REGION_S)
-        for i in range(args.warmup):
+        for i in range(max(args.warmup, WARMUP_AFTER_IDLE)):
             timed_step(i, ev[i % len(ev)])
         torch.cuda.synchronize(dev)
         barrier()
@@ -789,6 +790,7 @@ def main():
         barrier()
         t_layer = max_over_ranks(statistics.mean(e[0].elapsed_time(e[2]) for e in ev))
         t_first = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+        t_first_med = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in ev))
         t_second = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
         t_second_med = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in ev))
         t_second_min = max_over_ranks(min(e[1].elapsed_time(e[2]) for e in ev))
@@ -956,7 +958,8 @@ def main():
         "kernels": {
             "rotate_quant_kernel (first launch of the step, events)": {
                 "us": t_first * 1e3, "bound": "hbm", "achieved": q_bytes / (t_first * 1e-3) / 1e9, "unit": "GB/s",
-                "peak": hbm, "frac": q_bytes / (t_first * 1e-3) / 1e9 / hbm},
+                "peak": hbm, "frac": q_bytes / (t_first * 1e-3) / 1e9 / hbm,
+                "us_median": (t_first_med * 1e3) if not variant else None},
             "rotate_quant_kernel (standalone, timed alone)": {
                 "us": t_q * 1e3, "bound": "hbm", "achieved": q_gbs, "unit": "GB/s", "peak": hbm,
                 "frac": q_gbs / hbm, "algorithmic_bytes": q_bytes},
