@@ -1498,12 +1498,19 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
   p.num_m_blocks = (p.M + 2 * BM - 1) / (2 * BM);  // 256-row pair blocks
   p.num_n_blocks = (p.N + BN - 1) / BN;
   p.num_k_blocks = (p.K + BK - 1) / BK;
-  // Activation codes of at most 32 MiB stay in L2 for the whole launch: then one
-  // group over every pair-row reads each weight panel from DRAM once (2-3 % faster
-  // on the 4608-token layers than groups of 16, whose remainder group reads the
-  // weight again); larger ones go in groups of 16 pair-rows.
-  if (p.group_m <= 0)
-    p.group_m = static_cast<int64_t>(p.M) * p.K <= (int64_t(32) << 20) ? p.num_m_blocks : CONVROT_PAIR_GROUP_M;
+  // Tile order by what stays in L2 for the whole launch. Activation codes of at
+  // most 32 MiB: one group over every pair-row (N outside), so the codes stay and
+  // each weight panel is read from DRAM once (1.8-2.9 % faster on the 4608-token
+  // K = 3072 layers than groups of 16). Else a weight of at most 40 MiB: groups
+  // of one pair-row (N inside), so the weight stays and each pair-row of codes is
+  // read once (1.5-4.5 % faster on the 2048² MLP and the down projection). Else
+  // groups of 16 pair-rows.
+  if (p.group_m <= 0) {
+    const int64_t a_bytes = static_cast<int64_t>(p.M) * p.K, b_bytes = static_cast<int64_t>(p.N) * p.K;
+    p.group_m = a_bytes <= (int64_t(32) << 20)   ? p.num_m_blocks
+                : b_bytes <= (int64_t(40) << 20) ? 1
+                                                  : CONVROT_PAIR_GROUP_M;
+  }
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int sms = sm_count();
   if (sms < 2) return cudaErrorInvalidDevice;
