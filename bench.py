@@ -505,6 +505,11 @@ def bench_config(cr, L, name: str, dev, stream, reps: int, peaks: dict, i8_peak,
         "quant_in_step_us_median": qi_med * 1e3,
         "quant_in_step_frac_hbm": q_bytes / (qi_med * 1e-3) / 1e9 / hbm,
     }
+    if L.convrot_linear_launch_count(M, N, K, g) == 1:
+        # one kernel rotates, quantises and multiplies: the "GEMM" events bracket all of it
+        out["layer_kernels"] = "one (tokens quantised inside the weight-streaming GEMM)"
+        out["quant_in_step_us_median"] = None
+        out["quant_in_step_frac_hbm"] = None
     if i8_peak:
         out["gemm_frac_i8_peak_median"] = out["gemm_tops_median"] / i8_peak
     if M <= 128:

@@ -146,8 +146,16 @@ CONVROT_API convrot_status convrot_quant_act(const void* X, int64_t M, int64_t K
  * The int8 x int8 product accumulates exactly in int32 on the tcgen05 tensor
  * cores (InvokeAI "int8 Compute", second paragraph); dequantisation and the
  * bias are fused into the GEMM epilogue. Two kernels (rotate+quantise, then
- * the GEMM, chained with programmatic dependent launch);
- * convrot_linear_launch_count reports the number for a shape.
+ * the GEMM, chained with programmatic dependent launch), or, for a few tokens
+ * (M * K <= 16384, M <= 16, K <= 8192; bf16 dense rows), one weight-streaming
+ * kernel that rotates and quantises the tokens into shared memory itself
+ * (every CTA redundantly; the same arithmetic in the same order, so the same
+ * codes, scales and output bits as the two kernels);
+ * convrot_linear_launch_count reports the number for a shape. The GEMM
+ * kernels read the weight before they wait for the previous kernel on the
+ * stream (so that its stream overlaps that kernel's tail): Wq must not be
+ * written by a kernel that lets its dependents launch before it finishes
+ * (convrot_prepare_weight's kernels do not).
  *   X        [M,K] bf16, device.   M >= 0, N >= 1, K % g == 0, K <= CONVROT_MAX_K,
  *                                   N % 8 == 0.
  *   Wq       [N,K] int8, device (from convrot_prepare_weight with the same g).
@@ -268,7 +276,8 @@ CONVROT_API convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M
  * launch, ev_mid after the rotate+quantise kernel (may be NULL), ev_end
  * after the GEMM. The layer's and each kernel's device time can then be read with
  * cudaEventElapsedTime on the launching stream. ev_mid keeps the GEMM from
- * overlapping the first kernel's tail.
+ * overlapping the first kernel's tail. In the one-kernel form ev_mid is
+ * recorded right after ev_start (the rotate+quantise share reads 0).
  */
 CONVROT_API convrot_status convrot_linear_timed(const void* X, int64_t M, int64_t K, int g,
                                                 const int8_t* Wq, const float* w_scale, int64_t N,
@@ -277,7 +286,8 @@ CONVROT_API convrot_status convrot_linear_timed(const void* X, int64_t M, int64_
                                                 void* ev_start, void* ev_mid, void* ev_end,
                                                 convrot_stream_t stream);
 
-/* Kernel launches one convrot_linear call of this shape enqueues: 2, or 0 for M = 0 or an invalid shape. */
+/* Kernel launches one convrot_linear call of this shape enqueues: 2, 1 (the one-kernel form for a few
+ * tokens, see convrot_linear), or 0 for M = 0 or an invalid shape. */
 CONVROT_API int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g);
 
 /*

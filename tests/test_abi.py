@@ -140,6 +140,14 @@ def test_other_entry_points_reject_bad_arguments_on_host(L):
     assert L.convrot_linear_timed(FAKE, 64, 256, 256, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 30, None, None,
                                   FAKE, None) == 1
     assert L.convrot_linear_launch_count(4608, 9216, 3072, 256) == 2
+    # a few tokens (M * K <= 16384, M <= 16, K <= 8192): one kernel
+    assert L.convrot_linear_launch_count(1, 12288, 4096, 128) == 1
+    assert L.convrot_linear_launch_count(4, 12288, 4096, 128) == 1
+    assert L.convrot_linear_launch_count(2, 12288, 8192, 256) == 1
+    assert L.convrot_linear_launch_count(16, 12288, 1024, 256) == 1
+    assert L.convrot_linear_launch_count(5, 12288, 4096, 128) == 2
+    assert L.convrot_linear_launch_count(17, 12288, 512, 256) == 2
+    assert L.convrot_linear_launch_count(1, 12288, 8448, 256) == 2
     # the one-launch form: K beyond what one CTA's worker warps hold
     assert L.convrot_linear_one_launch(FAKE, 64, 20608, 128, FAKE, FAKE, 256, None, FAKE, FAKE, 1 << 40, None) == 2
     assert L.convrot_linear_one_launch(FAKE, 64, 256, 256, FAKE, FAKE, 256, None, None, FAKE, 1 << 30, None) == 1

@@ -373,6 +373,71 @@ def test_linear_weight_streaming_split_is_deterministic(cr):
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 
 
+# For a few tokens (M * K <= 16384) convrot_linear is one kernel that rotates
+# and quantises the tokens into shared memory itself: the same arithmetic in
+# the same order as the rotate+quantise kernel, so its codes, scales and
+# output equal those of the two halves (convrot_quant_act, then
+# convrot_gemm_dequant on the weight-streaming GEMM) bit for bit. Cases: the
+# text-encoder layer at 1 and 4 tokens, K at its limit (8192, two ring
+# stages), 16 tokens, more weight tiles than SMs, the smallest K, N not a
+# multiple of the tile rows, both g, a zero token among others.
+@pytest.mark.parametrize("M,N,K,g", [(1, 12288, 4096, 128), (4, 12288, 4096, 128), (2, 1032, 8192, 256),
+                                     (1, 4104, 8192, 128), (16, 19712, 1024, 256), (16, 8, 128, 128),
+                                     (7, 264, 256, 256), (11, 2056, 768, 256)])
+def test_linear_one_kernel_form_equals_the_two_halves(cr, M, N, K, g):
+    import torch
+
+    assert cr.lib().convrot_linear_launch_count(M, N, K, g) == 1
+    d = _random_layer(M, N, K, g)
+    if M > 2:
+        d["x"][M // 2] = 0  # an all-zero token: scale 0, codes 0
+    Wq, sw = cr.convrot_prepare_weight(to_torch_bf16(d["w"]), g)
+    X = to_torch_bf16(d["x"])
+    bias = to_torch_bf16(d["bias"])
+    ws = torch.zeros(cr.convrot_linear_workspace_bytes(M, N, K, g), dtype=torch.uint8, device="cuda")
+    Y = cr.convrot_linear(X, Wq, sw, g, bias, ws=ws)
+    Xq, sx = cr.convrot_quant_act(X, g)
+    Y2 = cr.convrot_gemm_dequant(Xq, sx, Wq, sw, bias)
+    torch.cuda.synchronize()
+    assert cr.convrot_read_device_status(ws) == 0
+    wsn = ws.cpu().numpy()
+    lay = linear_ws_layout(M, K)
+    sx_ws = wsn[lay["scale"]:lay["scale"] + 4 * M].view(np.float32)
+    xq_ws = wsn[lay["codes"]:lay["codes"] + M * K].view(np.int8).reshape(M, K)
+    assert np.array_equal(xq_ws, Xq.cpu().numpy())
+    assert np.array_equal(sx_ws.view(np.uint32), sx.cpu().numpy().view(np.uint32))
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    # and the oracle: near-tie codes only, every output element within its bound
+    ref = oracle.linear(oracle.bf16_to_f64(d["x"]), *oracle.prepare_weight(oracle.bf16_to_f64(d["w"]), g), g,
+                        oracle.bf16_to_f64(d["bias"]))
+    assert nrmse(bf16_tensor_to_f64(Y), ref) <= NRMSE_TOL
+
+
+def test_linear_one_kernel_form_back_to_back_on_rotating_buffers(cr):
+    # calls that overlap through programmatic launch: each one's weight stream
+    # starts while the previous call runs; every output must match its own
+    # two-halves result
+    import torch
+
+    M, N, K, g = 4, 12288, 4096, 128
+    layers = []
+    for i in range(3):
+        d = _random_layer(M + i - 2, N, K, g)
+        Wq, sw = cr.convrot_prepare_weight(to_torch_bf16(d["w"]), g)
+        X = to_torch_bf16(d["x"])
+        layers.append((X, Wq, sw, cr.convrot_gemm_dequant(*cr.convrot_quant_act(X, g), Wq, sw)))
+    torch.cuda.synchronize()
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, N, K, g), dtype=torch.uint8, device="cuda")
+    outs = []
+    for r in range(12):
+        X, Wq, sw, _ = layers[r % 3]
+        outs.append((r % 3, cr.convrot_linear(X, Wq, sw, g, ws=ws)))
+    torch.cuda.synchronize()
+    assert cr.convrot_read_device_status(ws) == 0
+    for i, y in outs:
+        assert torch.equal(y.view(torch.int16), layers[i][3].view(torch.int16))
+
+
 @pytest.mark.parametrize("M,N,K,g", [(130, 264, 20480, 256),   # largest K of the one-launch form
                                      (1, 16, 384, 128), (385, 520, 1024, 256), (64, 256, 256, 256)])
 def test_linear_one_launch_matches_oracle(cr, M, N, K, g):

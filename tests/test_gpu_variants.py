@@ -123,6 +123,7 @@ CASES = [
     ("dit_mlp_up_1024", BF16, TENSOR, GELU),
     ("dit_mlp_up_1024", F16, CHANNEL, GELU),
     ("textenc_m16", BF16, CHANNEL, GELU),
+    ("textenc_m1", BF16, CHANNEL, NONE),
     ("textenc_m16", F16, TENSOR, NONE),
     ("textenc_m128", F16, CHANNEL, NONE),
 ]
@@ -243,11 +244,13 @@ def test_gelu_epilogue_against_the_exact_function(cr, name, M):
         assert np.all(np.abs(y[m] - ref) <= bound + 1e-12), np.max(np.abs(y[m] - ref) - bound)
 
 
-@pytest.mark.parametrize("name,dtype,act", [("tiny", BF16, NONE), ("dit_qkv_1024", F16, GELU),
-                                            ("textenc_m16", BF16, GELU), ("textenc_m128", F16, NONE)])
-def test_strided_rows_and_addend_match_oracle(cr, name, dtype, act):
-    # X and Y live inside wider row-major buffers (row strides K + 64 and N + 40),
-    # the addend shares Y's stride; the oracle sees the dense values
+@pytest.mark.parametrize("name,dtype,act,x_pad", [("tiny", BF16, NONE, 64), ("dit_qkv_1024", F16, GELU, 64),
+                                                  ("textenc_m16", BF16, GELU, 64), ("textenc_m128", F16, NONE, 64),
+                                                  ("textenc_m16", BF16, GELU, 0), ("textenc_m1", BF16, GELU, 0)])
+def test_strided_rows_and_addend_match_oracle(cr, name, dtype, act, x_pad):
+    # X and Y live inside wider row-major buffers (row strides K + x_pad and
+    # N + 40), the addend shares Y's stride; the oracle sees the dense values.
+    # Dense bf16 rows of one token (x_pad 0, textenc_m1) take the one-kernel form.
     import torch
 
     d = synth.make_workload(name)
@@ -260,7 +263,7 @@ def test_strided_rows_and_addend_match_oracle(cr, name, dtype, act):
     rng = np.random.default_rng(21)
     zb = _as_dtype_bits(synth.f32_to_bf16_bits((rng.standard_normal((M, N)) * 0.05).astype(np.float32)), dtype)
     Wq, sw = cr.convrot_prepare_weight_ex(_to_torch(wb, dtype), g, TENSOR)
-    ldx, ldy = K + 64, N + 40
+    ldx, ldy = K + x_pad, N + 40
     Xbig = _to_torch(np.zeros((M, ldx), np.uint16), dtype)
     Xbig[:, :K] = _to_torch(xb, dtype)
     Ybig = torch.full((M, ldy), float("nan"), dtype=Xbig.dtype, device="cuda")

@@ -118,13 +118,9 @@ struct EpiOptions {
   }
 };
 
-convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, int64_t M, int64_t N, int64_t K,
-                        const float* x_scale, const float* w_scale, const void* bias, int* status,
-                        cudaStream_t stream, EpiOptions opt = EpiOptions(), int32_t* split_part = nullptr,
-                        unsigned* split_count = nullptr) {
+convrot::GemmParams gemm_params(int64_t M, int64_t N, int64_t K, const float* x_scale, const float* w_scale,
+                                const void* bias, int* status, const EpiOptions& opt) {
   convrot::GemmParams p{};
-  p.split_part = split_part;
-  p.split_count = split_count;
   p.out_f16 = opt.out_f16;
   p.wscale_per_channel = opt.wscale_per_channel;
   p.addend = static_cast<const uint16_t*>(opt.addend);
@@ -141,8 +137,19 @@ convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, 
                                                                           CONVROT_WS_CLOCK_RECORD_OFFSET);
   p.timeout_ns = kWaitTimeoutNs;
   p.group_m = 0;
+  return p;
+}
+
+convrot_status run_gemm(int epi, const int8_t* Xq, const int8_t* Wq, void* out, int64_t M, int64_t N, int64_t K,
+                        const float* x_scale, const float* w_scale, const void* bias, int* status,
+                        cudaStream_t stream, EpiOptions opt = EpiOptions(), int32_t* split_part = nullptr,
+                        unsigned* split_count = nullptr) {
+  convrot::GemmParams p = gemm_params(M, N, K, x_scale, w_scale, bias, status, opt);
+  p.split_part = split_part;
+  p.split_count = split_count;
   return from_cuda(convrot::launch_gemm_i8(epi, Xq, Wq, out, p, stream));
 }
+
 
 }  // namespace
 
@@ -187,8 +194,10 @@ convrot_status convrot_prepare_weight_ex(const void* W, int dtype, int64_t N, in
   p.status = nullptr;
   p.timeout_ns = kWaitTimeoutNs;
   if (wscale_mode == CONVROT_WSCALE_CHANNEL) {
-    // one scale per weight row: the per-row (activation) form of the kernel
+    // one scale per weight row: the per-row (activation) form of the kernel,
+    // which lets its dependents launch only at exit (they may read the weight early)
     p.tensor_absmax = nullptr;
+    p.late_trigger = 1;
     return from_cuda(convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s));
   }
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < convrot_prepare_weight_workspace_bytes())
@@ -246,6 +255,12 @@ size_t convrot_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int g) {
 }  // extern "C"
 
 namespace {
+
+// Whether convrot_linear (and its variants) run the layer as the one fused
+// weight-streaming kernel: M * K <= 16384 (at most 16 tokens), bf16 dense rows.
+bool linear_is_one_kernel(int64_t M, int64_t K, const EpiOptions& opt) {
+  return opt.out_f16 == 0 && opt.ldx == 0 && convrot::smallm_fused_shape(M, K);
+}
 
 // The layer: the rotate+quantise kernel followed by the GEMM, or (one_launch)
 // the single kernel whose worker warps rotate and quantise while its tensor
@@ -318,6 +333,23 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
     return CONVROT_OK;
   }
 
+  const int epi = opt.act ? convrot::kEpiDequantGenGelu
+                           : (opt.general() ? convrot::kEpiDequantGen : convrot::kEpiDequantBf16);
+  if (linear_is_one_kernel(M, K, opt)) {
+    // a few tokens: one kernel rotates and quantises them into shared
+    // memory and streams the weight; its CTA 0 also leaves the codes and the
+    // token scales in the workspace
+    convrot::GemmParams gp = gemm_params(M, N, K, nullptr, w_scale, bias, status, opt);
+    gp.X = static_cast<const uint16_t*>(X);
+    gp.Xq = Xq;
+    gp.x_scale_out = x_scale;
+    for (cudaEvent_t ev : {ev0, ev1})
+      if (ev != nullptr && cudaEventRecord(ev, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (convrot::launch_linear_smallm_fused(epi, g, Wq, Y, gp, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    if (ev2 != nullptr && cudaEventRecord(ev2, s) != cudaSuccess) return CONVROT_ERR_CUDA;
+    return CONVROT_OK;
+  }
+
   convrot::RotQuantParams p{};
   p.src = static_cast<const uint16_t*>(X);
   p.in_f16 = opt.out_f16;  // X, bias and Y share the compute dtype
@@ -343,8 +375,6 @@ convrot_status linear_impl(const void* X, int64_t M, int64_t K, int g, const int
   if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (convrot::launch_rotate_quant(g, convrot::kRqActivation, p, s) != cudaSuccess) return CONVROT_ERR_CUDA;
   if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return CONVROT_ERR_CUDA;
-  const int epi = opt.act ? convrot::kEpiDequantGenGelu
-                           : (opt.general() ? convrot::kEpiDequantGen : convrot::kEpiDequantBf16);
   const convrot_status st =
       run_gemm(epi, Xq, Wq, Y, M, N, K, x_scale, w_scale, bias, status, s, opt, split_part, split_count);
   if (st != CONVROT_OK) return st;
@@ -393,7 +423,7 @@ convrot_status convrot_linear_ex(const void* X, int dtype, int64_t M, int64_t K,
 
 int convrot_linear_launch_count(int64_t M, int64_t N, int64_t K, int g) {
   if (check_rotation_shape(M, K, g) != CONVROT_OK || check_gemm_shape(M, N, K, 8) != CONVROT_OK) return 0;
-  return M == 0 ? 0 : 2;
+  return M == 0 ? 0 : linear_is_one_kernel(M, K, EpiOptions()) ? 1 : 2;
 }
 
 convrot_status convrot_linear_one_launch(const void* X, int64_t M, int64_t K, int g, const int8_t* Wq,

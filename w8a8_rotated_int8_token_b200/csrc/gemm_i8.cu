@@ -1006,35 +1006,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 // exact, so the result does not depend on the order of arrival, and no CTA
 // ever waits for another.
 
-constexpr int SM_BW = 128;  // weight rows per tile
+constexpr int SM_BW = 128;  // weight rows the MMA covers (M = 128); a tile loads at most this many
 
 // KPS: consecutive 128-byte k-blocks per ring stage (one TMA box each), so
 // that each weight row is read in runs of KPS * 128 bytes.
 #ifndef CONVROT_SMALLM_KPS
 #define CONVROT_SMALLM_KPS 2
 #endif
-
-template <int BNT, int KPS = 1>
-struct SmallSmem {
-  static constexpr int kW1 = SM_BW * BK;  // 16 KB: one weight k-block
-  static constexpr int kX1 = BNT * BK;    // 2..8 KB: one token k-block
-  static constexpr int kW = kW1 * KPS;
-  static constexpr int kX = kX1 * KPS;
-  static constexpr int kFit = (KPS == 1 ? 200 * 1024 : 216 * 1024) / (kW + kX);
-#ifdef CONVROT_SMALLM_STAGES
-  static constexpr int kStages = CONVROT_SMALLM_STAGES < kFit ? CONVROT_SMALLM_STAGES : kFit;
-#else
-  static constexpr int kStages = kFit > 10 ? 10 : kFit;
+// Whole-tile form, off: size the weight tile so that the tiles cover the SMs
+// once (ceil(N / SMs) rows, rounded up to the 8-row swizzle atom) instead of
+// 128 rows on ceil(N / 128) SMs. Measured slower on every text-encoder shape
+// (M = 1, N = 12288: 15.4 against 14.5 us per layer call on 140 SMs; N = 4096:
+// 15.8 against 13.0 us).
+#ifndef CONVROT_SMALLM_FIT_ROWS
+#define CONVROT_SMALLM_FIT_ROWS 0
 #endif
-  static constexpr int kOffW = 0;
-  static constexpr int kOffX = kStages * kW;
-  static constexpr int kOffBar = kStages * (kW + kX);
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;
+
+// Fused form (FQ): for a few tokens the kernel rotates and quantises them
+// itself, into a shared-memory copy of all K codes, so that a layer call is
+// one launch whose weight stream starts while the previous kernel still runs.
+// Its CTAs have kSmallQuantWarps more warps, and warps 2.. (the epilogue warps
+// and those) do the quantisation, redundantly in every CTA, in passes of
+// kSmallQuantThreads * 64 values. Used where one pass holds all tokens
+// (M * K <= 16384): each further pass costs about 2.5 us (the token loads
+// queue behind the weight stream already in flight), so at M = 16, K = 4096
+// the two-kernel form is faster (14.6 against 23.6 us); at M = 1 the fused
+// form saves the rotate kernel and two dependent-launch hops (13.3 against
+// 14.5 us).
+#ifndef CONVROT_SMALLM_FUSED
+#define CONVROT_SMALLM_FUSED 1
+#endif
+// Whole tiles, off: the weight panel of each tile (a contiguous range of rows)
+// prefetched into L2 once the first ring stages are requested. Measured
+// slower on every text-encoder shape (0.5-1.5 us per layer call).
+#ifndef CONVROT_SMALLM_PANEL_PREFETCH
+#define CONVROT_SMALLM_PANEL_PREFETCH 0
+#endif
+constexpr int kSmallQuantM = 16;                          // tokens (one 16-column MMA)
+constexpr int kSmallQuantMaxK = 8192;                     // codes: 16 x K bytes of shared memory
+constexpr int kSmallQuantWarps = 4;                       // warps added to the CTA
+constexpr int kSmallQuantThreads = (EPI_WARPS + kSmallQuantWarps) * 32;  // warps 2..9
+constexpr uint32_t kSmallPanelChunk = 32 * 1024;          // bytes per L2 prefetch instruction
+
+// Shared memory of the weight-streaming kernel: a 1 KB header (barriers,
+// TMEM address, flags, the fused form's token scales and row maxima), then
+// (fused form) the token codes, then the weight ring (S stages of R weight
+// rows x KPS k-blocks, packed: k-block i of stage s starts (s * KPS + i) * R *
+// 128 bytes in), then (two-kernel form) the token ring. The MMA always reads
+// 128 weight rows from a k-block's start; the rows past R belong to the next
+// box (or, for the ring's last box, to what follows, inside the allocation)
+// and only fill TMEM lanes the epilogue never reads.
+template <int BNT, int KPS = 1, bool FQ = false>
+struct SmallSmem {
+  static constexpr int kX1 = BNT * BK;  // 2..8 KB: one token k-block
+  static constexpr int kX = FQ ? 0 : kX1 * KPS;
+  static constexpr int kMaxStages = 16;
+  static constexpr int kRing = KPS == 1 ? 200 * 1024 : 216 * 1024;
+  static constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 1 + 1;
+  static constexpr int kOffBar = 0;
   static constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemPtr + 8;
   static constexpr int kOffLast = kOffAbort + 8;  // split form: "this CTA finishes the tile"
-  static constexpr int kBytes = kOffLast + 8;
-  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kOffXs = 512;                       // fused form: the token scales
+  static constexpr int kOffRmax = kOffXs + 4 * kSmallQuantM;  // fused form: 2 x 16 row maxima
+  static constexpr int kHeader = 1024;
+  static_assert(kOffLast + 8 <= kOffXs && kOffRmax + 8 * kSmallQuantM <= kHeader, "header overflow");
+  static_assert(!FQ || BNT == kSmallQuantM, "the fused form has one 16-token MMA column block");
+  static constexpr int kAlloc = 1024 + kHeader + kRing;  // + the 1 KB alignment slack
+  // bytes of the fused form's codes (all K of BNT tokens)
+  __host__ __device__ static constexpr int codes_bytes(int K) { return FQ ? BNT * K : 0; }
+  // weight bytes of one stage for R rows
+  __host__ __device__ static constexpr int w_stage(int rows) { return rows * BK * KPS; }
+  // ring stages for R rows: the MMA's overrun past the last box ((128 - R)
+  // rows) stays inside the allocation
+  __host__ __device__ static constexpr int stages(int rows, int K) {
+    const int fit = (kRing - codes_bytes(K) - (SM_BW - rows) * BK) / (w_stage(rows) + kX);
+#ifdef CONVROT_SMALLM_STAGES
+    const int cap = CONVROT_SMALLM_STAGES < kMaxStages ? CONVROT_SMALLM_STAGES : kMaxStages;
+#else
+    const int cap = kMaxStages;
+#endif
+    return fit < cap ? fit : cap;
+  }
 };
 
 // The sequence of (weight tile, k-block range) segments a CTA works on; every
@@ -1085,16 +1138,16 @@ __device__ __forceinline__ void epi_named_barrier() { asm volatile("bar.sync 1, 
 
 // One output value of the weight-streaming epilogue: token m, output channel n.
 template <int EPI>
-__device__ __forceinline__ void smallm_store(const GemmParams& p, void* out, int m, int n, int32_t acc, float sw,
-                                             float swn, float bn) {
+__device__ __forceinline__ void smallm_store(const GemmParams& p, void* out, int m, int n, int32_t acc, float xs,
+                                             float sw, float swn, float bn) {
   if (EPI == kEpiDequantBf16) {
-    const float y = fmaf(static_cast<float>(acc), __ldg(p.x_scale + m) * sw, bn);
+    const float y = fmaf(static_cast<float>(acc), xs * sw, bn);
     static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(y);
   } else if (epi_is_general(EPI)) {
     const int64_t at = static_cast<int64_t>(m) * (p.ldy ? p.ldy : p.N) + n;
     float bias_add = bn;
     if (p.addend != nullptr) bias_add += out16_to_f32(__ldg(p.addend + at), p.out_f16 != 0);
-    float y = fmaf(static_cast<float>(acc), __ldg(p.x_scale + m) * swn, bias_add);
+    float y = fmaf(static_cast<float>(acc), xs * swn, bias_add);
     if (EPI == kEpiDequantGenGelu) y = gelu_erf(y);
     if (p.out_f16)
       static_cast<__half*>(out)[at] = __float2half_rn(y);
@@ -1105,12 +1158,133 @@ __device__ __forceinline__ void smallm_store(const GemmParams& p, void* out, int
   }
 }
 
-template <int EPI, int BNT, int KPS>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// Fused form: the rotation and quantisation of the M <= 16 tokens by the
+// kSmallQuantThreads threads of warps 2.. (qt = their index), straight from
+// X in global memory into the shared-memory B operand: code k of token m at
+// codes + (k / 128) * BNT * 128 + m * 128 + (k % 128), its 16-byte chunk
+// swizzled by m % 8 (the layout a 128-byte-swizzled TMA box of BNT rows
+// gives), the token scales into xs. The arithmetic and its order are those
+// of the rotate+quantise kernel (pair stage on the top piece bit from the
+// input words, the lane's own stages, the shuffle stages on the lane bits;
+// absmax; the correctly rounded scale; code = rne(u * 127 / absmax_u)), so
+// every code and scale equals that kernel's. Rows past M are not written:
+// their MMA columns are never stored. With gcodes (CTA 0) the codes and
+// scales also go to global memory ([M, K] row-major and [M]).
+template <int G, int BNT>
+__device__ __forceinline__ void smallm_quant(const GemmParams& p, uint8_t* codes, float* xs, unsigned* rmax2,
+                                             int qt, int8_t* gcodes, float* gscale) {
+  using namespace fwht;
+  constexpr int LG = G / 64;
+  constexpr int PIECE = G / 8;
+  const int K = p.K;
+  const int tpr = K / 64;                     // threads per token (64 values each)
+  const int rpp = kSmallQuantThreads / tpr;   // tokens per pass (>= 2 for K <= 8192)
+  const int row_in_pass = qt / tpr;
+  const int t = qt - row_in_pass * tpr;
+  const int grp = t / LG;
+  const int l = t - grp * LG;
+  const bool lane_active = row_in_pass < rpp;
+  for (int pass = 0; pass * rpp < p.M; ++pass) {
+    const int row = pass * rpp + row_in_pass;
+    const bool valid = lane_active && row < p.M;
+    unsigned* rmax = rmax2 + (pass & 1) * BNT;
+    if (qt < BNT) rmax[qt] = 0u;
+    float2 v[4][8];
+    if (valid) {
+      const uint16_t* src = p.X + static_cast<int64_t>(row) * K + grp * G + 8 * l;
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(raw[j].x), "=r"(raw[j].y), "=r"(raw[j].z), "=r"(raw[j].w)
+                     : "l"(src + j * PIECE));
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const uint32_t aw[4] = {raw[jj].x, raw[jj].y, raw[jj].z, raw[jj].w};
+        const uint32_t bw[4] = {raw[jj + 4].x, raw[jj + 4].y, raw[jj + 4].z, raw[jj + 4].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          fwht_first_pair<false>(aw[q],
+                                 make_float2(__uint_as_float(bw[q] << 16), __uint_as_float(bw[q] & 0xFFFF0000u)),
+                                 v[jj][2 * q], v[jj][2 * q + 1]);
+      }
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[jj][e] = make_float2(0.0f, 0.0f);
+    }
+    fwht_lane_local(v);
+    fwht_lane_shuffle<LG>(v, l);
+    float m = absmax64_v3(v);
+#pragma unroll
+    for (int s = 1; s < LG; s <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+    named_barrier_sync(2, kSmallQuantThreads);  // this pass's row maxima are zero
+    if (valid && l == 0) atomicMax(&rmax[row_in_pass], __float_as_uint(m));
+    named_barrier_sync(2, kSmallQuantThreads);
+    if (valid) {
+      const float amax_u = __uint_as_float(rmax[row_in_pass]);
+      if (t == 0) {
+        const float sc = scale_of<G>(amax_u);
+        xs[row] = sc;
+        if (gscale != nullptr) gscale[row] = sc;
+      }
+      const CodeFactor cf = code_factor(amax_u);
+      if (cf.pre != 1.0f) {  // tiny row: multiply by 2^64 first (exact), then by ci
+        const float2 pre2 = make_float2(cf.pre, cf.pre);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[jj][e] = __fmul2_rn(v[jj][e], pre2);
+      }
+      const float2 ci2 = make_float2(cf.ci, cf.ci);
+      const float2 magic2 = make_float2(kRoundMagic, kRoundMagic);
+      uint8_t* const row_base = codes + row * BK;
+      const int sw = row & 7;
+      auto put8 = [&](int k, uint2 val) {  // 8 codes at columns k..k+7 (k % 8 == 0)
+        const int j = k & (BK - 1);
+        *reinterpret_cast<uint2*>(row_base + (k / BK) * (BNT * BK) + ((((j >> 4) ^ sw) << 4) | (j & 15))) = val;
+      };
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        float2 r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __ffma2_rn(v[jj][e], ci2, magic2);
+        // piece jj from the .x halves, piece jj+4 from the .y halves
+        uint2 lo, hi;
+        lo.x = pack4(r[0].x, r[1].x, r[2].x, r[3].x);
+        lo.y = pack4(r[4].x, r[5].x, r[6].x, r[7].x);
+        hi.x = pack4(r[0].y, r[1].y, r[2].y, r[3].y);
+        hi.y = pack4(r[4].y, r[5].y, r[6].y, r[7].y);
+        const int k = grp * G + jj * PIECE + 8 * l;
+        put8(k, lo);
+        put8(k + 4 * PIECE, hi);
+        if (gcodes != nullptr) {
+          int8_t* g8 = gcodes + static_cast<int64_t>(row) * K + k;
+          *reinterpret_cast<uint2*>(g8) = lo;
+          *reinterpret_cast<uint2*>(g8 + 4 * PIECE) = hi;
+        }
+      }
+    }
+  }
+  // the codes are read by the tensor cores (async proxy)
+  fence_proxy_async_smem();
+  named_barrier_sync(2, kSmallQuantThreads);
+}
+
+template <int EPI, int BNT, int KPS, int QG = 0>
+__global__ void __launch_bounds__(QG != 0 ? NUM_THREADS + 32 * kSmallQuantWarps : NUM_THREADS, 1)
     gemm_i8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                           void* __restrict__ out, const int8_t* __restrict__ Wq, const GemmParams p) {
-  using L = SmallSmem<BNT, KPS>;
-  constexpr int S = L::kStages;
+  constexpr bool FQ = QG != 0;  // fused form: the kernel quantises the tokens itself
+  using L = SmallSmem<BNT, KPS, FQ>;
+  const int R = p.tile_rows;  // weight rows per tile
+  const int S = L::stages(R, p.K);
+  const int kW1 = R * BK;  // one weight box
+  const int kW = kW1 * KPS;
+  const int off_w = L::kHeader + L::codes_bytes(p.K);
+  const int off_x = off_w + S * kW;
+  constexpr int kMaxS = L::kMaxStages;
   constexpr uint32_t kIdesc = idesc_i8(SM_BW, BNT);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1120,13 +1294,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tmem_full = bars + 2 * S;
   uint64_t* tmem_empty = tmem_full + 2;
   uint64_t* drain = tmem_empty + 2;
+  uint64_t* x_ready = drain + 1;  // fused form: the token codes are in shared memory
+  uint8_t* const codes = smem + L::kHeader;
+  float* const xs_s = reinterpret_cast<float*>(smem + L::kOffXs);
+  unsigned* const rmax_s = reinterpret_cast<unsigned*>(smem + L::kOffRmax);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::kOffTmemPtr);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::kOffLast);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_tiles = (p.N + SM_BW - 1) / SM_BW;
+  const int num_tiles = (p.N + R - 1) / R;
 
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmW);
@@ -1140,6 +1318,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tmem_empty[b], EPI_WARPS);
     }
     mbar_init(drain, 1);
+    mbar_init(x_ready, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -1153,23 +1332,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_ptr;
   // The weight stream does not depend on the previous kernel (see the pair
   // kernel): the weight loads of the first S stages go out before the wait,
-  // the activation-code loads and the token scales after it.
+  // the activation-code loads and the token scales after it. The fused form
+  // loads no tokens: its producer never waits, and it lets the next kernel
+  // launch as soon as the first stages and the panel prefetch are out.
 
   if (warp == 0) {
     if (lane == 0) {
       SmallSegments seg(p, num_tiles);
       int s = 0;
       uint32_t ph = 0;
-      int pending_phase[S];
+      int pending_phase[kMaxS];
       for (int i = 0; i < S; ++i) pending_phase[i] = -1;
       bool ok = true;
-      int early_s[S], early_kb[S];
+      int early_s[kMaxS], early_kb[kMaxS];
       int n_early = 0;
-      bool waited = false;
+      bool waited = FQ;
+      int issued = 0;
+      bool prefetched = !(CONVROT_SMALLM_PANEL_PREFETCH && !seg.split &&
+                          static_cast<int64_t>(p.N) * p.K <= (int64_t(64) << 20));
+      auto prefetch_panels = [&]() {
+        // this CTA's tiles (each R contiguous weight rows) into L2
+        for (int t = static_cast<int>(blockIdx.x); t < num_tiles; t += static_cast<int>(gridDim.x)) {
+          const int64_t r0 = static_cast<int64_t>(t) * R;
+          const int64_t r1 = r0 + R < p.N ? r0 + R : p.N;
+          const uint8_t* base = reinterpret_cast<const uint8_t*>(Wq) + r0 * p.K;
+          const int64_t bytes = (r1 - r0) * p.K;
+          for (int64_t off = 0; off < bytes; off += kSmallPanelChunk)
+            bulk_prefetch_l2(base + off, static_cast<uint32_t>(bytes - off < kSmallPanelChunk ? bytes - off
+                                                                                             : kSmallPanelChunk));
+        }
+        prefetched = true;
+        if (FQ) griddep_launch_dependents();
+      };
       auto load_x = [&](int st, int kb) {
 #pragma unroll
         for (int i = 0; i < KPS; ++i)
-          tma_load_2d(smem + L::kOffX + st * L::kX + i * L::kX1, &tmX, &full[st], (kb + i) * BK, 0);
+          tma_load_2d(smem + off_x + st * L::kX + i * L::kX1, &tmX, &full[st], (kb + i) * BK, 0);
       };
       auto release_early = [&]() {
         griddep_wait();
@@ -1184,11 +1382,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], L::kW + L::kX);
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kW + L::kX));
 #pragma unroll
           for (int i = 0; i < KPS; ++i)
-            tma_load_2d(smem + L::kOffW + s * L::kW + i * L::kW1, &tmW, &full[s], (kb + i) * BK, tile * SM_BW);
-          if (waited) {
+            tma_load_2d(smem + off_w + s * kW + i * kW1, &tmW, &full[s], (kb + i) * BK, tile * R);
+          if (FQ) {
+          } else if (waited) {
             load_x(s, kb);
           } else {
             early_s[n_early] = s;
@@ -1200,9 +1399,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             s = 0;
             ph ^= 1u;
           }
+          if (!prefetched && ++issued == S) prefetch_panels();
         }
       }
       if (!waited) release_early();
+      if (!prefetched && ok) prefetch_panels();
       griddep_launch_dependents();
       if (!ok) {
         raise_abort(abort, p.status);
@@ -1217,6 +1418,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      bool x_in = !FQ;  // fused form: the token codes are in shared memory
       int it = 0;
       int tile, k0, k1;
       while (ok && seg.get(tile, k0, k1)) {
@@ -1233,11 +1435,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
+          if (!x_in) {
+            if (!mbar_wait_bounded(x_ready, 0u, abort, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            x_in = true;
+          }
           tc_fence_after();
 #pragma unroll
           for (int i = 0; i < KPS; ++i) {
-            const uint32_t w_base = smem_addr(smem + L::kOffW + s * L::kW + i * L::kW1);
-            const uint32_t x_base = smem_addr(smem + L::kOffX + s * L::kX + i * L::kX1);
+            if (FQ && kb + i >= p.num_k_blocks) break;  // no codes past K (the weight box there is zeros)
+            const uint32_t w_base = smem_addr(smem + off_w + s * kW + i * kW1);
+            const uint32_t x_base = FQ ? smem_addr(codes + (kb + i) * L::kX1)
+                                       : smem_addr(smem + off_x + s * L::kX + i * L::kX1);
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k) {
               mma_i8(d, smem_desc_k_sw128(w_base + k * UMMA_K), smem_desc_k_sw128(x_base + k * UMMA_K), kIdesc,
@@ -1259,10 +1470,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_bounded(drain, 0u, nullptr, p.timeout_ns);
     }
   } else {
-    griddep_wait();  // the token scales (and the split counters' zeroing) come from the previous kernel
+    if constexpr (FQ) {
+      // warps 2..: wait for the previous kernel (X may be its output; this
+      // call's status word and output may still be read by it), clear the
+      // status word (CTA 0), rotate and quantise the tokens
+      griddep_wait();
+      if (blockIdx.x == 0 && threadIdx.x == 64 && p.status != nullptr) *p.status = 0;
+      const bool keep = blockIdx.x == 0 && p.Xq != nullptr && p.x_scale_out != nullptr;
+      smallm_quant<QG, BNT>(p, codes, xs_s, rmax_s, static_cast<int>(threadIdx.x) - 64, keep ? p.Xq : nullptr,
+                            keep ? p.x_scale_out : nullptr);
+      if (threadIdx.x == 64) mbar_arrive(x_ready);
+    } else {
+      griddep_wait();  // the token scales (and the split counters' zeroing) come from the previous kernel
+    }
+  }
+  if (warp >= 2 && warp < 2 + EPI_WARPS) {
     SmallSegments seg(p, num_tiles);
     const int q = warp & 3;
     const int nl = q * 32 + lane;  // weight row within the tile (TMEM lane)
+    const bool row_ok = nl < R;    // lanes past the tile's rows hold no output
     const float sw = epi_weight_scale<EPI>(p);
     int it = 0;
     int si = 0;  // segment index within this CTA
@@ -1271,7 +1497,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     while (seg.get(tile, k0, k1)) {
       const int b = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
-      const int n = tile * SM_BW + nl;
+      const int n = row_ok ? tile * R + nl : p.N;
       const bool whole = (k0 == 0 && k1 == seg.KB);
       float bn = 0.0f;
       float swn = sw;  // this thread's output channel's weight scale
@@ -1335,7 +1561,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (write_out && ok && n < p.N) {
 #pragma unroll
         for (int m = 0; m < BNT; ++m)
-          if (m < p.M) smallm_store<EPI>(p, out, m, n, acc[m], sw, swn, bn);
+          if (m < p.M) smallm_store<EPI>(p, out, m, n, acc[m], FQ ? xs_s[m] : __ldg(p.x_scale + m), sw, swn, bn);
       }
       ++it;
       ++si;
@@ -1536,16 +1762,27 @@ cudaError_t launch_pair(const int8_t* A, const int8_t* B, void* out, GemmParams 
 
 namespace {
 
+// Weight rows per tile of the weight-streaming form: whole tiles take the
+// fewest rows (a multiple of 8) that cover the N rows with one tile per SM;
+// the split form keeps 128-row tiles.
+int smallm_tile_rows(int N, int sms, bool split) {
+  if (!CONVROT_SMALLM_FIT_ROWS || split) return SM_BW;
+  const int per_sm = (N + sms - 1) / sms;
+  const int rows = (per_sm + 7) / 8 * 8;
+  return rows < SM_BW ? rows : SM_BW;
+}
+
 template <int EPI, int BNT, int KPS>
 cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  p.tile_rows = smallm_tile_rows(p.N, sms, p.split_part != nullptr);
   CUtensorMap tw, tx;
-  if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, SM_BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, p.tile_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, p.K, p.M, BK, BNT, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   p.num_k_blocks = (p.K + BK - 1) / BK;
-  const int tiles = (p.N + SM_BW - 1) / SM_BW;
-  const int sms = sm_count();
-  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int tiles = (p.N + p.tile_rows - 1) / p.tile_rows;
   int grid = tiles < sms ? tiles : sms;
   if (p.split_part != nullptr) {
     // every SM streams an equal share of the (tile, k-block) units
@@ -1569,6 +1806,42 @@ cudaError_t launch_smallm_t(const int8_t* A, const int8_t* B, void* out, GemmPar
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_i8_smallm_kernel<EPI, BNT, KPS>, tw, tx, out, B, p);
+}
+
+// The fused weight-streaming form (M <= kSmallQuantM): one kernel that
+// rotates and quantises the tokens (group size G) and multiplies them with
+// the weight; whole tiles only.
+template <int EPI, int G>
+cudaError_t launch_smallm_fq(const int8_t* B, void* out, GemmParams p, cudaStream_t stream) {
+  constexpr int BNT = 16, KPS = CONVROT_SMALLM_KPS;
+  using L = SmallSmem<BNT, KPS, true>;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  p.split_part = nullptr;
+  p.tile_rows = smallm_tile_rows(p.N, sms, false);
+  if (p.X == nullptr || p.M < 1 || p.M > kSmallQuantM || p.K > kSmallQuantMaxK || L::stages(p.tile_rows, p.K) < 2)
+    return cudaErrorInvalidValue;
+  CUtensorMap tw;
+  if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, p.K, p.N, BK, p.tile_rows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  p.num_k_blocks = (p.K + BK - 1) / BK;
+  const int tiles = (p.N + p.tile_rows - 1) / p.tile_rows;
+  const int grid = tiles < sms ? tiles : sms;
+  constexpr int smem = L::kAlloc;
+  static std::atomic<int> attr_done[kMaxDevices];
+  cudaError_t e = ensure_smem_attr(gemm_i8_smallm_kernel<EPI, BNT, KPS, G>, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(NUM_THREADS + 32 * kSmallQuantWarps);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_smallm_kernel<EPI, BNT, KPS, G>, tw, tw, out, B, p);
 }
 
 template <int EPI, int KPS>
@@ -1601,6 +1874,26 @@ cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out,
   if (epi == kEpiDequantGen) return launch_pair<kEpiDequantGen>(A, B, out, p, stream);
   if (epi == kEpiDequantGenGelu) return launch_pair<kEpiDequantGenGelu>(A, B, out, p, stream);
   if (epi == kEpiRawS32) return launch_pair<kEpiRawS32>(A, B, out, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+bool smallm_fused_shape(int64_t M, int64_t K) {
+  using L = SmallSmem<16, CONVROT_SMALLM_KPS, true>;
+  return CONVROT_SMALLM_FUSED && M >= 1 && M <= kSmallQuantM && K >= BK && K <= kSmallQuantMaxK &&
+         M * K <= int64_t(kSmallQuantThreads) * 64 && L::stages(SM_BW, static_cast<int>(K)) >= 2;
+}
+
+cudaError_t launch_linear_smallm_fused(int epi, int g, const int8_t* Wq, void* Y, GemmParams p,
+                                       cudaStream_t stream) {
+  if (g == 128) {
+    if (epi == kEpiDequantBf16) return launch_smallm_fq<kEpiDequantBf16, 128>(Wq, Y, p, stream);
+    if (epi == kEpiDequantGen) return launch_smallm_fq<kEpiDequantGen, 128>(Wq, Y, p, stream);
+    if (epi == kEpiDequantGenGelu) return launch_smallm_fq<kEpiDequantGenGelu, 128>(Wq, Y, p, stream);
+  } else if (g == 256) {
+    if (epi == kEpiDequantBf16) return launch_smallm_fq<kEpiDequantBf16, 256>(Wq, Y, p, stream);
+    if (epi == kEpiDequantGen) return launch_smallm_fq<kEpiDequantGen, 256>(Wq, Y, p, stream);
+    if (epi == kEpiDequantGenGelu) return launch_smallm_fq<kEpiDequantGenGelu, 256>(Wq, Y, p, stream);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -49,6 +49,9 @@ struct GemmParams {
   // tile's first operands have landed and again after its last tile's MMAs are
   // issued (the SM clock the kernel ran at), or null
   unsigned long long* clock_rec;
+  // weight-streaming form: weight rows per CTA tile (a multiple of 8, at most
+  // 128; filled by the launcher)
+  int tile_rows;
 };
 
 constexpr int kMaxFusedRows = 64;  // rows one CTA rotates and quantises per pass (fused form)
@@ -83,6 +86,14 @@ cudaError_t launch_gemm_i8(int epi, const int8_t* A, const int8_t* B, void* out,
 // M-blocks. p.ready holds num_m_blocks counters; p.epoch must differ from
 // every earlier call's epoch on the same workspace.
 cudaError_t launch_linear_fused(int g, const int8_t* Wq, void* Y, GemmParams p, cudaStream_t stream);
+
+// The fused weight-streaming form: whether it takes M tokens of K channels
+// (M <= 16, K <= 8192, M * K <= 16384: one quantisation pass), and its launch (Y = dequant(quant(X) Wq^T) in one
+// kernel; p.X holds the bf16 tokens, p.x_scale is not used; epi is one of the
+// dequantising epilogues).
+bool smallm_fused_shape(int64_t M, int64_t K);
+cudaError_t launch_linear_smallm_fused(int epi, int g, const int8_t* Wq, void* Y, GemmParams p,
+                                       cudaStream_t stream);
 
 // One CTA waits on a barrier that nothing completes, for at most timeout_ns,
 // then ORs 5 into *status.

@@ -113,7 +113,11 @@ __global__ void __maxnreg__(rq_maxnreg<G>()) rotate_quant_kernel(RotQuantParams 
     __threadfence();
     __syncthreads();
   }
-  griddep_launch_dependents();
+  // A kernel that follows may read a weight before it waits for this one (the
+  // GEMMs stream the weight from their start): the weight-quantising passes
+  // therefore let it launch only when the codes are written (at exit).
+  const bool late = MODE == kRqWeightQuant || p.late_trigger != 0;
+  if (!late) griddep_launch_dependents();
 
   // The producer (thread 0) keeps S-1 row blocks of this CTA in flight: block
   // it+S-1 goes out as soon as block it has landed, into the slot that block
@@ -282,6 +286,7 @@ __global__ void __maxnreg__(rq_maxnreg<G>()) rotate_quant_kernel(RotQuantParams 
       }
     }
   }
+  if (late) __threadfence();  // the codes are visible before the implicit trigger at exit
   if (timed_out && tid == 0) {
     if (p.status != nullptr) atomicOr(p.status, kRqTimeoutStatus);
     // let the copies already issued land before the shared memory goes away

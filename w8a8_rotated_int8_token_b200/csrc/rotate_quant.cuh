@@ -35,6 +35,7 @@ struct RotQuantParams {
   int zero_count;
   int* status;              // a timed-out wait ORs 5 into it (may be null)
   uint64_t timeout_ns;      // bound of every device-side wait
+  int late_trigger;         // 1: dependents launch only at exit (dst is a weight a GEMM reads early)
   int threads_per_row;      // filled by launch_rotate_quant
   int rows_per_cta;         // filled by launch_rotate_quant
 };
