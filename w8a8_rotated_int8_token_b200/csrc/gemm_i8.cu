@@ -1333,8 +1333,9 @@ __global__ void __launch_bounds__(QG != 0 ? NUM_THREADS + 32 * kSmallQuantWarps 
   // The weight stream does not depend on the previous kernel (see the pair
   // kernel): the weight loads of the first S stages go out before the wait,
   // the activation-code loads and the token scales after it. The fused form
-  // loads no tokens: its producer never waits, and it lets the next kernel
-  // launch as soon as the first stages and the panel prefetch are out.
+  // loads no tokens: its producer never waits. Either form lets the next
+  // kernel launch once every load of this CTA is out (letting it launch after
+  // the first stages instead measured 0.7 us slower per call at M = 1).
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1362,7 +1363,6 @@ __global__ void __launch_bounds__(QG != 0 ? NUM_THREADS + 32 * kSmallQuantWarps 
                                                                                              : kSmallPanelChunk));
         }
         prefetched = true;
-        if (FQ) griddep_launch_dependents();
       };
       auto load_x = [&](int st, int kb) {
 #pragma unroll
