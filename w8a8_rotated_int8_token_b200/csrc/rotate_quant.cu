@@ -63,11 +63,10 @@ __device__ __forceinline__ float2 widen2(uint32_t w) {
 template <int G>
 constexpr int rq_maxnreg() { return G == 256 ? CONVROT_RQ_MAXNREG : 128; }
 
-template <int G, int MODE, bool F16IN>
+template <int G, int MODE, bool F16IN, int S>
 __global__ void __maxnreg__(rq_maxnreg<G>()) rotate_quant_kernel(RotQuantParams p) {
   constexpr int LG = G / 64;
   constexpr int PIECE = G / 8;  // elements between consecutive pieces of a lane
-  constexpr int S = kRqStages;
   // S input slots of rows_per_cta x K bf16, each rounded up to whole 4 KB
   // warp regions (g = 256 reuses a warp's region for its exchange)
   extern __shared__ __align__(128) uint8_t stage_mem[];
@@ -311,11 +310,11 @@ bool rotquant_shape(int64_t K, int* threads_per_row, int* rows_per_cta) {
 
 namespace {
 
-template <int G, int MODE, bool F16IN>
+template <int G, int MODE, bool F16IN, int S>
 cudaError_t launch_typed(RotQuantParams p, cudaStream_t stream) {
-  void (*kern)(RotQuantParams) = rotate_quant_kernel<G, MODE, F16IN>;
+  void (*kern)(RotQuantParams) = rotate_quant_kernel<G, MODE, F16IN, S>;
   const int threads = (p.rows_per_cta * p.threads_per_row + 31) / 32 * 32;
-  const size_t smem = static_cast<size_t>(kRqStages) * rotquant_slot_bytes(p.rows_per_cta, p.K);
+  const size_t smem = static_cast<size_t>(S) * rotquant_slot_bytes(p.rows_per_cta, p.K);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -369,11 +368,17 @@ cudaError_t launch_typed(RotQuantParams p, cudaStream_t stream) {
 
 }  // namespace
 
+template <int G, bool F16IN, int S>
+cudaError_t launch_mode_s(int mode, RotQuantParams p, cudaStream_t stream) {
+  if (mode == kRqActivation) return launch_typed<G, kRqActivation, F16IN, S>(p, stream);
+  if (mode == kRqWeightAbsmax) return launch_typed<G, kRqWeightAbsmax, F16IN, S>(p, stream);
+  return launch_typed<G, kRqWeightQuant, F16IN, S>(p, stream);
+}
+
 template <int G, bool F16IN>
 cudaError_t launch_mode(int mode, RotQuantParams p, cudaStream_t stream) {
-  if (mode == kRqActivation) return launch_typed<G, kRqActivation, F16IN>(p, stream);
-  if (mode == kRqWeightAbsmax) return launch_typed<G, kRqWeightAbsmax, F16IN>(p, stream);
-  return launch_typed<G, kRqWeightQuant, F16IN>(p, stream);
+  if (p.K >= kRqDeepMinK) return launch_mode_s<G, F16IN, kRqStagesDeep>(mode, p, stream);
+  return launch_mode_s<G, F16IN, kRqStages>(mode, p, stream);
 }
 
 cudaError_t launch_rotate_quant(int g, int mode, RotQuantParams p, cudaStream_t stream) {

@@ -14,10 +14,12 @@ enum RotQuantMode : int {
 };
 
 constexpr int kMaxRowsPerCta = 256;
-#ifndef CONVROT_RQ_SLOTS
-#define CONVROT_RQ_SLOTS 2
-#endif
-constexpr int kRqStages = CONVROT_RQ_SLOTS;  // input slots per CTA: the block computed and the ones in flight
+// Input slots per CTA: the block computed and the ones in flight. Rows of
+// K >= kRqDeepMinK (one row per CTA) take a third slot: 35.7 against 37.5 us
+// on the 4608 x 12288 activation, while shorter rows lose resident CTAs to it.
+constexpr int kRqStages = 2;
+constexpr int kRqStagesDeep = 3;
+constexpr int64_t kRqDeepMinK = 8192;
 constexpr int kRqTimeoutStatus = 5;   // CONVROT_ERR_DEVICE_TIMEOUT
 constexpr int kRotQuantMaxThreads = 512;  // K/64 threads per row: K <= 32768
 
