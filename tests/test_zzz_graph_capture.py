@@ -64,7 +64,8 @@ def _warm_up(cr, X, Wq, sw, g, bias, Y, ws):
 
 
 @pytest.mark.parametrize("M,N,K,g", [(576, 1024, 3072, 256),   # CTA-pair GEMM, ragged last M tile
-                                     (16, 2048, 4096, 128)])   # weight-streaming GEMM
+                                     (16, 2048, 4096, 128),    # weight-streaming GEMM
+                                     (2, 12288, 4096, 128)])   # the one-kernel form (M * K <= 16384)
 def test_captured_linear_replays_on_new_inputs(cr, M, N, K, g):
     import torch
 
