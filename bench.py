@@ -73,7 +73,7 @@ PROBE_OPS_PER_ITER_PER_PAIR = 2.0 * 256 * 256 * 128  # four 256x256x32 MMAs
 GEMM_SOURCES = ["gemm_i8.cu", "gemm_i8.cuh", "ptx_sm100.cuh"]
 GEMM_TRAFFIC = {
     "dit_qkv_1024": {"bytes": 42623232 + 42524160,
-                     "sources_sha256": "970db59ad36ac0efd5bb104535b2cde4e7daf3ff54c611206cbdd1eb585b9031"},
+                     "sources_sha256": "4c38e302f0c1937c269bdc42ceec44889b1300d216684d7c326b53e8b97befb2"},
 }
 
 # Every layer shape of the workload table, timed after the headline.

@@ -1028,8 +1028,8 @@ constexpr int SM_BW = 128;  // weight rows the MMA covers (M = 128); a tile load
 // Its CTAs have kSmallQuantWarps more warps, and warps 2.. (the epilogue warps
 // and those) do the quantisation, redundantly in every CTA, in passes of
 // kSmallQuantThreads * 64 values. Used where one pass holds all tokens
-// (M * K <= 16384): each further pass costs about 2.5 us (the token loads
-// queue behind the weight stream already in flight), so at M = 16, K = 4096
+// (M * K <= 16384): each further pass costs about 2.5 us (a pass waits for
+// its token loads, issued while the weight stream is in flight), so at M = 16, K = 4096
 // the two-kernel form is faster (14.6 against 23.6 us); at M = 1 the fused
 // form saves the rotate kernel and two dependent-launch hops (13.3 against
 // 14.5 us).
