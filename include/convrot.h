@@ -44,9 +44,10 @@
  *     (where the entry point has one) and returns without faulting;
  *     convrot_read_device_status reports it. convrot_linear's status word is
  *     cleared by the first CTA of its first kernel as it starts, before the
- *     GEMM may launch (a memset instead costs 3.7 us per call on the
+ *     GEMM may launch (in the one-kernel form, by the first CTA once its
+ *     predecessor has finished; a memset instead costs 3.7 us per call on the
  *     weight-streaming layers); the clear is not ordered against a timeout
- *     reported by another CTA of that first kernel, which could be lost only
+ *     reported by another CTA of that kernel, which could be lost only
  *     if that CTA had waited 2 s before the first CTA started. The other entry
  *     points with a workspace clear it with a 4-byte memset before launching.
  *   - Entry points hold no state between calls (convrot_linear_noalloc's
